@@ -1,0 +1,201 @@
+// Device-side view of a CONF-KV cache and helpers shared by the kernels.
+//
+// Layout in HBM (one "segment" = the cache of one (layer, sequence, KV head)):
+//   segment id s = (layer * max_batch + seq) * kv_heads + kv_head
+//   cold region  (older tokens, a hole-free prefix [0, n_cold) of `cap` rows)
+//       INT8 codes k8/v8 [S][cap][D] + fp32 scales ks/vs [S][cap]   (INT8 on)
+//       or fp16 rows  kc/vc [S][cap][D]                              (INT8 off)
+//       int32 pos_c [S][cap], fp32 sc_c [S][cap] (EMA, or priority in fixed mode)
+//   FP16 window ring (INT8 on only): W slots per segment, slot = pos mod W,
+//       allocated with a stride Wst = W rounded up to 4 slots
+//       fp16 kr/vr [S][Wst][D], int32 pos_r [S][Wst] (-1 = empty), fp32 sc_r [S][Wst]
+//   int32 n_cold [S], next_pos [S]
+// Rows are 64 or 128 B (INT8) and 128 or 256 B (fp16), so every row starts on a
+// 16-byte boundary and moves as 128-bit words.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace confkv {
+
+// sticky device error codes (values match confkv_status)
+constexpr int kErrNonfinite = 4;
+constexpr int kErrDevice = 7;
+
+// cumulative counters (confkv_stats)
+enum Counter {
+  kCntAttnInt8 = 0,
+  kCntAttnFp16 = 1,
+  kCntEvictScanned = 2,
+  kCntMovedRows = 3,
+  kCntRequant = 4,
+  kNumCounters = 8
+};
+
+struct Cache {
+  int L, Bmax, Hkv, Hq, G, D, W, cap;
+  int Wst;            // ring allocation stride per segment: W rounded up to 4 slots
+  int cold_int8;
+  int8_t* k8;
+  int8_t* v8;
+  __half* kc;
+  __half* vc;
+  float* ks;
+  float* vs;
+  int32_t* pos_c;
+  float* sc_c;
+  __half* kr;
+  __half* vr;
+  int32_t* pos_r;
+  float* sc_r;
+  int32_t* n_cold;
+  int32_t* next_pos;
+  int32_t* err;
+  unsigned long long* counters;
+};
+
+struct Policy {
+  int mode;           // 0 confidence, 1 fixed budget
+  int n_low, n_high;
+  float tau;
+  float alpha, one_minus_alpha;   // (1 - alpha) rounded once to fp32
+  float beta, one_minus_beta;
+  int P;              // protect_last
+  int n_sink;
+  int fixed_budget;
+  int gate;           // 0 prose, 1 literal
+  int pyramidal;
+};
+
+// A call covers layers [l0, l0 + nl) and sequences [0, B) of every KV head.
+struct Range {
+  int l0, nl, B;
+  __host__ __device__ int items(int Hkv) const { return nl * B * Hkv; }
+};
+
+__device__ __forceinline__ int seg_of(const Cache& c, const Range& r, int item, int* l_out, int* b_out,
+                                      int* h_out) {
+  int per_layer = r.B * c.Hkv;
+  int l = r.l0 + item / per_layer;
+  int rem = item % per_layer;
+  int b = rem / c.Hkv;
+  int h = rem % c.Hkv;
+  *l_out = l;
+  *b_out = b;
+  *h_out = h;
+  return (l * c.Bmax + b) * c.Hkv + h;
+}
+
+__device__ __forceinline__ void set_error(int32_t* err, int code) { atomicCAS(err, 0, code); }
+
+// ---------------------------------------------------------------------------
+// Exact int8 -> fp32 conversion without the conversion unit: the biased byte
+// u = x + 128 is permuted into the low mantissa byte of 2^23 (bit pattern
+// 0x4B0000uu, value 2^23 + u), and one fp32 subtraction of 2^23 + 128 leaves
+// x exactly. Four bytes of one word give two float2 pairs; the subtraction is
+// a packed f32x2 add.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void i8x4_to_f2x2(uint32_t w, float2& lo, float2& hi) {
+  const uint32_t u = w ^ 0x80808080u;
+  const float2 bias = make_float2(-8388736.0f, -8388736.0f);
+  float2 a, b;
+  a.x = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7540));
+  a.y = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7541));
+  b.x = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7542));
+  b.y = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7543));
+  lo = __fadd2_rn(a, bias);
+  hi = __fadd2_rn(b, bias);
+}
+
+__device__ __forceinline__ float2 h2_to_f2(uint32_t w) {
+  return __half22float2(*reinterpret_cast<const __half2*>(&w));
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Order-preserving map of an fp32 score to uint32 (-0 is folded onto +0).
+__device__ __forceinline__ uint32_t ordered_bits(float f) {
+  uint32_t u = __float_as_uint(f + 0.0f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Ranking score of one token: fixed mode ranks by the stored priority;
+// confidence mode by fl(fl(alpha*ema) + fl((1-alpha)*rec)), rec = (pos+1)/(t+1),
+// every operation an IEEE fp32 operation with no contraction.
+__device__ __forceinline__ float rank_score(const Policy& p, float sc, int pos, int t) {
+  if (p.mode == 1) return sc;
+  const float rec = __fdiv_rn((float)(pos + 1), (float)(t + 1));
+  return __fadd_rn(__fmul_rn(p.alpha, sc), __fmul_rn(p.one_minus_alpha, rec));
+}
+
+__device__ __forceinline__ unsigned long long rank_key(const Policy& p, float sc, int pos, int t) {
+  return ((unsigned long long)ordered_bits(rank_score(p, sc, pos, t)) << 32) | (uint32_t)pos;
+}
+
+constexpr unsigned long long kNoKey = ~0ull;
+
+// ---------------------------------------------------------------------------
+// Symmetric per-row INT8 quantisation by one warp: amax = max |x| over the
+// row, scale = amax / 127 and code = clamp(rint_half_even(x / scale), +-127),
+// both divisions IEEE fp32; a zero row gets scale 0 and codes 0.
+// ---------------------------------------------------------------------------
+template <int D>
+__device__ __forceinline__ void warp_quantize_row(const __half* __restrict__ src, int8_t* __restrict__ dst,
+                                                  float* __restrict__ scale_out, int lane) {
+  constexpr int E = D / 32;  // 2 or 4 elements per lane
+  float x[E];
+  if constexpr (E == 4) {
+    const uint2 w = *reinterpret_cast<const uint2*>(src + lane * 4);
+    float2 a = h2_to_f2(w.x), b = h2_to_f2(w.y);
+    x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
+  } else {
+    const uint32_t w = *reinterpret_cast<const uint32_t*>(src + lane * 2);
+    float2 a = h2_to_f2(w);
+    x[0] = a.x; x[1] = a.y;
+  }
+  float amax = 0.0f;
+#pragma unroll
+  for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(x[e]));
+  amax = warp_max(amax);
+  const float scale = __fdiv_rn(amax, 127.0f);
+  uint32_t packed = 0;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    int q = 0;
+    if (scale != 0.0f) {
+      q = __float2int_rn(__fdiv_rn(x[e], scale));
+      q = max(-127, min(127, q));
+    }
+    packed |= ((uint32_t)(q & 0xff)) << (8 * e);
+  }
+  if constexpr (E == 4) {
+    *reinterpret_cast<uint32_t*>(dst + lane * 4) = packed;
+  } else {
+    *reinterpret_cast<uint16_t*>(dst + lane * 2) = (uint16_t)packed;
+  }
+  if (lane == 0) *scale_out = scale;
+}
+
+// Copy one fp16 row of D elements by one warp.
+template <int D>
+__device__ __forceinline__ void warp_copy_row_h(const __half* __restrict__ src, __half* __restrict__ dst, int lane) {
+  if constexpr (D == 128) {
+    reinterpret_cast<uint2*>(dst)[lane] = reinterpret_cast<const uint2*>(src)[lane];
+  } else {
+    reinterpret_cast<uint32_t*>(dst)[lane] = reinterpret_cast<const uint32_t*>(src)[lane];
+  }
+}
+
+}  // namespace confkv

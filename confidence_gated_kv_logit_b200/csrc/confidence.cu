@@ -1,0 +1,197 @@
+// Confidence of the next-token distribution and the per-layer budget
+// (CONF-KV post, decode-loop pseudo-code and method paragraphs; CONF-KV
+// abstract for the gate polarity and the pyramidal variant).
+//
+// One pass over each row of logits keeps, per thread, the running maximum m,
+// S = sum exp(l - m), T = sum exp(l - m) (l - m) and the two largest logits
+// counted with multiplicity. Partials are merged with
+//   m = max(m_a, m_b),  S = S_a e^(m_a-m) + S_b e^(m_b-m),
+//   T = e^(m_a-m) (T_a + (m_a-m) S_a) + e^(m_b-m) (T_b + (m_b-m) S_b),
+// which follows from the definitions. Then
+//   H = ln S - T/S,  max p = 1/S,  margin = l_(1) - l_(2)  (= log p_(1) - log p_(2)),
+//   c = 0.4 (1 - H / ln V) + 0.3 sigmoid(margin) + 0.3 / S.
+// A row is split over several CTAs; each writes its partial and takes a ticket
+// from an atomic counter, and the CTA that takes the last ticket merges the
+// partials and writes c and the budgets (no CTA waits on another).
+#include <math_constants.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace confkv {
+
+namespace {
+
+constexpr int NT = 256;
+
+__device__ __forceinline__ void top2_insert(float x, float& t1, float& t2) {
+  if (x > t1) {
+    t2 = t1;
+    t1 = x;
+  } else if (x > t2) {
+    t2 = x;
+  }
+}
+
+__device__ __forceinline__ void merge(ConfPartial& a, const ConfPartial& b) {
+  a.bad |= b.bad;
+  top2_insert(b.top1, a.top1, a.top2);
+  top2_insert(b.top2, a.top1, a.top2);
+  if (b.S == 0.0f) return;
+  if (a.S == 0.0f) {
+    a.m = b.m;
+    a.S = b.S;
+    a.T = b.T;
+    return;
+  }
+  const float m = fmaxf(a.m, b.m);
+  const float da = a.m - m, db = b.m - m;
+  const float fa = __expf(da), fb = __expf(db);
+  a.T = fa * fmaf(da, a.S, a.T) + fb * fmaf(db, b.S, b.T);
+  a.S = fa * a.S + fb * b.S;
+  a.m = m;
+}
+
+__device__ __forceinline__ ConfPartial shfl_partial(const ConfPartial& p, int o) {
+  ConfPartial q;
+  q.m = __shfl_xor_sync(0xffffffffu, p.m, o);
+  q.S = __shfl_xor_sync(0xffffffffu, p.S, o);
+  q.T = __shfl_xor_sync(0xffffffffu, p.T, o);
+  q.top1 = __shfl_xor_sync(0xffffffffu, p.top1, o);
+  q.top2 = __shfl_xor_sync(0xffffffffu, p.top2, o);
+  q.bad = __shfl_xor_sync(0xffffffffu, p.bad, o);
+  return q;
+}
+
+__global__ void __launch_bounds__(NT) confidence_kernel(ConfLaunch a, Policy pol) {
+  __shared__ ConfPartial wpart[NT / 32];
+  __shared__ int is_last;
+  const int row = blockIdx.y;
+  const int chunk = (a.V + a.cpr - 1) / a.cpr;
+  const int v0 = blockIdx.x * chunk;
+  const int v1 = min(a.V, v0 + chunk);
+  const float* lg = a.logits + (size_t)row * a.V;
+
+  ConfPartial p;
+  p.m = -CUDART_INF_F;
+  p.S = 0.0f;
+  p.T = 0.0f;
+  p.top1 = -CUDART_INF_F;
+  p.top2 = -CUDART_INF_F;
+  p.bad = 0;
+  constexpr int U = 8;
+  for (int base = v0; base < v1; base += NT * U) {
+    float x[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = base + u * NT + threadIdx.x;
+      x[u] = i < v1 ? __ldcs(lg + i) : -CUDART_INF_F;
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = base + u * NT + threadIdx.x;
+      if (i >= v1) continue;
+      const float xv = x[u];
+      if (!(fabsf(xv) <= 3.402823466e38f)) {   // NaN or +-Inf
+        p.bad = 1;
+        continue;
+      }
+      if (xv > p.m) {
+        if (p.S > 0.0f) {
+          const float d = p.m - xv;
+          const float f = __expf(d);
+          p.T = f * fmaf(d, p.S, p.T);
+          p.S = f * p.S;
+        }
+        p.m = xv;
+      }
+      const float d = xv - p.m;
+      const float ev = __expf(d);
+      p.S += ev;
+      p.T = fmaf(ev, d, p.T);
+      top2_insert(xv, p.top1, p.top2);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const ConfPartial q = shfl_partial(p, o);
+    merge(p, q);
+  }
+  if ((threadIdx.x & 31) == 0) wpart[threadIdx.x >> 5] = p;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    ConfPartial acc = wpart[0];
+    for (int w = 1; w < NT / 32; ++w) merge(acc, wpart[w]);
+    a.part[(size_t)row * a.cpr + blockIdx.x] = acc;
+    __threadfence();
+    const unsigned prev = atomicAdd(&a.tickets[row], 1u);
+    is_last = (prev == (unsigned)a.cpr - 1u);
+  }
+  __syncthreads();
+  if (!is_last || threadIdx.x != 0) return;
+
+  // last CTA of this row: merge every partial (read past L1) and finish
+  __threadfence();
+  ConfPartial acc;
+  {
+    const ConfPartial* pp = a.part + (size_t)row * a.cpr;
+    acc.m = __ldcg(&pp[0].m);
+    acc.S = __ldcg(&pp[0].S);
+    acc.T = __ldcg(&pp[0].T);
+    acc.top1 = __ldcg(&pp[0].top1);
+    acc.top2 = __ldcg(&pp[0].top2);
+    acc.bad = __ldcg(&pp[0].bad);
+    for (int k = 1; k < a.cpr; ++k) {
+      ConfPartial q;
+      q.m = __ldcg(&pp[k].m);
+      q.S = __ldcg(&pp[k].S);
+      q.T = __ldcg(&pp[k].T);
+      q.top1 = __ldcg(&pp[k].top1);
+      q.top2 = __ldcg(&pp[k].top2);
+      q.bad = __ldcg(&pp[k].bad);
+      merge(acc, q);
+    }
+  }
+  a.tickets[row] = 0u;   // ready for the next launch
+
+  float c;
+  int N;
+  const int larger = max(pol.n_low, pol.n_high);
+  if (acc.bad || !(acc.S > 0.0f)) {
+    c = CUDART_NAN_F;
+    N = larger;
+    set_error(a.err, kErrNonfinite);
+  } else {
+    const float H = logf(acc.S) - acc.T / acc.S;
+    const float norm_entropy = H / logf((float)a.V);
+    const float margin = acc.top1 - acc.top2;
+    const float sig = 1.0f / (1.0f + expf(-margin));
+    const float p_max = 1.0f / acc.S;
+    c = 0.4f * (1.0f - norm_entropy) + 0.3f * sig + 0.3f * p_max;
+    const bool confident = c >= pol.tau;
+    if (pol.gate == 0) N = confident ? pol.n_low : pol.n_high;
+    else N = confident ? pol.n_high : pol.n_low;
+  }
+  a.c_ws[row] = c;
+  if (a.c_out) a.c_out[row] = c;
+  for (int l = 0; l < a.L; ++l) {
+    int bl = N;
+    if (pol.pyramidal && a.L > 1) {
+      const long long L1 = a.L - 1;
+      bl = (int)(((long long)N * (4 * L1 - 3 * (long long)l)) / (2 * L1));
+    }
+    a.budget_ws[(size_t)row * a.L + l] = bl;
+    if (a.budget_out) a.budget_out[(size_t)row * a.L + l] = bl;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_confidence(const ConfLaunch& a, const Policy& pol, cudaStream_t st, long long* launches) {
+  dim3 grid(a.cpr, a.B);
+  confidence_kernel<<<grid, NT, 0, st>>>(a, pol);
+  ++*launches;
+  return cudaGetLastError();
+}
+
+}  // namespace confkv

@@ -1,0 +1,253 @@
+// Eviction, compaction and conversion of the token leaving the FP16 window,
+// one CTA per segment (CONF-KV post, decode-loop pseudo-code: evict only when
+// the layer holds more than its budget, rank by alpha*EMA + (1-alpha)*recency,
+// never evict the last P tokens, then convert tokens older than the window to
+// INT8; the post's implementation note names contiguous compaction as the hard
+// part. KVpop summary 2.1 / 2.4: sinks always kept, fixed budget, running
+// threshold over static priorities).
+//
+// Per segment:
+//   1. n = cold tokens + occupied window slots; budget_eff = max(budget, P + s)
+//      (fixed mode: B); e = n - budget_eff victims if positive.
+//   2. keys (ordered score bits << 32 | position) of unprotected tokens; the e
+//      smallest are the victims: argmin when e = 1 (the steady state: one new
+//      token per step), MSD radix select otherwise (budget drops, step 1).
+//   3. victims in the window ring free their slot; victims in the cold region
+//      are recorded in a bitmask and the region is compacted: hole-fill moves
+//      the survivors above the new end into the holes below it (bytes
+//      proportional to e), stable compaction shifts every survivor after the
+//      first hole down in order. Both leave the same logical content.
+//   4. the token that the next append would push out of the window
+//      (position t+1-W) is quantised into the end of the cold region.
+#include "common.cuh"
+#include "kernels.h"
+#include "select.cuh"
+
+namespace confkv {
+
+namespace {
+
+constexpr int NT = 256;
+
+template <int D, bool CI8>
+struct Rows {
+  static constexpr int ROWB = CI8 ? D : 2 * D;   // bytes of one K (or V) row in the cold region
+  static constexpr int VEC = ROWB / 16;           // uint4 per row
+};
+
+// Move cold row `src` to `dst` (both < cap) with `lanes` threads cooperating.
+template <int D, bool CI8>
+__device__ __forceinline__ void move_cold_row(const Cache& c, int s, int src, int dst, int part) {
+  using R = Rows<D, CI8>;
+  const size_t so = (size_t)s * c.cap + src, dO = (size_t)s * c.cap + dst;
+  const uint4* ks = reinterpret_cast<const uint4*>(CI8 ? (const void*)(c.k8 + so * D) : (const void*)(c.kc + so * D));
+  const uint4* vs = reinterpret_cast<const uint4*>(CI8 ? (const void*)(c.v8 + so * D) : (const void*)(c.vc + so * D));
+  uint4* kd = reinterpret_cast<uint4*>(CI8 ? (void*)(c.k8 + dO * D) : (void*)(c.kc + dO * D));
+  uint4* vd = reinterpret_cast<uint4*>(CI8 ? (void*)(c.v8 + dO * D) : (void*)(c.vc + dO * D));
+  // part in [0, 2*VEC): first VEC words of K, then of V; part 0 also moves the metadata
+  if (part < R::VEC) kd[part] = ks[part];
+  else vd[part - R::VEC] = vs[part - R::VEC];
+  if (part == 0) {
+    c.pos_c[dO] = c.pos_c[so];
+    c.sc_c[dO] = c.sc_c[so];
+    if (CI8) {
+      c.ks[dO] = c.ks[so];
+      c.vs[dO] = c.vs[so];
+    }
+  }
+}
+
+template <int D, bool CI8>
+__global__ void __launch_bounds__(NT) evict_kernel(Cache c, Policy pol, EvictLaunch a) {
+  using R = Rows<D, CI8>;
+  __shared__ SelectSmem<NT> sm;
+  __shared__ int list_h[NT];
+  __shared__ int list_m[NT];
+  __shared__ __align__(16) unsigned char stage[16384];
+  __shared__ int stage_meta[4][64];
+
+  const int item = blockIdx.x;
+  int l, b, h;
+  const int s = seg_of(c, a.r, item, &l, &b, &h);
+  const int t = c.next_pos[s] - 1;
+  const int n_cold = c.n_cold[s];
+  const int W = c.W;
+  const int32_t* pos_c = c.pos_c + (size_t)s * c.cap;
+  const float* sc_c = c.sc_c + (size_t)s * c.cap;
+  int32_t* pos_r = c.pos_r + (size_t)s * c.Wst;
+  const float* sc_r = c.sc_r + (size_t)s * c.Wst;
+
+  int ring_here = 0;
+  for (int slot = threadIdx.x; slot < W; slot += NT) ring_here += pos_r[slot] >= 0;
+  const int n_ring = block_sum_int<NT>(ring_here, sm);
+  const int n = n_cold + n_ring;
+  const int budget_eff = pol.mode == 1 ? pol.fixed_budget
+                                       : max(a.budget[(size_t)b * c.L + l], pol.P + pol.n_sink);
+  const int e = n - budget_eff;
+  int n_cold_new = n_cold;
+  int moved = 0;
+
+  if (e > 0 && t >= 0) {
+    auto key = [&](int i) -> unsigned long long {
+      int pos;
+      float sc;
+      if (i < n_cold) {
+        pos = pos_c[i];
+        sc = sc_c[i];
+      } else {
+        pos = pos_r[i - n_cold];
+        if (pos < 0) return kNoKey;
+        sc = sc_r[i - n_cold];
+      }
+      if (t - pos < pol.P || pos < pol.n_sink) return kNoKey;
+      return rank_key(pol, sc, pos, t);
+    };
+    const int span = n_cold + W;
+    const SelectResult sel = (e == 1) ? block_argmin<NT>(key, span, sm) : block_select_smallest<NT>(key, span, e, sm);
+
+    // victim bitmask of the cold region, and count
+    uint32_t* vm = a.vmask + (size_t)s * a.mask_words;
+    const int words = (n_cold + 31) >> 5;
+    int ecold_here = 0;
+    for (int w = threadIdx.x; w < words; w += NT) {
+      uint32_t bits = 0;
+      for (int j = 0; j < 32; ++j) {
+        const int i = w * 32 + j;
+        if (i < n_cold && is_selected(key(i), sel)) bits |= 1u << j;
+      }
+      vm[w] = bits;
+      ecold_here += __popc(bits);
+    }
+    // window victims free their slot (each thread reads and writes only its own slots)
+    for (int slot = threadIdx.x; slot < W; slot += NT)
+      if (is_selected(key(n_cold + slot), sel)) pos_r[slot] = -1;
+    const int e_cold = block_sum_int<NT>(ecold_here, sm);   // includes a block barrier: vm is visible
+    const int n_keep = n_cold - e_cold;
+    auto victim = [&](int i) -> bool { return (vm[i >> 5] >> (i & 31)) & 1u; };
+
+    if (e_cold == 0) {
+      // every victim was in the window ring: the cold region is unchanged
+    } else if (!a.stable) {
+      // hole-fill: pair the k-th hole below n_keep with the k-th survivor above it
+      int hcur = 0, mcur = n_keep;
+      while (true) {
+        const int nh = block_collect<NT, NT>([&](int i) { return victim(i); }, &hcur, n_keep, list_h, sm);
+        const int nm = block_collect<NT, NT>([&](int i) { return !victim(i); }, &mcur, n_cold, list_m, sm);
+        const int np = min(nh, nm);
+        if (np == 0) break;
+        for (int w = threadIdx.x; w < np * 2 * R::VEC; w += NT) {
+          const int p = w / (2 * R::VEC);
+          move_cold_row<D, CI8>(c, s, list_m[p], list_h[p], w - p * 2 * R::VEC);
+        }
+        moved += np;
+        __syncthreads();
+      }
+    } else {
+      // stable: from the first hole on, every survivor moves down by the number
+      // of victims before it, in chunks staged through shared memory
+      constexpr int CH = 16384 / (2 * R::ROWB) < 64 ? 16384 / (2 * R::ROWB) : 64;
+      int dst_base = 0;
+      for (int base = 0; base < n_cold; base += CH) {
+        const int i = base + (int)threadIdx.x;
+        const bool live = threadIdx.x < CH && i < n_cold && !victim(i);
+        int total;
+        const int r = block_scan_flag<NT>(live, sm, &total);
+        // stage this chunk's survivors (rows and metadata), then write them back
+        for (int w = threadIdx.x; w < CH * 2 * R::VEC; w += NT) {
+          const int rr = w / (2 * R::VEC), part = w - rr * 2 * R::VEC;
+          const int src = base + rr;
+          if (src < n_cold) {
+            const size_t so = (size_t)s * c.cap + src;
+            const uint4* kv = part < R::VEC
+                                  ? reinterpret_cast<const uint4*>(CI8 ? (const void*)(c.k8 + so * D) : (const void*)(c.kc + so * D)) + part
+                                  : reinterpret_cast<const uint4*>(CI8 ? (const void*)(c.v8 + so * D) : (const void*)(c.vc + so * D)) + (part - R::VEC);
+            reinterpret_cast<uint4*>(stage)[w] = *kv;
+          }
+        }
+        if (live) {
+          const size_t so = (size_t)s * c.cap + i;
+          stage_meta[0][threadIdx.x] = pos_c[i];
+          stage_meta[1][threadIdx.x] = __float_as_int(sc_c[i]);
+          stage_meta[2][threadIdx.x] = CI8 ? __float_as_int(c.ks[so]) : 0;
+          stage_meta[3][threadIdx.x] = CI8 ? __float_as_int(c.vs[so]) : 0;
+          list_m[threadIdx.x] = dst_base + r;
+        }
+        if (threadIdx.x < CH) list_h[threadIdx.x] = live ? 1 : 0;
+        __syncthreads();
+        for (int w = threadIdx.x; w < CH * 2 * R::VEC; w += NT) {
+          const int rr = w / (2 * R::VEC), part = w - rr * 2 * R::VEC;
+          if (base + rr < n_cold && list_h[rr]) {
+            const size_t dO = (size_t)s * c.cap + list_m[rr];
+            uint4* kv = part < R::VEC
+                            ? reinterpret_cast<uint4*>(CI8 ? (void*)(c.k8 + dO * D) : (void*)(c.kc + dO * D)) + part
+                            : reinterpret_cast<uint4*>(CI8 ? (void*)(c.v8 + dO * D) : (void*)(c.vc + dO * D)) + (part - R::VEC);
+            *kv = reinterpret_cast<const uint4*>(stage)[w];
+            if (part == 0) {
+              c.pos_c[dO] = stage_meta[0][rr];
+              c.sc_c[dO] = __int_as_float(stage_meta[1][rr]);
+              if (CI8) {
+                c.ks[dO] = __int_as_float(stage_meta[2][rr]);
+                c.vs[dO] = __int_as_float(stage_meta[3][rr]);
+              }
+            }
+          }
+        }
+        if (threadIdx.x < CH && live && list_m[threadIdx.x] != i) ++moved;
+        dst_base += total;
+        __syncthreads();
+      }
+      moved = block_sum_int<NT>(moved, sm);
+    }
+    n_cold_new = n_keep;
+  }
+
+  // the token that the next append would push out of the window becomes INT8
+  __syncthreads();
+  const int leaving = t + 1 - W;
+  if (W > 0 && leaving >= 0 && threadIdx.x < 32) {
+    const int slot = (t + 1) % W;
+    const size_t rs = (size_t)s * c.Wst + slot;
+    if (c.pos_r[rs] == leaving) {
+      const int idx = n_cold_new;
+      if (idx >= c.cap) {
+        if (threadIdx.x == 0) set_error(c.err, kErrDevice);
+      } else {
+        const size_t cs = (size_t)s * c.cap + idx;
+        warp_quantize_row<D>(c.kr + rs * D, c.k8 + cs * D, c.ks + cs, threadIdx.x);
+        warp_quantize_row<D>(c.vr + rs * D, c.v8 + cs * D, c.vs + cs, threadIdx.x);
+        __syncwarp();
+        if (threadIdx.x == 0) {
+          c.pos_c[cs] = leaving;
+          c.sc_c[cs] = c.sc_r[rs];
+          c.pos_r[rs] = -1;
+          atomicAdd(&c.counters[kCntRequant], 1ull);
+        }
+        n_cold_new = idx + 1;
+      }
+    }
+  }
+  if (threadIdx.x == 0) {
+    c.n_cold[s] = n_cold_new;
+    atomicAdd(&c.counters[kCntEvictScanned], (unsigned long long)n);
+    if (moved > 0) atomicAdd(&c.counters[kCntMovedRows], (unsigned long long)moved);
+  }
+}
+
+template <int D, bool CI8>
+cudaError_t run(const Cache& c, const Policy& pol, const EvictLaunch& a, cudaStream_t st, long long* launches) {
+  const int items = a.r.items(c.Hkv);
+  evict_kernel<D, CI8><<<items, NT, 0, st>>>(c, pol, a);
+  ++*launches;
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_evict_compact(const Cache& c, const Policy& pol, const EvictLaunch& a, cudaStream_t st,
+                                 long long* launches) {
+  if (a.r.items(c.Hkv) == 0) return cudaSuccess;
+  if (c.D == 128) return c.cold_int8 ? run<128, true>(c, pol, a, st, launches) : run<128, false>(c, pol, a, st, launches);
+  return c.cold_int8 ? run<64, true>(c, pol, a, st, launches) : run<64, false>(c, pol, a, st, launches);
+}
+
+}  // namespace confkv

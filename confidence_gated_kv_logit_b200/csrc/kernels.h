@@ -1,0 +1,75 @@
+// Host-side launch interface of the CONF-KV kernels (internal to libconfkv).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace confkv {
+
+struct ConfPartial {
+  float m, S, T, top1, top2;
+  int bad;
+};
+
+// K1: confidence reduction over logits [B][V] -> c[B], budget[B][L].
+struct ConfLaunch {
+  const float* logits;
+  int B, V, L;
+  ConfPartial* part;      // [B][cpr]
+  unsigned* tickets;      // [B], zero between launches
+  int cpr;                // CTAs per row
+  float* c_ws;            // [B]
+  int32_t* budget_ws;     // [B][L]
+  float* c_out;           // optional
+  int32_t* budget_out;    // optional
+  int32_t* err;
+};
+cudaError_t launch_confidence(const ConfLaunch& a, const Policy& pol, cudaStream_t st, long long* launches);
+
+// K2: prefill ingest.
+struct PrefillLaunch {
+  Range r;
+  const int32_t* lens;    // device [B]
+  int t_stride;
+  const __half* k;        // [nl][B][Hkv][t_stride][D]
+  const __half* v;
+  const float* prio;      // [nl][B][Hkv][t_stride] (fixed mode) or null
+  int32_t* keep_list;     // fixed mode: [items][fixed_budget] positions kept (ascending)
+  int32_t* keep_count;    // fixed mode: [items]
+};
+cudaError_t launch_prefill(const Cache& c, const Policy& pol, const PrefillLaunch& a, cudaStream_t st,
+                           long long* launches);
+
+// K3 + K3c + EMA: decode attention.
+struct AttnLaunch {
+  Range r;
+  const __half* q;        // [nl][B][Hq][D]
+  const __half* k_new;    // [nl][B][Hkv][D]
+  const __half* v_new;
+  const float* prio_new;  // [nl][B][Hkv] (fixed mode) or null
+  float* out;             // [nl][B][Hq][D]
+  float* lse_out;         // [nl][B][Hq] or null
+  float* lse_ws;          // [S][G]
+  float* scores;          // [S][G][score_stride]
+  int score_stride;
+  float* part;            // [units][G][D+2]
+  int part_units;         // capacity of part in (item, split) units
+  int max_cold_tokens;    // host upper bound of n_cold over the call's segments
+  int num_sms;
+};
+cudaError_t launch_decode_attn(const Cache& c, const Policy& pol, const AttnLaunch& a, cudaStream_t st,
+                               long long* launches);
+
+// K4 + K5 + K6: select, compaction, conversion of the token leaving the window.
+struct EvictLaunch {
+  Range r;
+  const int32_t* budget;  // [Bmax][L]
+  uint32_t* vmask;        // [S][mask_words] victim bitmask scratch
+  int mask_words;
+  int stable;             // 1: order-preserving compaction
+};
+cudaError_t launch_evict_compact(const Cache& c, const Policy& pol, const EvictLaunch& a, cudaStream_t st,
+                                 long long* launches);
+
+}  // namespace confkv

@@ -1,0 +1,174 @@
+// Block-wide building blocks for the segmented top-k select (one CTA per
+// segment): flag scans, ordered collection, argmin and MSD radix select on
+// 64-bit keys (score bits, position) that are unique within a segment.
+#pragma once
+
+#include "common.cuh"
+
+namespace confkv {
+
+template <int NT>
+struct SelectSmem {
+  unsigned hist[256];
+  unsigned long long prefix, mask;
+  int rem, done;
+  int warp_tot[NT / 32];
+  unsigned long long wmin[NT / 32];
+  int next;
+  int misc[4];
+};
+
+// Exclusive prefix of a 0/1 flag over the block; *total receives the count.
+template <int NT>
+__device__ __forceinline__ int block_scan_flag(bool f, SelectSmem<NT>& sm, int* total) {
+  const unsigned bal = __ballot_sync(0xffffffffu, f);
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  if (lane == 0) sm.warp_tot[w] = __popc(bal);
+  __syncthreads();
+  int off = 0, tot = 0;
+#pragma unroll
+  for (int i = 0; i < NT / 32; ++i) {
+    const int v = sm.warp_tot[i];
+    off += (i < w) ? v : 0;
+    tot += v;
+  }
+  __syncthreads();
+  *total = tot;
+  return off + __popc(bal & ((1u << lane) - 1u));
+}
+
+template <int NT>
+__device__ __forceinline__ int block_sum_int(int v, SelectSmem<NT>& sm) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if ((threadIdx.x & 31) == 0) sm.warp_tot[threadIdx.x >> 5] = v;
+  __syncthreads();
+  int tot = 0;
+#pragma unroll
+  for (int i = 0; i < NT / 32; ++i) tot += sm.warp_tot[i];
+  __syncthreads();
+  return tot;
+}
+
+// Collect, in increasing order, up to CAP indices i in [*cur, end) with
+// pred(i), into list[]. Advances *cur past the last collected index (or to
+// end). Every thread returns the same count and cursor.
+template <int NT, int CAP, class Pred>
+__device__ int block_collect(Pred pred, int* cur, int end, int* list, SelectSmem<NT>& sm) {
+  int count = 0;
+  int c0 = *cur;
+  while (count < CAP && c0 < end) {
+    const int i = c0 + threadIdx.x;
+    const bool f = i < end && pred(i);
+    int total;
+    const int r = count + block_scan_flag<NT>(f, sm, &total);
+    if (f && r < CAP) list[r] = i;
+    if (count + total > CAP) {
+      if (f && r == CAP - 1) sm.next = i + 1;
+      __syncthreads();
+      c0 = sm.next;
+      count = CAP;
+      __syncthreads();
+      break;
+    }
+    count += total;
+    c0 += NT;
+  }
+  *cur = min(c0, end);
+  return count;
+}
+
+struct SelectResult {
+  unsigned long long prefix, mask;   // selected: key != kNoKey && (key & mask) <= prefix
+};
+
+// Smallest key among kf(0..n-1) (absent keys are kNoKey).
+template <int NT, class KeyFn>
+__device__ SelectResult block_argmin(KeyFn kf, int n, SelectSmem<NT>& sm) {
+  unsigned long long best = kNoKey;
+  for (int i = threadIdx.x; i < n; i += NT) {
+    const unsigned long long k = kf(i);
+    best = k < best ? k : best;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
+    best = other < best ? other : best;
+  }
+  if ((threadIdx.x & 31) == 0) sm.wmin[threadIdx.x >> 5] = best;
+  __syncthreads();
+  unsigned long long m = kNoKey;
+#pragma unroll
+  for (int i = 0; i < NT / 32; ++i) m = sm.wmin[i] < m ? sm.wmin[i] : m;
+  __syncthreads();
+  return SelectResult{m, ~0ull};
+}
+
+// The k smallest keys (1 <= k <= number of present keys), by MSD radix select
+// with 8-bit digits. Stops early once the bucket holding the k-th key is
+// entirely selected.
+template <int NT, class KeyFn>
+__device__ SelectResult block_select_smallest(KeyFn kf, int n, int k, SelectSmem<NT>& sm) {
+  if (threadIdx.x == 0) {
+    sm.prefix = 0;
+    sm.mask = 0;
+    sm.rem = k;
+    sm.done = 0;
+  }
+  __syncthreads();
+  for (int shift = 56; shift >= 0; shift -= 8) {
+    for (int i = threadIdx.x; i < 256; i += NT) sm.hist[i] = 0;
+    __syncthreads();
+    const unsigned long long prefix = sm.prefix, mask = sm.mask;
+    for (int i = threadIdx.x; i < n; i += NT) {
+      const unsigned long long key = kf(i);
+      if (key != kNoKey && (key & mask) == prefix) atomicAdd(&sm.hist[(key >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      const int lane = threadIdx.x;
+      unsigned cnt[8];
+      unsigned tot = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        cnt[j] = sm.hist[lane * 8 + j];
+        tot += cnt[j];
+      }
+      unsigned incl = tot;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      const unsigned excl = incl - tot;
+      const unsigned rem = (unsigned)sm.rem;
+      __syncwarp();
+      if (excl < rem && rem <= incl) {
+        unsigned below = excl;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (below + cnt[j] >= rem) {
+            const unsigned nrem = rem - below;
+            sm.prefix = prefix | ((unsigned long long)(lane * 8 + j) << shift);
+            sm.mask = mask | (0xffull << shift);
+            sm.rem = (int)nrem;
+            sm.done = (cnt[j] == nrem) ? 1 : 0;
+            break;
+          }
+          below += cnt[j];
+        }
+      }
+    }
+    __syncthreads();
+    if (sm.done) break;
+  }
+  SelectResult r{sm.prefix, sm.mask};
+  __syncthreads();
+  return r;
+}
+
+__device__ __forceinline__ bool is_selected(unsigned long long key, const SelectResult& r) {
+  return key != kNoKey && (key & r.mask) <= r.prefix;
+}
+
+}  // namespace confkv

@@ -181,9 +181,16 @@ def prefill_segment(k16, v16, prio, params: Params) -> Segment:
 def decode_attn_segment(seg: Segment, q, k_new, v_new, prio_new, params: Params):
     """Append the new token, attend with the G query heads, update the EMA.
 
+    While attention runs at step t a token is FP16 exactly when t - pos < W;
+    normally eviction of the previous step has already converted the token
+    leaving the window, and this only acts when a step skipped eviction.
     Returns (out [G, D], lse [G], w [G, n]) in fp64.
     """
     seg.append(k_new, v_new, prio_new if params.mode == "fixed" else None)
+    if params.int8:
+        t = seg.next_pos - 1
+        for i in np.flatnonzero(seg.is_fp16 & (t - seg.pos >= params.fp16_window)):
+            seg.to_int8(i)
     k_hat, v_hat = seg.rows_hat()
     out, lse, w = attend(q, k_hat, v_hat)
     if params.mode != "fixed":

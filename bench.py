@@ -1,0 +1,416 @@
+#!/usr/bin/env python
+"""Decode-step benchmark of the CONF-KV B200 library.
+
+Workload (one "step" = one decode step of the whole hot path for every layer,
+sequence and KV head): Llama-3-8B shape, 32 layers, 32 query / 8 KV heads,
+head_dim 128, batch 16, every sequence prefilled to 32768 tokens (fp16
+N(0,1), 1% of keys x4), vocab 128256 with bursty logits, N_low 1024 /
+N_high 2048, P 128, W 256, tau 0.6, alpha 0.5, EMA decay 0.9. A step is
+  decode_attn(all layers) -> confidence(logits) -> evict_compact(all layers).
+The first step after prefill evicts ~31K tokens per segment and is timed on
+its own ("step1_ms"); the timed region covers steady-state steps after it.
+
+Prints one JSON line. `--impl reference` times the CPU oracle on the same
+metric instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode tok/s at Llama-8B shape (attn+evict)"
+FULL = dict(L=32, Hq=32, Hkv=8, D=128, B=16, T=32768, V=128256, n_low=1024, n_high=2048, P=128, W=256,
+            tau=0.6, alpha=0.5, beta=0.9)
+POOL = 48   # distinct pre-generated step inputs, reused cyclically (1.4 GB/step working set >> L2)
+
+
+def args_parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--layers", type=int, default=None, help="smaller case for profiling captures")
+    ap.add_argument("--prefill", type=int, default=None, help="smaller case for profiling captures")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    return ap.parse_args()
+
+
+def workload(args):
+    w = dict(FULL)
+    if args.layers:
+        w["L"] = args.layers
+    if args.prefill:
+        w["T"] = args.prefill
+    return w
+
+
+def workload_name(w):
+    name = (f"llama3-8b-shape decode: {w['L']} layers, {w['Hq']}q/{w['Hkv']}kv heads, D{w['D']}, batch {w['B']}, "
+            f"prefill {w['T']}, vocab {w['V']}, N {w['n_low']}/{w['n_high']}, P{w['P']}, W{w['W']}, "
+            f"steady-state steps after the bulk first step")
+    return name if (w["L"], w["T"]) == (FULL["L"], FULL["T"]) else "reduced case (profiling): " + name
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def attn_traffic(w):
+    """dram bytes per attention launch from the committed ncu summary, if the
+    kernel source has not changed since it was taken (else None)."""
+    src = os.path.join(ROOT, "confidence_gated_kv_logit_b200", "csrc", "attention.cu")
+    path = os.path.join(ROOT, "profiles", "attention_llama8b_traffic.txt")
+    try:
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        kv = {}
+        for line in open(path):
+            if "=" in line and not line.startswith("#"):
+                k, v = line.strip().split("=", 1)
+                kv[k.strip()] = v.strip()
+        if kv.get("attention_cu_sha256") != sha:
+            return None
+        # scaled from the captured case by segments processed per launch
+        per_seg = float(kv["dram_bytes_per_segment"])
+        return per_seg * w["L"] * w["B"] * w["Hkv"]
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 8]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if "Active" in r[5 + i] and "Not" not in r[5 + i]})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": float(rows[0][2]) if rows[0][2].strip().replace(".", "").isdigit() else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def physical_gpu_index(local_rank: int) -> int:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    ids = [x.strip() for x in vis.split(",") if x.strip()]
+    if ids and all(x.isdigit() for x in ids) and local_rank < len(ids):
+        return int(ids[local_rank])
+    return local_rank
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle legs (cpu_baseline and --impl reference)
+# ---------------------------------------------------------------------------
+
+def oracle_sample(w, seconds: float, steps_hint: int = 1):
+    """Time the oracle on a bounded sample of the workload; returns tok/s for
+    the whole workload extrapolated from per-segment-step and per-row times."""
+    import numpy as np
+    import torch
+    from threadpoolctl import threadpool_info
+
+    from confidence_gated_kv_logit_b200 import synth
+    from oracle.confidence import confidence
+    from oracle.segment import (Params, decode_attn_segment, evict_compact_segment, prefill_segment)
+
+    p = Params(n_low=w["n_low"], n_high=w["n_high"], tau=w["tau"], alpha=w["alpha"], ema_decay=w["beta"],
+               protect_last=w["P"], fp16_window=w["W"])
+    G = w["Hq"] // w["Hkv"]
+    g = synth.generator(1234)
+    nseg = 2
+    segs = []
+    for h in range(nseg):
+        k, v = synth.prefill_kv(1, 1, w["T"], w["D"], g)
+        segs.append(prefill_segment(k[0, 0].numpy(), v[0, 0].numpy(), None, p))
+    # bulk first step (not timed)
+    for i in range(nseg):
+        q, kn, vn = synth.step_qkv((1,), G, 1, w["D"], g)
+        decode_attn_segment(segs[i], q[0].numpy(), kn[0, 0].numpy(), vn[0, 0].numpy(), None, p)
+        segs[i] = evict_compact_segment(segs[i], w["n_low"], p)
+    # steady segment-steps, timed
+    t_seg, n_seg = 0.0, 0
+    t_row, n_row = 0.0, 0
+    deadline = time.perf_counter() + seconds
+    while (time.perf_counter() < deadline or n_seg < 2 * steps_hint) and n_seg < 10000:
+        for i in range(nseg):
+            q, kn, vn = synth.step_qkv((1,), G, 1, w["D"], g)
+            qn, knn, vnn = q[0].numpy(), kn[0, 0].numpy(), vn[0, 0].numpy()
+            t0 = time.perf_counter()
+            decode_attn_segment(segs[i], qn, knn, vnn, None, p)
+            segs[i] = evict_compact_segment(segs[i], w["n_low"], p)
+            t_seg += time.perf_counter() - t0
+            n_seg += 1
+        if n_row < max(2, n_seg // 8):
+            logits = synth.bursty_logits(1, w["V"], g).numpy()[0]
+            t0 = time.perf_counter()
+            confidence(logits)
+            t_row += time.perf_counter() - t0
+            n_row += 1
+    per_seg = t_seg / n_seg
+    per_row = t_row / max(1, n_row)
+    S = w["L"] * w["B"] * w["Hkv"]
+    step_s = per_seg * S + per_row * w["B"]
+    threads = max([x.get("num_threads", 1) for x in threadpool_info()] + [1])
+    return {
+        "value": w["B"] / step_s, "unit": "tok/s", "cores": threads, "kind": "oracle",
+        "sample": (f"{n_seg} steady segment-steps over {nseg} of {S} segments (layer 0, seq 0) after a "
+                   f"{w['T']}-token prefill and the bulk first step (budget N_low each step), plus {n_row} "
+                   f"confidence rows of vocab {w['V']}; step time = per-segment-step x {S} + per-row x {w['B']}"),
+        "ms_per_step": step_s * 1e3,
+    }
+
+
+def run_reference(args):
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    w = workload(args)
+    budget = max(1.0, 150.0 / max(1, args.steps + args.warmup))
+    r = oracle_sample(w, seconds=min(args.cpu_seconds * 3, budget * (args.steps + args.warmup)),
+                      steps_hint=args.steps)
+    line = {"metric": METRIC, "value": r["value"], "unit": "tok/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": r["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": workload_name(w), "global_batch": w["B"], "seq_len": w["T"],
+                       "parallelism": "cpu oracle, rank 0"},
+            "cpu_baseline": {k: r[k] for k in ("value", "unit", "cores", "kind", "sample")},
+            "e2e": {"value": r["value"], "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# GPU leg
+# ---------------------------------------------------------------------------
+
+def main():
+    args = args_parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import torch
+    import torch.distributed as dist
+
+    from __graft_entry__ import build
+    from confidence_gated_kv_logit_b200 import ALL_LAYERS, ConfKV, synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    if rank == 0:
+        build()
+    if world > 1:
+        dist.barrier()
+    from confidence_gated_kv_logit_b200 import binding
+    binding.load_library()
+
+    w = workload(args)
+    L, Hq, Hkv, D, B, T, V = (w[k] for k in ("L", "Hq", "Hkv", "D", "B", "T", "V"))
+    G = Hq // Hkv
+    h = ConfKV(L, Hkv, Hq, D, max_batch=B, max_prefill=T, n_low=w["n_low"], n_high=w["n_high"], tau=w["tau"],
+               alpha=w["alpha"], ema_decay=w["beta"], protect_last=w["P"], fp16_window=w["W"])
+    gen = synth.generator(1000 + rank, dev)
+    for l in range(L):
+        k, v = synth.prefill_kv(B, Hkv, T, D, gen, dev)
+        h.prefill(k, v, [T] * B, layer=l)
+        del k, v
+    torch.cuda.synchronize()
+    pool = []
+    for _ in range(POOL):
+        q, kn, vn = synth.step_qkv((L, B), Hq, Hkv, D, gen, dev)
+        pool.append((q, kn, vn, synth.bursty_logits(B, V, gen, dev)))
+    out = torch.empty((L, B, Hq, D), device=dev)
+    c_out = torch.empty(B, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        q, kn, vn, lg = pool[i % POOL]
+        h.decode_attn(q, kn, vn, out, ALL_LAYERS)
+        h.confidence(lg, c_out)
+        h.evict_compact(ALL_LAYERS)
+
+    # bulk first step, on its own
+    s0 = h.query()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    step(0)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    step1_ms = e0.elapsed_time(e1)
+    s1 = h.query()
+    for i in range(1, 1 + args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+
+    # ---- timed region ----
+    h.profile(True)
+    h.profile_read(reset=True)
+    sa = h.query()
+    sampler = ClockSampler(physical_gpu_index(local))
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(args.steps):
+        step(1 + args.warmup + i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    elapsed_ms = e0.elapsed_time(e1)
+    prof = h.profile_read(reset=True)
+    h.profile(False)
+    sb = h.query()
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    K = args.steps
+    value = world * B * K / (elapsed_ms / 1e3)
+
+    # ---- roofline of the dominant kernel (attention) ----
+    n8 = sb["attn_tokens_int8"] - sa["attn_tokens_int8"]
+    n16 = sb["attn_tokens_fp16"] - sa["attn_tokens_fp16"]
+    launches = max(1, prof["attention"]["launches"])
+    qo = L * B * Hq * (2 * D + 4 * D + 4)                       # q read, out + lse written
+    attn_bytes = (n8 * (2 * D + 8 + 4 * G) + n16 * (4 * D + 4 * G)) / launches + qo
+    attn_ms = prof["attention"]["ms"] / launches
+    peak, peak_kind = peaks()
+    achieved = attn_bytes / (attn_ms * 1e-3) / 1e9
+    traffic = attn_traffic(w)
+    # whole-step algorithmic bytes: attention + EMA pass + confidence + eviction scan/moves
+    ema_bytes = (n8 + n16) * (4 * G + 8) / K
+    evict_bytes = (sb["evict_tokens"] - sa["evict_tokens"]) * 8 / K
+    move_bytes = (sb["moved_rows"] - sa["moved_rows"]) * 2 * (2 * D + 16) / K
+    req_bytes = (sb["requant_rows"] - sa["requant_rows"]) * (6 * D + 8) / K
+    conf_bytes = B * V * 4
+    step_bytes = attn_bytes + ema_bytes + evict_bytes + move_bytes + req_bytes + conf_bytes
+    ms_step = elapsed_ms / K
+    kernel_ms = {k: round(v["ms"] / K, 4) for k, v in prof.items() if v["launches"]}
+
+    # ---- end to end through the public API with pinned host buffers ----
+    hpool = []
+    for i in range(8):
+        q, kn, vn, lg = pool[i]
+        hpool.append(tuple(x.cpu().pin_memory() for x in (q, kn, vn, lg)))
+    dq, dk, dv, dl = (torch.empty_like(x) for x in pool[0])
+    host_out = torch.empty((L, B, Hq, D), pin_memory=True)
+    host_c = torch.empty(B, pin_memory=True)
+    h2d = sum(x.numel() * x.element_size() for x in hpool[0])
+    d2h = host_out.numel() * 4 + host_c.numel() * 4
+    E = args.e2e_steps
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0.record(stream)
+    for i in range(E):
+        hq, hk, hv, hl = hpool[i % len(hpool)]
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        dl.copy_(hl, non_blocking=True)
+        h.decode_attn(dq, dk, dv, out, ALL_LAYERS)
+        h.confidence(dl, c_out)
+        h.evict_compact(ALL_LAYERS)
+        host_out.copy_(out, non_blocking=True)
+        host_c.copy_(c_out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * B * E / (e2e_ms / 1e3)
+
+    stats = h.query()
+    full_cache = L * B * Hkv * (T + 1 + args.warmup + K + E) * 4 * D
+    sw512 = L * B * Hkv * 512 * 4 * D
+    assert h.last_error() == 0, "device error word set"
+
+    if rank == 0:
+        cpu = None
+        if not args.no_cpu_baseline and world == 1:
+            r = oracle_sample(w, seconds=args.cpu_seconds)
+            cpu = {k: r[k] for k in ("value", "unit", "cores", "kind", "sample")}
+        line = {
+            "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+            "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic",
+            "config": {"workload": workload_name(w), "global_batch": B * world, "seq_len": T,
+                       "parallelism": f"replicas x{world} (independent sequences, no collective)",
+                       "l2": "no flush: the per-step working set (~1.4 GB of KV + inputs) exceeds the 126 MB L2",
+                       "input_pool": f"{POOL} pre-generated step inputs reused cyclically"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,
+                         "kernel": "attn_kernel", "algorithmic_bytes_per_launch": attn_bytes,
+                         "ms_per_launch": attn_ms},
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "tok/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "steps": E},
+            "gpu_launches": sb["kernel_launches"] - sa["kernel_launches"],
+            "clocks": clocks,
+            "step1_ms": step1_ms,
+            "step1_attn_tokens": {"int8": s1["attn_tokens_int8"] - s0["attn_tokens_int8"],
+                                  "fp16": s1["attn_tokens_fp16"] - s0["attn_tokens_fp16"]},
+            "step_hbm_gbs": step_bytes / (ms_step * 1e-3) / 1e9,
+            "kernel_ms_per_step": kernel_ms,
+            "kv_resident_bytes": {"conf_kv": stats["bytes_payload"], "full_fp16": full_cache, "sliding_window_512": sw512,
+                                  "tokens_int8": stats["tokens_int8"], "tokens_fp16": stats["tokens_fp16"]},
+        }
+        print(json.dumps(line), flush=True)
+    h.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

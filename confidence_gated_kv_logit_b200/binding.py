@@ -26,7 +26,9 @@ STATUS = {0: "OK", 1: "ERR_ARG", 2: "ERR_CAPACITY", 3: "ERR_STATE", 4: "ERR_NONF
 
 EXPORTED = ["confkv_default_params", "confkv_create", "confkv_destroy", "confkv_prefill",
             "confkv_confidence", "confkv_decode_attn", "confkv_evict_compact", "confkv_query",
-            "confkv_export_segment", "confkv_last_error", "confkv_status_string", "confkv_version"]
+            "confkv_export_segment", "confkv_last_error", "confkv_profile_enable", "confkv_profile_read",
+            "confkv_status_string", "confkv_version"]
+KERNEL_KINDS = ["confidence", "append", "attention", "combine", "ema", "evict", "prefill", "unused"]
 
 
 class ConfKVError(RuntimeError):
@@ -55,6 +57,10 @@ class Stats(ctypes.Structure):
                 ("kernel_launches", ctypes.c_int64)]
 
 
+class Profile(ctypes.Structure):
+    _fields_ = [("launches", ctypes.c_int64 * 8), ("ms", ctypes.c_double * 8)]
+
+
 _LIB = None
 
 
@@ -77,6 +83,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.confkv_query.argtypes = [P, ctypes.POINTER(Stats)]
     lib.confkv_export_segment.argtypes = [P, I32, I32, I32, VP, ctypes.POINTER(ctypes.c_size_t)]
     lib.confkv_last_error.argtypes = [P, I32]
+    lib.confkv_profile_enable.argtypes = [P, I32]
+    lib.confkv_profile_read.argtypes = [P, ctypes.POINTER(Profile), I32]
     lib.confkv_status_string.argtypes = [ctypes.c_int]
     lib.confkv_status_string.restype = ctypes.c_char_p
     lib.confkv_version.restype = ctypes.c_int32
@@ -206,6 +214,15 @@ class ConfKV:
         s = Stats()
         _check(load_library().confkv_query(self._h, ctypes.byref(s)), "confkv_query")
         return {name: getattr(s, name) for name, _ in Stats._fields_}
+
+    def profile(self, enable: bool):
+        _check(load_library().confkv_profile_enable(self._h, 1 if enable else 0), "confkv_profile_enable")
+
+    def profile_read(self, reset: bool = True) -> dict:
+        pr = Profile()
+        _check(load_library().confkv_profile_read(self._h, ctypes.byref(pr), 1 if reset else 0), "confkv_profile_read")
+        return {name: {"launches": int(pr.launches[i]), "ms": float(pr.ms[i])}
+                for i, name in enumerate(KERNEL_KINDS) if name != "unused"}
 
     def last_error(self, clear: bool = False) -> int:
         return int(load_library().confkv_last_error(self._h, 1 if clear else 0))

@@ -7,6 +7,7 @@ statically, so the library needs only the driver at run time.
 from __future__ import annotations
 
 import glob
+import hashlib
 import os
 import subprocess
 import sys
@@ -14,6 +15,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libconfkv.so")
+STAMP = LIB + ".sha256"
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -28,13 +30,23 @@ def sources():
     return sorted(glob.glob(os.path.join(HERE, "csrc", "*.cu")))
 
 
-def needs_build() -> bool:
-    if not os.path.exists(LIB):
-        return True
-    t = os.path.getmtime(LIB)
-    deps = sources() + glob.glob(os.path.join(HERE, "csrc", "*.cuh")) + glob.glob(os.path.join(HERE, "csrc", "*.h"))
+def source_digest() -> str:
+    """Hash of every input of the build (sources, headers, flags)."""
+    deps = sorted(sources() + glob.glob(os.path.join(HERE, "csrc", "*.cuh")) + glob.glob(os.path.join(HERE, "csrc", "*.h")))
     deps.append(os.path.join(ROOT, "include", "confkv.h"))
-    return any(os.path.getmtime(d) > t for d in deps)
+    h = hashlib.sha256(" ".join(NVCC_FLAGS).encode())
+    for d in deps:
+        h.update(os.path.relpath(d, ROOT).encode())
+        with open(d, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def needs_build() -> bool:
+    if not os.path.exists(LIB) or not os.path.exists(STAMP):
+        return True
+    with open(STAMP) as f:
+        return f.read().strip() != source_digest()
 
 
 def build(verbose: bool = False, ptxas_info: bool = False, force: bool = False) -> str:
@@ -53,6 +65,8 @@ def build(verbose: bool = False, ptxas_info: bool = False, force: bool = False) 
     if ptxas_info or verbose:
         sys.stdout.write(res.stdout + res.stderr)
     os.replace(LIB + ".tmp", LIB)
+    with open(STAMP, "w") as f:
+        f.write(source_digest())
     return LIB
 
 

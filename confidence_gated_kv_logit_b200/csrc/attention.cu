@@ -113,6 +113,7 @@ struct Cfg {
   static constexpr int TW_C = TT_C / NCW;         // tokens per consumer warp per tile
   static constexpr int TW_R = TT_R / NCW;
   static constexpr int TW_MAX = TW_C > TW_R ? TW_C : TW_R;
+  static constexpr int MAX_STEPS = TW_MAX / NG;   // score steps per warp per tile
   static constexpr int MINB = G >= 4 ? 2 : 3;     // CTAs per SM the register budget is sized for
   static constexpr int NSTAGE = MINB == 2 ? 4 : 3;
   static constexpr int AUX_BYTES = 2 * (TT_C > TT_R ? TT_C : TT_R) * 4;
@@ -285,14 +286,17 @@ __global__ void __launch_bounds__(160, (G >= 4 ? 2 : 3)) attn_kernel(Cache c, At
       const int tw = cold ? C::TW_C : C::TW_R;
       const int j0 = cold ? t * C::TT_C : (t - u.tiles_c) * C::TT_R;
       const int cnt = cold ? min(C::TT_C, u.n_cold - j0) : min(C::TT_R, c.W - j0);
-      if (lane == 0) {
-        if (cold) n_rows_c += cnt;
-        else n_rows_r += cnt;
-      }
       const int wb = warp * tw;         // first token of this warp in the tile
       uint32_t vmask = 0;               // tokens of this warp that are valid
       const int steps = tw / C::NG;
-      for (int stp = 0; stp < steps; ++stp) {
+      // scores of this warp's tokens (log2 units); the maximum is updated once
+      // per tile so that every probability of the tile uses the same reference
+      float u2s[C::MAX_STEPS][G];
+      float vsc[C::MAX_STEPS];
+      bool up = false;
+#pragma unroll
+      for (int stp = 0; stp < C::MAX_STEPS; ++stp) {
+        if (stp >= steps) break;
         const int tl = stp * C::NG + gi;      // token index within this warp's share
         const int tok = wb + tl;              // token index within the tile
         bool valid = tok < cnt;
@@ -328,42 +332,53 @@ __global__ void __launch_bounds__(160, (G >= 4 ? 2 : 3)) attn_kernel(Cache c, At
           for (int g = 0; g < G; ++g) part[g] += __shfl_xor_sync(0xffffffffu, part[g], o);
         }
         const float kscale = (cold && CI8 && valid) ? reinterpret_cast<const float*>(sb + 2 * C::KV_BYTES)[tok] : 1.0f;
-        float u2[G];
-        bool up = false;
+        vsc[stp] = (cold && CI8 && valid) ? reinterpret_cast<const float*>(sb + 2 * C::KV_BYTES + C::TT_C * 4)[tok]
+                                          : 1.0f;
 #pragma unroll
         for (int g = 0; g < G; ++g) {
           const float sg = part[g] * kscale;
           if (valid && sub == g) sc_base[(size_t)g * a.score_stride + (cold ? 0 : c.cap) + j0 + tok] = sg;
-          u2[g] = valid ? sg * kLog2e : -CUDART_INF_F;
-          up |= u2[g] > m[g];
-        }
-        if (__any_sync(0xffffffffu, up)) {
-#pragma unroll
-          for (int g = 0; g < G; ++g) {
-            const float nm = fmaxf(m[g], warp_max(u2[g]));
-            if (nm > m[g]) {
-              const float corr = exp2f(m[g] - nm);
-              lsum[g] *= corr;
-#pragma unroll
-              for (int e = 0; e < C::E / 2; ++e) acc[g][e] = __fmul2_rn(acc[g][e], make_float2(corr, corr));
-              m[g] = nm;
-            }
-          }
-        }
-        const float vscale = (cold && CI8 && valid)
-                                 ? reinterpret_cast<const float*>(sb + 2 * C::KV_BYTES + C::TT_C * 4)[tok]
-                                 : 1.0f;
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const float p = valid ? exp2f(u2[g] - m[g]) : 0.0f;
-          lsum[g] += p;
-          if (sub == g) ps[tl * 8 + g] = p * vscale;
+          u2s[stp][g] = valid ? sg * kLog2e : -CUDART_INF_F;
+          up |= u2s[stp][g] > m[g];
         }
         const uint32_t bal = __ballot_sync(0xffffffffu, valid && sub == 0);
         // bit gi of the ballot (taken from lane gi*LPT) -> token tl = stp*NG + gi
 #pragma unroll
         for (int k = 0; k < C::NG; ++k)
           if (bal & (1u << (k * C::LPT))) vmask |= 1u << (stp * C::NG + k);
+      }
+      if (__any_sync(0xffffffffu, up)) {
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          float tmax = -CUDART_INF_F;
+#pragma unroll
+          for (int stp = 0; stp < C::MAX_STEPS; ++stp)
+            if (stp < steps) tmax = fmaxf(tmax, u2s[stp][g]);
+          const float nm = fmaxf(m[g], warp_max(tmax));
+          if (nm > m[g]) {
+            const float corr = exp2f(m[g] - nm);
+            lsum[g] *= corr;
+#pragma unroll
+            for (int e = 0; e < C::E / 2; ++e) acc[g][e] = __fmul2_rn(acc[g][e], make_float2(corr, corr));
+            m[g] = nm;
+          }
+        }
+      }
+#pragma unroll
+      for (int stp = 0; stp < C::MAX_STEPS; ++stp) {
+        if (stp >= steps) break;
+        const int tl = stp * C::NG + gi;
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const float u = u2s[stp][g];
+          const float p = u == -CUDART_INF_F ? 0.0f : exp2f(u - m[g]);   // invalid tokens carry nothing
+          lsum[g] += p;
+          if (sub == g) ps[tl * 8 + g] = p * vsc[stp];
+        }
+      }
+      if (lane == 0) {
+        if (cold) n_rows_c += __popc(vmask);
+        else n_rows_r += __popc(vmask);
       }
       __syncwarp();
       // ---- P.V over this warp's tokens: lanes over the head dimension ----
@@ -540,7 +555,8 @@ __global__ void __launch_bounds__(256) ema_kernel(Cache c, AttnLaunch a, Policy 
 }
 
 template <int D, int G, bool CI8>
-cudaError_t run_attn(const Cache& c, const Policy& pol, const AttnLaunch& a, cudaStream_t st, long long* launches) {
+cudaError_t run_attn(const Cache& c, const Policy& pol, const AttnLaunch& a, cudaStream_t st, long long* launches,
+                     Prof* prof) {
   using C = Cfg<D, G, CI8>;
   const int items = a.r.items(c.Hkv);
   cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, G, CI8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -565,14 +581,19 @@ cudaError_t run_attn(const Cache& c, const Policy& pol, const AttnLaunch& a, cud
   while (splits > 1 && (long long)items * splits > a.part_units) --splits;
   const int units = items * splits;
   const int grid = min(units, resident);
-  attn_kernel<D, G, CI8><<<grid, 160, C::SMEM_BYTES, st>>>(c, a, splits, units, rsqrtf((float)D));
+  {
+    ProfScope ps(prof, kKAttention, st);
+    attn_kernel<D, G, CI8><<<grid, 160, C::SMEM_BYTES, st>>>(c, a, splits, units, rsqrtf((float)D));
+  }
   ++*launches;
   if (splits > 1) {
     const int warps = items * G;
+    ProfScope ps(prof, kKCombine, st);
     combine_kernel<D, G><<<(warps * 32 + 255) / 256, 256, 0, st>>>(c, a, splits);
     ++*launches;
   }
   if (pol.mode == 0) {
+    ProfScope ps(prof, kKEma, st);
     ema_kernel<G><<<items, 256, 0, st>>>(c, a, pol);
     ++*launches;
   }
@@ -580,37 +601,41 @@ cudaError_t run_attn(const Cache& c, const Policy& pol, const AttnLaunch& a, cud
 }
 
 template <int D, int G>
-cudaError_t run_attn_g(const Cache& c, const Policy& pol, const AttnLaunch& a, cudaStream_t st, long long* n) {
-  return c.cold_int8 ? run_attn<D, G, true>(c, pol, a, st, n) : run_attn<D, G, false>(c, pol, a, st, n);
+cudaError_t run_attn_g(const Cache& c, const Policy& pol, const AttnLaunch& a, cudaStream_t st, long long* n,
+                       Prof* prof) {
+  return c.cold_int8 ? run_attn<D, G, true>(c, pol, a, st, n, prof) : run_attn<D, G, false>(c, pol, a, st, n, prof);
 }
 
 }  // namespace
 
 cudaError_t launch_decode_attn(const Cache& c, const Policy& pol, const AttnLaunch& a, cudaStream_t st,
-                               long long* launches) {
+                               long long* launches, Prof* prof) {
   const int items = a.r.items(c.Hkv);
   if (items == 0) return cudaSuccess;
   const int blocks = (items * 32 + 255) / 256;
-  if (c.D == 128)
-    append_kernel<128><<<blocks, 256, 0, st>>>(c, a.r, a.k_new, a.v_new, a.prio_new, pol.mode == 1);
-  else
-    append_kernel<64><<<blocks, 256, 0, st>>>(c, a.r, a.k_new, a.v_new, a.prio_new, pol.mode == 1);
+  {
+    ProfScope ps(prof, kKAppend, st);
+    if (c.D == 128)
+      append_kernel<128><<<blocks, 256, 0, st>>>(c, a.r, a.k_new, a.v_new, a.prio_new, pol.mode == 1);
+    else
+      append_kernel<64><<<blocks, 256, 0, st>>>(c, a.r, a.k_new, a.v_new, a.prio_new, pol.mode == 1);
+  }
   ++*launches;
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (c.D == 128) {
     switch (c.G) {
-      case 1: return run_attn_g<128, 1>(c, pol, a, st, launches);
-      case 2: return run_attn_g<128, 2>(c, pol, a, st, launches);
-      case 4: return run_attn_g<128, 4>(c, pol, a, st, launches);
-      case 5: return run_attn_g<128, 5>(c, pol, a, st, launches);
-      case 8: return run_attn_g<128, 8>(c, pol, a, st, launches);
+      case 1: return run_attn_g<128, 1>(c, pol, a, st, launches, prof);
+      case 2: return run_attn_g<128, 2>(c, pol, a, st, launches, prof);
+      case 4: return run_attn_g<128, 4>(c, pol, a, st, launches, prof);
+      case 5: return run_attn_g<128, 5>(c, pol, a, st, launches, prof);
+      case 8: return run_attn_g<128, 8>(c, pol, a, st, launches, prof);
     }
   } else {
     switch (c.G) {
-      case 1: return run_attn_g<64, 1>(c, pol, a, st, launches);
-      case 2: return run_attn_g<64, 2>(c, pol, a, st, launches);
-      case 4: return run_attn_g<64, 4>(c, pol, a, st, launches);
+      case 1: return run_attn_g<64, 1>(c, pol, a, st, launches, prof);
+      case 2: return run_attn_g<64, 2>(c, pol, a, st, launches, prof);
+      case 4: return run_attn_g<64, 4>(c, pol, a, st, launches, prof);
     }
   }
   return cudaErrorInvalidValue;

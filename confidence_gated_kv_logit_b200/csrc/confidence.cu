@@ -187,8 +187,10 @@ __global__ void __launch_bounds__(NT) confidence_kernel(ConfLaunch a, Policy pol
 
 }  // namespace
 
-cudaError_t launch_confidence(const ConfLaunch& a, const Policy& pol, cudaStream_t st, long long* launches) {
+cudaError_t launch_confidence(const ConfLaunch& a, const Policy& pol, cudaStream_t st, long long* launches,
+                              Prof* prof) {
   dim3 grid(a.cpr, a.B);
+  ProfScope ps(prof, kKConfidence, st);
   confidence_kernel<<<grid, NT, 0, st>>>(a, pol);
   ++*launches;
   return cudaGetLastError();

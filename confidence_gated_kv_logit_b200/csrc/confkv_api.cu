@@ -79,6 +79,8 @@ struct confkv_handle {
   int32_t* keep_list;
   int32_t* keep_count;
   long long launches;
+  confkv::Prof prof;
+  confkv::Prof* prof_ptr() { return prof.on ? &prof : nullptr; }
 };
 
 // Handles currently alive; lets a destroyed or foreign pointer be rejected
@@ -377,7 +379,7 @@ confkv_status confkv_prefill(confkv_handle* h, int32_t layer, int32_t batch, con
   a.prio = priority;
   a.keep_list = h->keep_list;
   a.keep_count = h->keep_count;
-  e = confkv::launch_prefill(h->c, h->pol, a, st, &h->launches);
+  e = confkv::launch_prefill(h->c, h->pol, a, st, &h->launches, h->prof_ptr());
   if (e != cudaSuccess) return CONFKV_ERR_CUDA;
   // the host copy of lens must stay valid until the copy has been consumed
   e = cudaStreamSynchronize(st);
@@ -407,7 +409,8 @@ confkv_status confkv_confidence(confkv_handle* h, const float* logits, int32_t b
   a.c_out = c_out;
   a.budget_out = budget_out;
   a.err = h->c.err;
-  return cuda_status(confkv::launch_confidence(a, h->pol, static_cast<cudaStream_t>(stream), &h->launches));
+  return cuda_status(
+      confkv::launch_confidence(a, h->pol, static_cast<cudaStream_t>(stream), &h->launches, h->prof_ptr()));
 }
 
 confkv_status confkv_decode_attn(confkv_handle* h, int32_t layer, const void* q, const void* k_new,
@@ -442,7 +445,8 @@ confkv_status confkv_decode_attn(confkv_handle* h, int32_t layer, const void* q,
   a.part_units = h->part_units;
   a.max_cold_tokens = (int)std::min<long long>(ub, h->c.cap);
   a.num_sms = h->num_sms;
-  cudaError_t e = confkv::launch_decode_attn(h->c, h->pol, a, static_cast<cudaStream_t>(stream), &h->launches);
+  cudaError_t e =
+      confkv::launch_decode_attn(h->c, h->pol, a, static_cast<cudaStream_t>(stream), &h->launches, h->prof_ptr());
   if (e != cudaSuccess) return cuda_status(e);
   for (int l = r.l0; l < r.l0 + r.nl; ++l) h->ub_len[l] += 1;
   return CONFKV_OK;
@@ -461,7 +465,8 @@ confkv_status confkv_evict_compact(confkv_handle* h, int32_t layer, void* stream
   a.vmask = h->vmask;
   a.mask_words = h->mask_words;
   a.stable = h->p.compact == CONFKV_COMPACT_STABLE;
-  cudaError_t e = confkv::launch_evict_compact(h->c, h->pol, a, static_cast<cudaStream_t>(stream), &h->launches);
+  cudaError_t e =
+      confkv::launch_evict_compact(h->c, h->pol, a, static_cast<cudaStream_t>(stream), &h->launches, h->prof_ptr());
   if (e != cudaSuccess) return cuda_status(e);
   for (int l = r.l0; l < r.l0 + r.nl; ++l) h->ub_len[l] = std::min<long long>(h->ub_len[l], h->max_eff[l]);
   return CONFKV_OK;
@@ -573,6 +578,25 @@ confkv_status confkv_export_segment(confkv_handle* h, int32_t layer, int32_t seq
   d2h(o, c.vr + rs * c.D, W * c.D * 2);
   *bytes = need;
   return e == cudaSuccess ? CONFKV_OK : CONFKV_ERR_CUDA;
+}
+
+confkv_status confkv_profile_enable(confkv_handle* h, int32_t enable) {
+  if (!alive(h)) return CONFKV_ERR_STATE;
+  h->prof.collect();
+  h->prof.on = enable != 0;
+  return CONFKV_OK;
+}
+
+confkv_status confkv_profile_read(confkv_handle* h, confkv_profile* out, int32_t reset) {
+  if (!alive(h)) return CONFKV_ERR_STATE;
+  if (!out) return CONFKV_ERR_ARG;
+  h->prof.collect();
+  for (int i = 0; i < CONFKV_K_KINDS; ++i) {
+    out->launches[i] = h->prof.launches[i];
+    out->ms[i] = h->prof.ms[i];
+  }
+  if (reset) h->prof.reset();
+  return CONFKV_OK;
 }
 
 confkv_status confkv_last_error(confkv_handle* h, int32_t clear) {

@@ -234,8 +234,10 @@ __global__ void __launch_bounds__(NT) evict_kernel(Cache c, Policy pol, EvictLau
 }
 
 template <int D, bool CI8>
-cudaError_t run(const Cache& c, const Policy& pol, const EvictLaunch& a, cudaStream_t st, long long* launches) {
+cudaError_t run(const Cache& c, const Policy& pol, const EvictLaunch& a, cudaStream_t st, long long* launches,
+                Prof* prof) {
   const int items = a.r.items(c.Hkv);
+  ProfScope ps(prof, kKEvict, st);
   evict_kernel<D, CI8><<<items, NT, 0, st>>>(c, pol, a);
   ++*launches;
   return cudaGetLastError();
@@ -244,10 +246,11 @@ cudaError_t run(const Cache& c, const Policy& pol, const EvictLaunch& a, cudaStr
 }  // namespace
 
 cudaError_t launch_evict_compact(const Cache& c, const Policy& pol, const EvictLaunch& a, cudaStream_t st,
-                                 long long* launches) {
+                                 long long* launches, Prof* prof) {
   if (a.r.items(c.Hkv) == 0) return cudaSuccess;
-  if (c.D == 128) return c.cold_int8 ? run<128, true>(c, pol, a, st, launches) : run<128, false>(c, pol, a, st, launches);
-  return c.cold_int8 ? run<64, true>(c, pol, a, st, launches) : run<64, false>(c, pol, a, st, launches);
+  if (c.D == 128)
+    return c.cold_int8 ? run<128, true>(c, pol, a, st, launches, prof) : run<128, false>(c, pol, a, st, launches, prof);
+  return c.cold_int8 ? run<64, true>(c, pol, a, st, launches, prof) : run<64, false>(c, pol, a, st, launches, prof);
 }
 
 }  // namespace confkv

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include "common.cuh"
+#include "prof.h"
 
 namespace confkv {
 
@@ -25,7 +26,8 @@ struct ConfLaunch {
   int32_t* budget_out;    // optional
   int32_t* err;
 };
-cudaError_t launch_confidence(const ConfLaunch& a, const Policy& pol, cudaStream_t st, long long* launches);
+cudaError_t launch_confidence(const ConfLaunch& a, const Policy& pol, cudaStream_t st, long long* launches,
+                              Prof* prof);
 
 // K2: prefill ingest.
 struct PrefillLaunch {
@@ -39,7 +41,7 @@ struct PrefillLaunch {
   int32_t* keep_count;    // fixed mode: [items]
 };
 cudaError_t launch_prefill(const Cache& c, const Policy& pol, const PrefillLaunch& a, cudaStream_t st,
-                           long long* launches);
+                           long long* launches, Prof* prof);
 
 // K3 + K3c + EMA: decode attention.
 struct AttnLaunch {
@@ -59,7 +61,7 @@ struct AttnLaunch {
   int num_sms;
 };
 cudaError_t launch_decode_attn(const Cache& c, const Policy& pol, const AttnLaunch& a, cudaStream_t st,
-                               long long* launches);
+                               long long* launches, Prof* prof);
 
 // K4 + K5 + K6: select, compaction, conversion of the token leaving the window.
 struct EvictLaunch {
@@ -70,6 +72,6 @@ struct EvictLaunch {
   int stable;             // 1: order-preserving compaction
 };
 cudaError_t launch_evict_compact(const Cache& c, const Policy& pol, const EvictLaunch& a, cudaStream_t st,
-                                 long long* launches);
+                                 long long* launches, Prof* prof);
 
 }  // namespace confkv

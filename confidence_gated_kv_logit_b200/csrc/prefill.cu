@@ -133,7 +133,8 @@ __global__ void __launch_bounds__(NT) prefill_ingest_kernel(Cache c, PrefillLaun
 }  // namespace
 
 cudaError_t launch_prefill(const Cache& c, const Policy& pol, const PrefillLaunch& a, cudaStream_t st,
-                           long long* launches) {
+                           long long* launches, Prof* prof) {
+  ProfScope ps(prof, kKPrefill, st);
   const int items = a.r.items(c.Hkv);
   if (items == 0) return cudaSuccess;
   const bool fixed = pol.mode == 1;

@@ -206,6 +206,22 @@ CONFKV_API confkv_status confkv_export_segment(confkv_handle* h, int32_t layer, 
  * clear nonzero it is reset. */
 CONFKV_API confkv_status confkv_last_error(confkv_handle* h, int32_t clear);
 
+/* Per-kernel timing. While enabled, every kernel launch of the handle is
+ * bracketed by CUDA events on its stream (a few microseconds of host work per
+ * launch, nothing on the device). confkv_profile_read synchronises on the
+ * recorded events and returns, per kernel kind, the launches and the summed
+ * milliseconds since the last reset. */
+enum {
+  CONFKV_K_CONFIDENCE = 0, CONFKV_K_APPEND = 1, CONFKV_K_ATTENTION = 2, CONFKV_K_COMBINE = 3,
+  CONFKV_K_EMA = 4, CONFKV_K_EVICT = 5, CONFKV_K_PREFILL = 6, CONFKV_K_KINDS = 8
+};
+typedef struct {
+  int64_t launches[CONFKV_K_KINDS];
+  double ms[CONFKV_K_KINDS];
+} confkv_profile;
+CONFKV_API confkv_status confkv_profile_enable(confkv_handle* h, int32_t enable);
+CONFKV_API confkv_status confkv_profile_read(confkv_handle* h, confkv_profile* out, int32_t reset);
+
 /* Static description of a status code. */
 CONFKV_API const char* confkv_status_string(confkv_status s);
 

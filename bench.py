@@ -132,6 +132,14 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+def _report_device_error(h, where):
+    st, site, seg, val = h.last_error_detail()
+    if st != 0:
+        print(f"device error word {st} after {where}: check site {site}, segment {seg}, value {val}",
+              file=sys.stderr, flush=True)
+        raise SystemExit(3)
+
+
 def physical_gpu_index(local_rank: int) -> int:
     vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
     ids = [x.strip() for x in vis.split(",") if x.strip()]
@@ -282,9 +290,11 @@ def main():
     torch.cuda.synchronize()
     step1_ms = e0.elapsed_time(e1)
     s1 = h.query()
+    _report_device_error(h, "first step")
     for i in range(1, 1 + args.warmup):
         step(i)
     torch.cuda.synchronize()
+    _report_device_error(h, "warm-up")
 
     # ---- timed region ----
     h.profile(True)
@@ -304,6 +314,7 @@ def main():
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
+    _report_device_error(h, "timed region")
     elapsed_ms = e0.elapsed_time(e1)
     prof = h.profile_read(reset=True)
     h.profile(False)
@@ -364,6 +375,7 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
+    _report_device_error(h, "end-to-end region")
     if world > 1:
         t = torch.tensor([e2e_ms], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -373,7 +385,7 @@ def main():
     stats = h.query()
     full_cache = L * B * Hkv * (T + 1 + args.warmup + K + E) * 4 * D
     sw512 = L * B * Hkv * 512 * 4 * D
-    assert h.last_error() == 0, "device error word set"
+    _report_device_error(h, "the run")
 
     if rank == 0:
         cpu = None

@@ -14,7 +14,9 @@ import os
 import numpy as np
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libconfkv.so")
+# CONFKV_LIBRARY selects another build of the same library (e.g. the
+# self-checking one); there is no non-CUDA implementation to fall back to.
+LIB_PATH = os.environ.get("CONFKV_LIBRARY", os.path.join(HERE, "libconfkv.so"))
 
 ALL_LAYERS = -1
 MODE_CONF, MODE_FIXED = 0, 1
@@ -26,7 +28,8 @@ STATUS = {0: "OK", 1: "ERR_ARG", 2: "ERR_CAPACITY", 3: "ERR_STATE", 4: "ERR_NONF
 
 EXPORTED = ["confkv_default_params", "confkv_create", "confkv_destroy", "confkv_prefill",
             "confkv_confidence", "confkv_decode_attn", "confkv_evict_compact", "confkv_query",
-            "confkv_export_segment", "confkv_last_error", "confkv_profile_enable", "confkv_profile_read",
+            "confkv_export_segment", "confkv_last_error", "confkv_last_error_detail",
+            "confkv_profile_enable", "confkv_profile_read",
             "confkv_status_string", "confkv_version"]
 KERNEL_KINDS = ["confidence", "append", "attention", "combine", "ema", "evict", "prefill", "unused"]
 
@@ -83,6 +86,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.confkv_query.argtypes = [P, ctypes.POINTER(Stats)]
     lib.confkv_export_segment.argtypes = [P, I32, I32, I32, VP, ctypes.POINTER(ctypes.c_size_t)]
     lib.confkv_last_error.argtypes = [P, I32]
+    lib.confkv_last_error_detail.argtypes = [P, ctypes.POINTER(ctypes.c_int32)]
     lib.confkv_profile_enable.argtypes = [P, I32]
     lib.confkv_profile_read.argtypes = [P, ctypes.POINTER(Profile), I32]
     lib.confkv_status_string.argtypes = [ctypes.c_int]
@@ -226,6 +230,11 @@ class ConfKV:
 
     def last_error(self, clear: bool = False) -> int:
         return int(load_library().confkv_last_error(self._h, 1 if clear else 0))
+
+    def last_error_detail(self) -> tuple:
+        d = (ctypes.c_int32 * 3)()
+        st = int(load_library().confkv_last_error_detail(self._h, d))
+        return st, int(d[0]), int(d[1]), int(d[2])
 
     def export_segment(self, layer: int, seq: int, kv_head: int) -> dict:
         """Raw state of one segment, as numpy arrays in physical order."""

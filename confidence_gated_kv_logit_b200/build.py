@@ -49,6 +49,19 @@ def needs_build() -> bool:
         return f.read().strip() != source_digest()
 
 
+def build_checked(verbose: bool = False) -> str:
+    """Build libconfkv_checked.so: the same library with every data-dependent
+    index checked on the device (failures are recorded and skipped)."""
+    out = os.path.join(HERE, "libconfkv_checked.so")
+    nvcc = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
+    cmd = [nvcc, *NVCC_FLAGS, "-DCONFKV_CHECKED", "-shared", "-I", os.path.join(ROOT, "include"), "-o", out, *sources()]
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    if res.returncode != 0:
+        sys.stderr.write(res.stdout + res.stderr)
+        raise RuntimeError("nvcc failed to build libconfkv_checked.so")
+    return out
+
+
 def build(verbose: bool = False, ptxas_info: bool = False, force: bool = False) -> str:
     if not force and not needs_build():
         return LIB

@@ -47,6 +47,7 @@ __global__ void __launch_bounds__(256) append_kernel(Cache c, Range r, const __h
   int l, b, h;
   const int s = seg_of(c, r, warp, &l, &b, &h);
   const int t = c.next_pos[s];
+  if (!guard(t >= 0 && c.n_cold[s] >= 0 && c.n_cold[s] <= c.cap, c.err, kSiteAppendSeg, s, t)) return;
   const size_t in_row = ((size_t)((l - r.l0) * r.B + b) * c.Hkv + h);
   const __half* kn = k_new + in_row * D;
   const __half* vn = v_new + in_row * D;
@@ -140,6 +141,13 @@ __device__ __forceinline__ Unit make_unit(const Cache& c, const Range& r, int sp
   const int split = unit - item * splits;
   u.s = seg_of(c, r, item, &u.l, &u.b, &u.h);
   u.n_cold = c.n_cold[u.s];
+  if (u.n_cold < 0 || u.n_cold > c.cap) {   // corrupt segment: record once (by its split 0) and skip
+    if (split == 0 && threadIdx.x == 0) record_violation(c.err, kSiteAttnSeg, u.s, u.n_cold);
+    u.n_cold = 0;
+    u.tiles_c = 0;
+    u.t0 = u.t1 = 0;
+    return u;
+  }
   u.tiles_c = (u.n_cold + C::TT_C - 1) / C::TT_C;
   const int tiles_r = (c.W + C::TT_R - 1) / C::TT_R;
   const int tiles = u.tiles_c + tiles_r;
@@ -196,6 +204,16 @@ __global__ void __launch_bounds__(160, (G >= 4 ? 2 : 3)) attn_kernel(Cache c, At
           }
           unsigned char* sb = stages + st * C::STAGE_BYTES;
           const bool cold = t < u.tiles_c;
+          if (kChecked) {
+            const int j0 = cold ? t * C::TT_C : (t - u.tiles_c) * C::TT_R;
+            const int cnt = cold ? min(C::TT_C, u.n_cold - j0) : min(C::TT_R, c.W - j0);
+            const int lim = cold ? c.cap : c.Wst;
+            if (!guard(cnt >= 1 && j0 >= 0 && j0 + ((cnt + 3) & ~3) <= lim, c.err, kSiteAttnTile, u.s, j0)) {
+              *abort_flag = 1;   // consumers give up on their bounded wait for this tile
+              stop = true;
+              break;
+            }
+          }
           if (cold) {
             const int j0 = t * C::TT_C;
             const int cnt = min(C::TT_C, u.n_cold - j0);
@@ -248,7 +266,9 @@ __global__ void __launch_bounds__(160, (G >= 4 ? 2 : 3)) attn_kernel(Cache c, At
     // query slice of this lane, scaled by 1/sqrt(D)
     float2 q2[G][8];
     {
-      const __half* qp = a.q + ((size_t)((u.l - a.r.l0) * a.r.B + u.b) * c.Hq + u.h * G) * D + sub * 16;
+      const size_t qrow = (size_t)((u.l - a.r.l0) * a.r.B + u.b) * c.Hq + u.h * G;
+      if (kChecked) guard(qrow + G <= (size_t)a.r.items(c.Hkv) * G, c.err, kSiteAttnQ, u.s, (int)qrow);
+      const __half* qp = a.q + qrow * D + sub * 16;
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         const uint4 w0 = *reinterpret_cast<const uint4*>(qp + g * D);
@@ -337,7 +357,11 @@ __global__ void __launch_bounds__(160, (G >= 4 ? 2 : 3)) attn_kernel(Cache c, At
 #pragma unroll
         for (int g = 0; g < G; ++g) {
           const float sg = part[g] * kscale;
-          if (valid && sub == g) sc_base[(size_t)g * a.score_stride + (cold ? 0 : c.cap) + j0 + tok] = sg;
+          if (valid && sub == g) {
+            const int col = (cold ? 0 : c.cap) + j0 + tok;
+            if (!kChecked || guard(col >= 0 && col < a.score_stride, c.err, kSiteAttnScore, u.s, col))
+              sc_base[(size_t)g * a.score_stride + col] = sg;
+          }
           u2s[stp][g] = valid ? sg * kLog2e : -CUDART_INF_F;
           up |= u2s[stp][g] > m[g];
         }
@@ -462,6 +486,7 @@ __global__ void __launch_bounds__(160, (G >= 4 ? 2 : 3)) attn_kernel(Cache c, At
       }
       if (splits == 1) {
         const size_t orow = (size_t)((u.l - a.r.l0) * a.r.B + u.b) * c.Hq + u.h * G + g;
+        if (kChecked && !guard(orow < (size_t)a.r.items(c.Hkv) * G, c.err, kSiteAttnOut, u.s, (int)orow)) continue;
         a.out[orow * D + d] = A / L;
         if (d == 0) {
           const float lse = (M + __log2f(L)) * kLn2;
@@ -533,6 +558,7 @@ __global__ void __launch_bounds__(256) ema_kernel(Cache c, AttnLaunch a, Policy 
 #pragma unroll
   for (int g = 0; g < G; ++g) lse[g] = a.lse_ws[(size_t)s * G + g];
   const int n_cold = c.n_cold[s];
+  if (!guard(n_cold >= 0 && n_cold <= c.cap, c.err, kSiteEmaSeg, s, n_cold)) return;
   const float* sb = a.scores + (size_t)s * G * a.score_stride;
   const float invG = 1.0f / G;
   for (int i = threadIdx.x; i < n_cold + c.W; i += blockDim.x) {

@@ -90,6 +90,38 @@ __device__ __forceinline__ int seg_of(const Cache& c, const Range& r, int item, 
 
 __device__ __forceinline__ void set_error(int32_t* err, int code) { atomicCAS(err, 0, code); }
 
+// err[0] is the sticky status word; err[1..3] describe the first failed device
+// check: (site, segment, offending value).
+__device__ __forceinline__ void record_violation(int32_t* err, int site, int seg, int val) {
+  if (atomicCAS(err, 0, kErrDevice) == 0) {
+    err[1] = site;
+    err[2] = seg;
+    err[3] = val;
+  }
+}
+
+// Returns ok; records the first failure. Used for checks that are always on
+// (per segment) and, in builds with CONFKV_CHECKED, for every data-dependent index.
+__device__ __forceinline__ bool guard(bool ok, int32_t* err, int site, int seg, int val) {
+  if (!ok) record_violation(err, site, seg, val);
+  return ok;
+}
+
+#ifdef CONFKV_CHECKED
+constexpr bool kChecked = true;
+#else
+constexpr bool kChecked = false;
+#endif
+
+// Check sites (value of err[1]).
+enum Site {
+  kSiteAppendSeg = 101, kSiteAppendSlot = 102,
+  kSiteAttnSeg = 201, kSiteAttnTile = 202, kSiteAttnScore = 203, kSiteAttnOut = 204, kSiteAttnQ = 205,
+  kSiteEmaSeg = 301, kSiteEmaCol = 302,
+  kSiteEvictSeg = 401, kSiteEvictPair = 402, kSiteEvictRequant = 403, kSiteEvictWord = 404,
+  kSitePrefillRow = 501, kSiteCombine = 601
+};
+
 // ---------------------------------------------------------------------------
 // Exact int8 -> fp32 conversion without the conversion unit: the biased byte
 // u = x + 128 is permuted into the low mantissa byte of 2^23 (bit pattern

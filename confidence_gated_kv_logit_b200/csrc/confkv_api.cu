@@ -268,7 +268,7 @@ confkv_status confkv_create(int32_t layers, int32_t kv_heads, int32_t q_heads, i
   chk(B.alloc(&c.sc_r, rrows));
   chk(B.alloc(&c.n_cold, S));
   chk(B.alloc(&c.next_pos, S));
-  chk(B.alloc(&c.err, 1));
+  chk(B.alloc(&c.err, 4));
   chk(B.alloc(&c.counters, (size_t)confkv::kNumCounters));
   chk(B.alloc(&h->lens_dev, (size_t)p.max_batch));
   chk(B.alloc(&h->budget, (size_t)p.max_batch * layers));
@@ -304,7 +304,7 @@ confkv_status confkv_create(int32_t layers, int32_t kv_heads, int32_t q_heads, i
     }
     chk(cudaMemset(c.n_cold, 0, S * 4));
     chk(cudaMemset(c.next_pos, 0, S * 4));
-    chk(cudaMemset(c.err, 0, 4));
+    chk(cudaMemset(c.err, 0, 16));
     chk(cudaMemset(c.counters, 0, confkv::kNumCounters * 8));
     chk(cudaMemset(h->tickets, 0, (size_t)p.max_batch * 4));
     chk(cudaMemset(h->scores, 0, S * G * (size_t)h->score_stride * 4));
@@ -580,6 +580,19 @@ confkv_status confkv_export_segment(confkv_handle* h, int32_t layer, int32_t seq
   return e == cudaSuccess ? CONFKV_OK : CONFKV_ERR_CUDA;
 }
 
+confkv_status confkv_last_error_detail(confkv_handle* h, int32_t* detail) {
+  if (!alive(h)) return CONFKV_ERR_STATE;
+  if (!detail) return CONFKV_ERR_ARG;
+  int32_t v[4] = {0, 0, 0, 0};
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpy(v, h->c.err, 16, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return CONFKV_ERR_CUDA;
+  detail[0] = v[1];
+  detail[1] = v[2];
+  detail[2] = v[3];
+  return static_cast<confkv_status>(v[0]);
+}
+
 confkv_status confkv_profile_enable(confkv_handle* h, int32_t enable) {
   if (!alive(h)) return CONFKV_ERR_STATE;
   h->prof.collect();
@@ -604,7 +617,7 @@ confkv_status confkv_last_error(confkv_handle* h, int32_t clear) {
   int32_t v = 0;
   cudaError_t e = cudaDeviceSynchronize();
   if (e == cudaSuccess) e = cudaMemcpy(&v, h->c.err, 4, cudaMemcpyDeviceToHost);
-  if (e == cudaSuccess && clear) e = cudaMemset(h->c.err, 0, 4);
+  if (e == cudaSuccess && clear) e = cudaMemset(h->c.err, 0, 16);
   if (e == cudaSuccess && clear) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return CONFKV_ERR_CUDA;
   return static_cast<confkv_status>(v);

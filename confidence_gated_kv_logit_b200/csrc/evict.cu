@@ -72,6 +72,7 @@ __global__ void __launch_bounds__(NT) evict_kernel(Cache c, Policy pol, EvictLau
   const int t = c.next_pos[s] - 1;
   const int n_cold = c.n_cold[s];
   const int W = c.W;
+  if (!guard(n_cold >= 0 && n_cold <= c.cap && t >= -1, c.err, kSiteEvictSeg, s, n_cold)) return;
   const int32_t* pos_c = c.pos_c + (size_t)s * c.cap;
   const float* sc_c = c.sc_c + (size_t)s * c.cap;
   int32_t* pos_r = c.pos_r + (size_t)s * c.Wst;
@@ -137,6 +138,9 @@ __global__ void __launch_bounds__(NT) evict_kernel(Cache c, Policy pol, EvictLau
         if (np == 0) break;
         for (int w = threadIdx.x; w < np * 2 * R::VEC; w += NT) {
           const int p = w / (2 * R::VEC);
+          if (kChecked && !guard(list_h[p] >= 0 && list_h[p] < n_keep && list_m[p] >= n_keep && list_m[p] < n_cold,
+                                 c.err, kSiteEvictPair, s, list_m[p]))
+            continue;
           move_cold_row<D, CI8>(c, s, list_m[p], list_h[p], w - p * 2 * R::VEC);
         }
         moved += np;
@@ -209,8 +213,8 @@ __global__ void __launch_bounds__(NT) evict_kernel(Cache c, Policy pol, EvictLau
     const size_t rs = (size_t)s * c.Wst + slot;
     if (c.pos_r[rs] == leaving) {
       const int idx = n_cold_new;
-      if (idx >= c.cap) {
-        if (threadIdx.x == 0) set_error(c.err, kErrDevice);
+      if (idx >= c.cap || idx < 0) {
+        if (threadIdx.x == 0) record_violation(c.err, kSiteEvictRequant, s, idx);
       } else {
         const size_t cs = (size_t)s * c.cap + idx;
         warp_quantize_row<D>(c.kr + rs * D, c.k8 + cs * D, c.ks + cs, threadIdx.x);

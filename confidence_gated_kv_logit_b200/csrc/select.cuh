@@ -51,8 +51,9 @@ __device__ __forceinline__ int block_sum_int(int v, SelectSmem<NT>& sm) {
 }
 
 // Collect, in increasing order, up to CAP indices i in [*cur, end) with
-// pred(i), into list[]. Advances *cur past the last collected index (or to
-// end). Every thread returns the same count and cursor.
+// pred(i), into list[] (shared memory). Advances *cur past the last collected
+// index (or to end). Every thread returns the same count and cursor, and the
+// list is complete and visible to all threads on return.
 template <int NT, int CAP, class Pred>
 __device__ int block_collect(Pred pred, int* cur, int end, int* list, SelectSmem<NT>& sm) {
   int count = 0;
@@ -75,6 +76,7 @@ __device__ int block_collect(Pred pred, int* cur, int end, int* list, SelectSmem
     c0 += NT;
   }
   *cur = min(c0, end);
+  __syncthreads();   // list[] entries written by other threads are visible to every caller thread
   return count;
 }
 

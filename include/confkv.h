@@ -206,6 +206,13 @@ CONFKV_API confkv_status confkv_export_segment(confkv_handle* h, int32_t layer, 
  * clear nonzero it is reset. */
 CONFKV_API confkv_status confkv_last_error(confkv_handle* h, int32_t clear);
 
+/* Synchronising: like confkv_last_error (not clearing), and when a device-side
+ * check failed, detail[3] receives (check site, segment id, offending value)
+ * of the first failure. Sites: 1xx append, 2xx attention, 3xx EMA, 4xx
+ * eviction, 5xx prefill, 6xx combine; the work guarded by a failed check is
+ * skipped, never performed out of bounds. */
+CONFKV_API confkv_status confkv_last_error_detail(confkv_handle* h, int32_t* detail);
+
 /* Per-kernel timing. While enabled, every kernel launch of the handle is
  * bracketed by CUDA events on its stream (a few microseconds of host work per
  * launch, nothing on the device). confkv_profile_read synchronises on the

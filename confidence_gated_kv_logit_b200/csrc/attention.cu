@@ -25,6 +25,11 @@
 #include "kernels.h"
 #include "tma.cuh"
 
+// CTAs per SM the register budget of the G >= 4 attention kernels targets.
+#ifndef CONFKV_G4_MINB
+#define CONFKV_G4_MINB 2
+#endif
+
 namespace confkv {
 
 namespace {
@@ -114,17 +119,26 @@ struct Cfg {
   static constexpr int TW_C = TT_C / NCW;         // tokens per consumer warp per tile
   static constexpr int TW_R = TT_R / NCW;
   static constexpr int TW_MAX = TW_C > TW_R ? TW_C : TW_R;
-  static constexpr int MAX_STEPS = TW_MAX / NG;   // score steps per warp per tile
-  static constexpr int MINB = G >= 4 ? 2 : 3;     // CTAs per SM the register budget is sized for
+  // Score reduction across the LPT lanes of a token: when G divides LPT, each
+  // lane group scores TPG = LPT/G tokens at once and a transposed (reduce-
+  // scatter) butterfly leaves exactly one (token, head) score in every lane;
+  // otherwise one token per group and a plain butterfly, lanes sub < G keep
+  // one head each.
+  static constexpr bool XPOSE = (LPT % G) == 0;
+  static constexpr int TPG = XPOSE ? LPT / G : 1;
+  static constexpr int STEP_TOK = NG * TPG;       // tokens per warp per score step
+  static constexpr int SPT_C = (TW_C + STEP_TOK - 1) / STEP_TOK;
+  static constexpr int SPT_R = (TW_R + STEP_TOK - 1) / STEP_TOK;
+  static constexpr int MAX_STEPS = SPT_C > SPT_R ? SPT_C : SPT_R;
+  static constexpr int MINB = G >= 4 ? CONFKV_G4_MINB : 3;   // CTAs per SM the register budget is sized for
   static constexpr int NSTAGE = MINB == 2 ? 4 : 3;
   static constexpr int AUX_BYTES = 2 * (TT_C > TT_R ? TT_C : TT_R) * 4;
   static constexpr int STAGE_BYTES = 2 * KV_BYTES + AUX_BYTES;
-  static constexpr int PS_BYTES = NCW * TW_MAX * 8 * 4;          // probabilities, padded to 8 heads
+  static constexpr int PS_BYTES = NCW * TW_MAX * 8 * 4;          // probabilities [8 heads][TW_MAX] per warp
   static constexpr int MERGE_BYTES = NCW * G * (D + 2) * 4;
   static constexpr int SMEM_BYTES = NSTAGE * STAGE_BYTES + PS_BYTES + MERGE_BYTES + 2 * NSTAGE * 8 + 16;
   static_assert(G <= LPT, "at most head_dim/16 query heads per KV head");
-  static_assert(TW_C % NG == 0 && TW_R % NG == 0, "tile split");
-  static_assert(TW_MAX <= 32, "validity mask is one word");
+  static_assert(TW_MAX <= 32, "a warp's share of a tile is at most 32 tokens");
 };
 
 struct Unit {
@@ -157,8 +171,223 @@ __device__ __forceinline__ Unit make_unit(const Cache& c, const Range& r, int sp
   return u;
 }
 
+
+// Per-warp online-softmax state of one unit.
+template <int D, int G>
+struct WarpState {
+  float m[G];                // running maximum per head (log2 units), uniform in the warp
+  float2 acc[G][D / 32];     // P.V partial sums: .x over even tokens, .y over odd tokens of a pair
+  float l_own;               // this lane's share of the softmax sum of its own head
+};
+
+enum TileKind { kTileCold8 = 0, kTileCold16 = 1, kTileRing = 2 };
+
+// One warp's share of one staged tile: scores (with the lane-group reduction),
+// the once-per-tile maximum update, probabilities, then P.V over token pairs.
+// Loops have compile-time trip counts; rows outside the tile are loaded
+// predicated to zero instead of branching.
+template <int D, int G, bool CI8, int KIND>
+__device__ __forceinline__ void consume_tile(const Cache& c, const AttnLaunch& a, const unsigned char* sb,
+                                             const float2 (&q2)[G][8], WarpState<D, G>& ws, float* ps,
+                                             float* sc_base, int s_id, int j0, int cnt, int warp, int lane,
+                                             unsigned long long& n_rows) {
+  using C = Cfg<D, G, CI8>;
+  constexpr bool COLD = KIND != kTileRing;
+  constexpr bool I8 = KIND == kTileCold8;
+  constexpr int TW = COLD ? C::TW_C : C::TW_R;
+  constexpr int ROWB = I8 ? D : 2 * D;
+  constexpr int STEPS = (TW + C::STEP_TOK - 1) / C::STEP_TOK;
+  constexpr int E = D / 32;
+  const int sub = lane % C::LPT;
+  const int gi = lane / C::LPT;
+  const bool own = C::XPOSE || sub < G;
+  const int g_own = C::XPOSE ? sub % G : (sub < G ? sub : 0);
+  const int t_own = C::XPOSE ? sub / G : 0;
+  const int wb = warp * TW;
+  const float* aux = reinterpret_cast<const float*>(sb + 2 * C::KV_BYTES);
+  const unsigned char* kb = sb;
+  const unsigned char* vb = sb + C::KV_BYTES;
+
+  float u_own[STEPS];
+  int tl_own[STEPS];
+  float lmax = -CUDART_INF_F;
+#pragma unroll
+  for (int stp = 0; stp < STEPS; ++stp) {
+    float v[C::XPOSE ? C::LPT : G];
+#pragma unroll
+    for (int tg = 0; tg < C::TPG; ++tg) {
+      const int tl = stp * C::STEP_TOK + tg * C::NG + gi;
+      const int tok = wb + tl;
+      const bool in = tl < TW && tok < cnt;
+      const int row = in ? tok : wb;      // any staged row; its data is masked below
+      float2 x2[8];
+      if constexpr (I8) {
+        uint4 w = *reinterpret_cast<const uint4*>(kb + row * ROWB + sub * 16);
+        if (!in) w = make_uint4(0u, 0u, 0u, 0u);
+        i8x4_to_f2x2(w.x ^ (in ? 0u : 0x80808080u), x2[0], x2[1]);
+        i8x4_to_f2x2(w.y ^ (in ? 0u : 0x80808080u), x2[2], x2[3]);
+        i8x4_to_f2x2(w.z ^ (in ? 0u : 0x80808080u), x2[4], x2[5]);
+        i8x4_to_f2x2(w.w ^ (in ? 0u : 0x80808080u), x2[6], x2[7]);
+      } else {
+        uint4 w0 = *reinterpret_cast<const uint4*>(kb + row * ROWB + sub * 32);
+        uint4 w1 = *reinterpret_cast<const uint4*>(kb + row * ROWB + sub * 32 + 16);
+        if (!in) {
+          w0 = make_uint4(0u, 0u, 0u, 0u);
+          w1 = w0;
+        }
+        x2[0] = h2_to_f2(w0.x); x2[1] = h2_to_f2(w0.y); x2[2] = h2_to_f2(w0.z); x2[3] = h2_to_f2(w0.w);
+        x2[4] = h2_to_f2(w1.x); x2[5] = h2_to_f2(w1.y); x2[6] = h2_to_f2(w1.z); x2[7] = h2_to_f2(w1.w);
+      }
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        float2 sa = make_float2(0.0f, 0.0f), sb2 = make_float2(0.0f, 0.0f);
+#pragma unroll
+        for (int i = 0; i < 8; i += 2) {
+          sa = __ffma2_rn(q2[g][i], x2[i], sa);
+          sb2 = __ffma2_rn(q2[g][i + 1], x2[i + 1], sb2);
+        }
+        const float2 t2 = __fadd2_rn(sa, sb2);
+        v[tg * G + g] = t2.x + t2.y;
+      }
+    }
+    float mine;
+    if constexpr (C::XPOSE) {
+#pragma unroll
+      for (int o = C::LPT / 2; o >= 1; o >>= 1) {
+        const bool upper = (sub & o) != 0;
+#pragma unroll
+        for (int k = 0; k < o; ++k) {
+          const float send = upper ? v[k] : v[k + o];
+          const float keep = upper ? v[k + o] : v[k];
+          v[k] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+      }
+      mine = v[0];                       // value index sub = (token t_own, head g_own)
+    } else {
+#pragma unroll
+      for (int o = 1; o < C::LPT; o <<= 1) {
+#pragma unroll
+        for (int g = 0; g < G; ++g) v[g] += __shfl_xor_sync(0xffffffffu, v[g], o);
+      }
+      mine = v[0];
+#pragma unroll
+      for (int g = 1; g < G; ++g) mine = (sub == g) ? v[g] : mine;
+    }
+    const int tl = stp * C::STEP_TOK + t_own * C::NG + gi;
+    const int tok = wb + tl;
+    const bool in_own = own && tl < TW && tok < cnt;
+    bool valid = in_own;
+    if constexpr (!COLD) valid = valid && reinterpret_cast<const int32_t*>(aux)[in_own ? tok : 0] >= 0;
+    const float kscale = I8 ? aux[in_own ? tok : 0] : 1.0f;
+    const float sg = mine * kscale;
+    if (valid) {
+      const int col = (COLD ? 0 : c.cap) + j0 + tok;
+      if (!kChecked || guard(col >= 0 && col < a.score_stride, c.err, kSiteAttnScore, s_id, col))
+        sc_base[(size_t)g_own * a.score_stride + col] = sg;
+    }
+    u_own[stp] = valid ? sg * kLog2e : -CUDART_INF_F;
+    tl_own[stp] = (own && tl < TW) ? tl : -1;
+    lmax = fmaxf(lmax, u_own[stp]);
+    if constexpr (!COLD) {
+      const uint32_t bal = __ballot_sync(0xffffffffu, valid && g_own == 0);
+      if (lane == 0) n_rows += __popc(bal);
+    }
+  }
+
+  // ---- running maximum: updated once per tile, only when it grows ----
+  float m_own = ws.m[0];
+#pragma unroll
+  for (int g = 1; g < G; ++g) m_own = (g_own == g) ? ws.m[g] : m_own;
+  if (__any_sync(0xffffffffu, lmax > m_own)) {
+    float l_scale = 1.0f;
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const float hm = warp_max(g_own == g ? lmax : -CUDART_INF_F);
+      if (hm > ws.m[g]) {
+        const float corr = exp2f(ws.m[g] - hm);
+#pragma unroll
+        for (int e = 0; e < E; ++e) ws.acc[g][e] = __fmul2_rn(ws.acc[g][e], make_float2(corr, corr));
+        if (g_own == g) l_scale = corr;
+        ws.m[g] = hm;
+      }
+    }
+    ws.l_own *= l_scale;
+    m_own = ws.m[0];
+#pragma unroll
+    for (int g = 1; g < G; ++g) m_own = (g_own == g) ? ws.m[g] : m_own;
+  }
+  // probabilities, head-major: ps[g * TW_MAX + token]; the V scale is folded in
+#pragma unroll
+  for (int stp = 0; stp < STEPS; ++stp) {
+    const float uu = u_own[stp];
+    const float p = uu == -CUDART_INF_F ? 0.0f : exp2f(uu - m_own);   // invalid tokens carry nothing
+    ws.l_own += p;
+    const int tl = tl_own[stp];
+    if (tl >= 0) {
+      const float vscale = (I8 && p != 0.0f) ? aux[C::TT_C + wb + tl] : 1.0f;
+      ps[g_own * C::TW_MAX + tl] = p * vscale;
+    }
+  }
+  const int nv = max(0, min(TW, cnt - wb));   // this warp's staged rows in the tile
+  if (COLD && lane == 0) n_rows += nv;
+  __syncwarp();
+
+  // ---- P.V over token pairs: lanes over the head dimension ----
+#pragma unroll
+  for (int pp = 0; pp < TW / 2; ++pp) {
+    const int t0 = 2 * pp, t1 = t0 + 1;
+    const bool in0 = t0 < nv, in1 = t1 < nv;
+    float2 x2[E];                     // (token t0, token t1) value pairs per dimension
+    if constexpr (I8) {
+      uint32_t w0, w1;
+      if constexpr (E == 4) {
+        w0 = *reinterpret_cast<const uint32_t*>(vb + (wb + (in0 ? t0 : 0)) * ROWB + lane * 4);
+        w1 = *reinterpret_cast<const uint32_t*>(vb + (wb + (in1 ? t1 : 0)) * ROWB + lane * 4);
+      } else {
+        w0 = *reinterpret_cast<const uint16_t*>(vb + (wb + (in0 ? t0 : 0)) * ROWB + lane * 2);
+        w1 = *reinterpret_cast<const uint16_t*>(vb + (wb + (in1 ? t1 : 0)) * ROWB + lane * 2);
+      }
+      const uint32_t u0 = in0 ? (w0 ^ 0x80808080u) : 0x80808080u;   // masked rows read as zeros
+      const uint32_t u1 = in1 ? (w1 ^ 0x80808080u) : 0x80808080u;
+      const float2 bias = make_float2(-8388736.0f, -8388736.0f);
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const uint32_t sel = 0x7540u + (uint32_t)e;    // byte e of the word into 2^23's mantissa
+        float2 f;
+        f.x = __uint_as_float(__byte_perm(u0, 0x4B000000u, sel));
+        f.y = __uint_as_float(__byte_perm(u1, 0x4B000000u, sel));
+        x2[e] = __fadd2_rn(f, bias);
+      }
+    } else {
+      uint32_t w0[E / 2], w1[E / 2];
+      if constexpr (E == 4) {
+        const uint2 a0 = *reinterpret_cast<const uint2*>(vb + (wb + (in0 ? t0 : 0)) * ROWB + lane * 8);
+        const uint2 a1 = *reinterpret_cast<const uint2*>(vb + (wb + (in1 ? t1 : 0)) * ROWB + lane * 8);
+        w0[0] = a0.x; w0[1] = a0.y; w1[0] = a1.x; w1[1] = a1.y;
+      } else {
+        w0[0] = *reinterpret_cast<const uint32_t*>(vb + (wb + (in0 ? t0 : 0)) * ROWB + lane * 4);
+        w1[0] = *reinterpret_cast<const uint32_t*>(vb + (wb + (in1 ? t1 : 0)) * ROWB + lane * 4);
+      }
+#pragma unroll
+      for (int k = 0; k < E / 2; ++k) {
+        const uint32_t a0 = in0 ? w0[k] : 0u, a1 = in1 ? w1[k] : 0u;
+        x2[2 * k] = h2_to_f2(__byte_perm(a0, a1, 0x5410));       // (t0 dim 2k,   t1 dim 2k)
+        x2[2 * k + 1] = h2_to_f2(__byte_perm(a0, a1, 0x7632));   // (t0 dim 2k+1, t1 dim 2k+1)
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const float2 p2 = *reinterpret_cast<const float2*>(ps + g * C::TW_MAX + t0);
+      const float2 pm = make_float2(in0 ? p2.x : 0.0f, in1 ? p2.y : 0.0f);
+#pragma unroll
+      for (int e = 0; e < E; ++e) ws.acc[g][e] = __ffma2_rn(pm, x2[e], ws.acc[g][e]);
+    }
+  }
+  __syncwarp();
+}
+
 template <int D, int G, bool CI8>
-__global__ void __launch_bounds__(160, (G >= 4 ? 2 : 3)) attn_kernel(Cache c, AttnLaunch a, int splits, int units,
+__global__ void __launch_bounds__(160, (G >= 4 ? CONFKV_G4_MINB : 3)) attn_kernel(Cache c, AttnLaunch a, int splits, int units,
                                                                   float qscale) {
   using C = Cfg<D, G, CI8>;
   extern __shared__ __align__(128) unsigned char smem[];
@@ -256,7 +485,8 @@ __global__ void __launch_bounds__(160, (G >= 4 ? 2 : 3)) attn_kernel(Cache c, At
 
   // -------------------------------- consumers --------------------------------
   const int sub = lane % C::LPT;       // which 16-dim slice of a row this lane scores
-  const int gi = lane / C::LPT;        // which token of a score step this lane's group takes
+  const bool own = C::XPOSE || sub < G;
+  const int g_own = C::XPOSE ? sub % G : (sub < G ? sub : 0);
   float* ps = ps_all + warp * C::TW_MAX * 8;
   volatile int* stop_snapshot = abort_flag + 1;
   int ctr = 0;
@@ -281,15 +511,14 @@ __global__ void __launch_bounds__(160, (G >= 4 ? 2 : 3)) attn_kernel(Cache c, At
         }
       }
     }
-    float m[G], lsum[G];
-    float2 acc[G][C::E / 2];
+    WarpState<D, G> ws;
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      m[g] = -CUDART_INF_F;
-      lsum[g] = 0.0f;
+      ws.m[g] = -CUDART_INF_F;
 #pragma unroll
-      for (int e = 0; e < C::E / 2; ++e) acc[g][e] = make_float2(0.0f, 0.0f);
+      for (int e = 0; e < C::E; ++e) ws.acc[g][e] = make_float2(0.0f, 0.0f);
     }
+    ws.l_own = 0.0f;
     unsigned long long n_rows_c = 0, n_rows_r = 0;
     float* sc_base = a.scores + (size_t)u.s * G * a.score_stride;
 
@@ -302,146 +531,29 @@ __global__ void __launch_bounds__(160, (G >= 4 ? 2 : 3)) attn_kernel(Cache c, At
       }
       if (*abort_flag) break;   // every consumer warp still reaches the merge barriers
       const unsigned char* sb = stages + st * C::STAGE_BYTES;
-      const bool cold = t < u.tiles_c;
-      const int tw = cold ? C::TW_C : C::TW_R;
-      const int j0 = cold ? t * C::TT_C : (t - u.tiles_c) * C::TT_R;
-      const int cnt = cold ? min(C::TT_C, u.n_cold - j0) : min(C::TT_R, c.W - j0);
-      const int wb = warp * tw;         // first token of this warp in the tile
-      uint32_t vmask = 0;               // tokens of this warp that are valid
-      const int steps = tw / C::NG;
-      // scores of this warp's tokens (log2 units); the maximum is updated once
-      // per tile so that every probability of the tile uses the same reference
-      float u2s[C::MAX_STEPS][G];
-      float vsc[C::MAX_STEPS];
-      bool up = false;
-#pragma unroll
-      for (int stp = 0; stp < C::MAX_STEPS; ++stp) {
-        if (stp >= steps) break;
-        const int tl = stp * C::NG + gi;      // token index within this warp's share
-        const int tok = wb + tl;              // token index within the tile
-        bool valid = tok < cnt;
-        if (!cold && valid) valid = reinterpret_cast<const int32_t*>(sb + 2 * C::KV_BYTES)[tok] >= 0;
-        float part[G];
-#pragma unroll
-        for (int g = 0; g < G; ++g) part[g] = 0.0f;
-        if (valid) {
-          float2 x2[8];
-          if (cold && CI8) {
-            const uint4 w = *reinterpret_cast<const uint4*>(sb + tok * D + sub * 16);
-            i8x4_to_f2x2(w.x, x2[0], x2[1]);
-            i8x4_to_f2x2(w.y, x2[2], x2[3]);
-            i8x4_to_f2x2(w.z, x2[4], x2[5]);
-            i8x4_to_f2x2(w.w, x2[6], x2[7]);
-          } else {
-            const uint4 w0 = *reinterpret_cast<const uint4*>(sb + tok * (2 * D) + sub * 32);
-            const uint4 w1 = *reinterpret_cast<const uint4*>(sb + tok * (2 * D) + sub * 32 + 16);
-            x2[0] = h2_to_f2(w0.x); x2[1] = h2_to_f2(w0.y); x2[2] = h2_to_f2(w0.z); x2[3] = h2_to_f2(w0.w);
-            x2[4] = h2_to_f2(w1.x); x2[5] = h2_to_f2(w1.y); x2[6] = h2_to_f2(w1.z); x2[7] = h2_to_f2(w1.w);
-          }
-#pragma unroll
-          for (int g = 0; g < G; ++g) {
-            float2 s2 = make_float2(0.0f, 0.0f);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) s2 = __ffma2_rn(q2[g][i], x2[i], s2);
-            part[g] = s2.x + s2.y;
-          }
-        }
-#pragma unroll
-        for (int o = 1; o < C::LPT; o <<= 1) {
-#pragma unroll
-          for (int g = 0; g < G; ++g) part[g] += __shfl_xor_sync(0xffffffffu, part[g], o);
-        }
-        const float kscale = (cold && CI8 && valid) ? reinterpret_cast<const float*>(sb + 2 * C::KV_BYTES)[tok] : 1.0f;
-        vsc[stp] = (cold && CI8 && valid) ? reinterpret_cast<const float*>(sb + 2 * C::KV_BYTES + C::TT_C * 4)[tok]
-                                          : 1.0f;
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const float sg = part[g] * kscale;
-          if (valid && sub == g) {
-            const int col = (cold ? 0 : c.cap) + j0 + tok;
-            if (!kChecked || guard(col >= 0 && col < a.score_stride, c.err, kSiteAttnScore, u.s, col))
-              sc_base[(size_t)g * a.score_stride + col] = sg;
-          }
-          u2s[stp][g] = valid ? sg * kLog2e : -CUDART_INF_F;
-          up |= u2s[stp][g] > m[g];
-        }
-        const uint32_t bal = __ballot_sync(0xffffffffu, valid && sub == 0);
-        // bit gi of the ballot (taken from lane gi*LPT) -> token tl = stp*NG + gi
-#pragma unroll
-        for (int k = 0; k < C::NG; ++k)
-          if (bal & (1u << (k * C::LPT))) vmask |= 1u << (stp * C::NG + k);
+      if (t < u.tiles_c) {
+        const int j0 = t * C::TT_C;
+        const int cnt = min(C::TT_C, u.n_cold - j0);
+        if constexpr (CI8)
+          consume_tile<D, G, CI8, kTileCold8>(c, a, sb, q2, ws, ps, sc_base, u.s, j0, cnt, warp, lane, n_rows_c);
+        else
+          consume_tile<D, G, CI8, kTileCold16>(c, a, sb, q2, ws, ps, sc_base, u.s, j0, cnt, warp, lane, n_rows_c);
+      } else {
+        const int j0 = (t - u.tiles_c) * C::TT_R;
+        const int cnt = min(C::TT_R, c.W - j0);
+        consume_tile<D, G, CI8, kTileRing>(c, a, sb, q2, ws, ps, sc_base, u.s, j0, cnt, warp, lane, n_rows_r);
       }
-      if (__any_sync(0xffffffffu, up)) {
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          float tmax = -CUDART_INF_F;
-#pragma unroll
-          for (int stp = 0; stp < C::MAX_STEPS; ++stp)
-            if (stp < steps) tmax = fmaxf(tmax, u2s[stp][g]);
-          const float nm = fmaxf(m[g], warp_max(tmax));
-          if (nm > m[g]) {
-            const float corr = exp2f(m[g] - nm);
-            lsum[g] *= corr;
-#pragma unroll
-            for (int e = 0; e < C::E / 2; ++e) acc[g][e] = __fmul2_rn(acc[g][e], make_float2(corr, corr));
-            m[g] = nm;
-          }
-        }
-      }
-#pragma unroll
-      for (int stp = 0; stp < C::MAX_STEPS; ++stp) {
-        if (stp >= steps) break;
-        const int tl = stp * C::NG + gi;
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const float u = u2s[stp][g];
-          const float p = u == -CUDART_INF_F ? 0.0f : exp2f(u - m[g]);   // invalid tokens carry nothing
-          lsum[g] += p;
-          if (sub == g) ps[tl * 8 + g] = p * vsc[stp];
-        }
-      }
-      if (lane == 0) {
-        if (cold) n_rows_c += __popc(vmask);
-        else n_rows_r += __popc(vmask);
-      }
-      __syncwarp();
-      // ---- P.V over this warp's tokens: lanes over the head dimension ----
-      uint32_t mk = vmask;
-      while (mk) {
-        const int tl = __ffs(mk) - 1;
-        mk &= mk - 1;
-        const int tok = wb + tl;
-        float2 x2[C::E / 2];
-        if (cold && CI8) {
-          if constexpr (C::E == 4) {
-            const uint32_t w = *reinterpret_cast<const uint32_t*>(sb + C::KV_BYTES + tok * D + lane * 4);
-            i8x4_to_f2x2(w, x2[0], x2[1]);
-          } else {
-            const uint32_t w = *reinterpret_cast<const uint16_t*>(sb + C::KV_BYTES + tok * D + lane * 2);
-            float2 hi;
-            i8x4_to_f2x2(w, x2[0], hi);
-          }
-        } else {
-          if constexpr (C::E == 4) {
-            const uint2 w = *reinterpret_cast<const uint2*>(sb + C::KV_BYTES + tok * (2 * D) + lane * 8);
-            x2[0] = h2_to_f2(w.x);
-            x2[1] = h2_to_f2(w.y);
-          } else {
-            const uint32_t w = *reinterpret_cast<const uint32_t*>(sb + C::KV_BYTES + tok * (2 * D) + lane * 4);
-            x2[0] = h2_to_f2(w);
-          }
-        }
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const float p = ps[tl * 8 + g];
-#pragma unroll
-          for (int e = 0; e < C::E / 2; ++e) acc[g][e] = __ffma2_rn(make_float2(p, p), x2[e], acc[g][e]);
-        }
-      }
-      __syncwarp();
       if (lane == 0) mbar_arrive(&empty[st]);
       ++ctr;
     }
+    // fold the (even token, odd token) halves of the P.V sums
+    float acc[G][C::E];
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+      for (int e = 0; e < C::E; ++e) acc[g][e] = ws.acc[g][e].x + ws.acc[g][e].y;
+    const float* m = ws.m;
+    const float l_own = ws.l_own;
 
     // ---- merge the four consumer warps of this unit ----
     float* mg = merge;                                  // [NCW][G] maxima
@@ -449,16 +561,13 @@ __global__ void __launch_bounds__(160, (G >= 4 ? 2 : 3)) attn_kernel(Cache c, At
     float* ag = merge + 2 * C::NCW * G;                 // [NCW][G][D] accumulators
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      const float ls = warp_sum(lsum[g]) * (1.0f / C::LPT);   // every lane of a group added the same p
+      const float ls = warp_sum((own && g_own == g) ? l_own : 0.0f);
       if (lane == 0) {
         mg[warp * G + g] = m[g];
         lg[warp * G + g] = ls;
       }
 #pragma unroll
-      for (int e = 0; e < C::E / 2; ++e) {
-        ag[(warp * G + g) * D + lane * C::E + 2 * e] = acc[g][e].x;
-        ag[(warp * G + g) * D + lane * C::E + 2 * e + 1] = acc[g][e].y;
-      }
+      for (int e = 0; e < C::E; ++e) ag[(warp * G + g) * D + lane * C::E + e] = acc[g][e];
     }
     if (lane == 0) {
       atomicAdd(&c.counters[kCntAttnInt8], CI8 ? n_rows_c : 0ull);

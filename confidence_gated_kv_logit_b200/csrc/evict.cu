@@ -104,27 +104,43 @@ __global__ void __launch_bounds__(NT) evict_kernel(Cache c, Policy pol, EvictLau
       return rank_key(pol, sc, pos, t);
     };
     const int span = n_cold + W;
-    const SelectResult sel = (e == 1) ? block_argmin<NT>(key, span, sm) : block_select_smallest<NT>(key, span, e, sm);
-
-    // victim bitmask of the cold region, and count
     uint32_t* vm = a.vmask + (size_t)s * a.mask_words;
-    const int words = (n_cold + 31) >> 5;
-    int ecold_here = 0;
-    for (int w = threadIdx.x; w < words; w += NT) {
-      uint32_t bits = 0;
-      for (int j = 0; j < 32; ++j) {
-        const int i = w * 32 + j;
-        if (i < n_cold && is_selected(key(i), sel)) bits |= 1u << j;
+    auto victim = [&](int i) -> bool { return (vm[i >> 5] >> (i & 31)) & 1u; };
+    if (e == 1 && !a.stable) {
+      // steady state: one victim; its index comes with the argmin, and at most
+      // one row (the last cold row) moves into its place
+      int vi;
+      block_argmin_idx<NT>(key, span, sm, &vi);
+      if (vi >= n_cold) {
+        if (threadIdx.x == 0) pos_r[vi - n_cold] = -1;
+      } else if (vi >= 0) {
+        const int last = n_cold - 1;
+        if (vi != last) {
+          for (int w = threadIdx.x; w < 2 * R::VEC; w += NT) move_cold_row<D, CI8>(c, s, last, vi, w);
+          moved = 1;
+        }
+        n_cold_new = n_cold - 1;
       }
-      vm[w] = bits;
-      ecold_here += __popc(bits);
+      __syncthreads();
+    } else {
+    const SelectResult sel = block_select_smallest<NT>(key, span, e, sm);
+
+    // victim bitmask of the cold region (one ballot per 32 tokens), and count
+    int ecold_here = 0;
+    for (int base = 0; base < n_cold; base += NT) {
+      const int i = base + (int)threadIdx.x;
+      const bool v = i < n_cold && is_selected(key(i), sel);
+      const unsigned bal = __ballot_sync(0xffffffffu, v);
+      if ((threadIdx.x & 31) == 0 && i < n_cold) {
+        vm[i >> 5] = bal;
+        ecold_here += __popc(bal);
+      }
     }
     // window victims free their slot (each thread reads and writes only its own slots)
     for (int slot = threadIdx.x; slot < W; slot += NT)
       if (is_selected(key(n_cold + slot), sel)) pos_r[slot] = -1;
     const int e_cold = block_sum_int<NT>(ecold_here, sm);   // includes a block barrier: vm is visible
     const int n_keep = n_cold - e_cold;
-    auto victim = [&](int i) -> bool { return (vm[i >> 5] >> (i & 31)) & 1u; };
 
     if (e_cold == 0) {
       // every victim was in the window ring: the cold region is unchanged
@@ -203,6 +219,7 @@ __global__ void __launch_bounds__(NT) evict_kernel(Cache c, Policy pol, EvictLau
       moved = block_sum_int<NT>(moved, sm);
     }
     n_cold_new = n_keep;
+    }
   }
 
   // the token that the next append would push out of the window becomes INT8

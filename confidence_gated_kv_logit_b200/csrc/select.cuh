@@ -14,6 +14,7 @@ struct SelectSmem {
   int rem, done;
   int warp_tot[NT / 32];
   unsigned long long wmin[NT / 32];
+  int widx[NT / 32];
   int next;
   int misc[4];
 };
@@ -104,6 +105,45 @@ __device__ SelectResult block_argmin(KeyFn kf, int n, SelectSmem<NT>& sm) {
   for (int i = 0; i < NT / 32; ++i) m = sm.wmin[i] < m ? sm.wmin[i] : m;
   __syncthreads();
   return SelectResult{m, ~0ull};
+}
+
+// Smallest key among kf(0..n-1) and the index that holds it (-1 if none).
+template <int NT, class KeyFn>
+__device__ unsigned long long block_argmin_idx(KeyFn kf, int n, SelectSmem<NT>& sm, int* idx_out) {
+  unsigned long long best = kNoKey;
+  int bi = -1;
+  for (int i = threadIdx.x; i < n; i += NT) {
+    const unsigned long long k = kf(i);
+    if (k < best) {
+      best = k;
+      bi = i;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+    if (other < best) {
+      best = other;
+      bi = oi;
+    }
+  }
+  if ((threadIdx.x & 31) == 0) {
+    sm.wmin[threadIdx.x >> 5] = best;
+    sm.widx[threadIdx.x >> 5] = bi;
+  }
+  __syncthreads();
+  unsigned long long m = kNoKey;
+  int mi = -1;
+#pragma unroll
+  for (int i = 0; i < NT / 32; ++i)
+    if (sm.wmin[i] < m) {
+      m = sm.wmin[i];
+      mi = sm.widx[i];
+    }
+  __syncthreads();
+  *idx_out = mi;
+  return m;
 }
 
 // The k smallest keys (1 <= k <= number of present keys), by MSD radix select

@@ -11,6 +11,7 @@ import numpy as np
 import pytest
 
 from oracle import quantize_row, dequantize_rows
+from oracle.quant import quantize_rows
 
 
 def _f32_nearest(fr: Fraction) -> float:
@@ -136,3 +137,14 @@ def test_pins_catch_planted_mistakes(kind):
 def test_unmutated_copy_passes():
     for pin in ALL_PINS:
         pin(_mutant("none"))
+
+
+def test_rows_equal_row_by_row():
+    rng = np.random.default_rng(8)
+    x = (rng.standard_normal((300, 128)) * rng.uniform(0.01, 20, size=(300, 1))).astype(np.float16)
+    x[17] = 0
+    x[40, :5] = [127, 2.5, 3.5, -2.5, -127]
+    codes, scales = quantize_rows(x)
+    for i in range(300):
+        c1, s1 = quantize_row(x[i])
+        assert np.array_equal(codes[i], c1) and scales[i] == s1, i

@@ -29,7 +29,7 @@ STATUS = {0: "OK", 1: "ERR_ARG", 2: "ERR_CAPACITY", 3: "ERR_STATE", 4: "ERR_NONF
 EXPORTED = ["confkv_default_params", "confkv_create", "confkv_destroy", "confkv_prefill",
             "confkv_confidence", "confkv_decode_attn", "confkv_evict_compact", "confkv_query",
             "confkv_export_segment", "confkv_last_error", "confkv_last_error_detail",
-            "confkv_profile_enable", "confkv_profile_read",
+            "confkv_profile_enable", "confkv_profile_read", "confkv_confidence_noalloc",
             "confkv_status_string", "confkv_version"]
 KERNEL_KINDS = ["confidence", "append", "attention", "combine", "ema", "evict", "prefill", "unused"]
 
@@ -87,6 +87,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.confkv_export_segment.argtypes = [P, I32, I32, I32, VP, ctypes.POINTER(ctypes.c_size_t)]
     lib.confkv_last_error.argtypes = [P, I32]
     lib.confkv_last_error_detail.argtypes = [P, ctypes.POINTER(ctypes.c_int32)]
+    lib.confkv_confidence_noalloc.argtypes = [ctypes.POINTER(Params), I32, VP, I32, I32, VP, VP, VP]
     lib.confkv_profile_enable.argtypes = [P, I32]
     lib.confkv_profile_read.argtypes = [P, ctypes.POINTER(Profile), I32]
     lib.confkv_status_string.argtypes = [ctypes.c_int]
@@ -136,6 +137,24 @@ def _stream(stream):
     import torch
     s = torch.cuda.current_stream() if stream is None else stream
     return ctypes.c_void_p(s.cuda_stream)
+
+
+def confidence_noalloc(logits, layers: int, c_out, budget_out, stream=None, **params):
+    """Confidence and per-layer budgets through confkv_confidence_noalloc: no
+    handle and no device allocation inside the library (for callers that
+    cannot allocate). Policy fields default as in confkv_default_params."""
+    import torch
+    B, V = logits.shape
+    p = default_params()
+    for k, v in params.items():
+        if not hasattr(p, k):
+            raise TypeError(f"unknown parameter {k}")
+        setattr(p, k, v)
+    lp = _ptr(logits, torch.float32, (B, V), "logits")
+    cp = _ptr(c_out, torch.float32, (B,), "c_out")
+    bp = _ptr(budget_out, torch.int32, (B, layers), "budget_out")
+    _check(load_library().confkv_confidence_noalloc(ctypes.byref(p), layers, lp, B, V, cp, bp, _stream(stream)),
+           "confkv_confidence_noalloc")
 
 
 class ConfKV:

@@ -229,6 +229,30 @@ typedef struct {
 CONFKV_API confkv_status confkv_profile_enable(confkv_handle* h, int32_t enable);
 CONFKV_API confkv_status confkv_profile_read(confkv_handle* h, confkv_profile* out, int32_t reset);
 
+/* Confidence and per-layer budgets without a handle and without allocating.
+ * The pages describe no counterpart: this entry point exists for callers that
+ * cannot allocate device memory, such as code running under an allocator
+ * that owns the whole device or a runtime that hands the library a fixed
+ * memory budget. It computes what confkv_confidence computes, for the gate,
+ * threshold, budgets and pyramid in *params (its other fields are ignored),
+ * for `layers` layers:
+ *   logits fp32 [batch][vocab], c_out fp32 [batch], budget_out int32
+ *   [batch][layers], all device memory owned by the caller (required).
+ * Its scratch is a fixed array inside the library (about 197 KB per device,
+ * held by every GPU that loads the library until the process exits), so:
+ *  - batch may be at most 256 and vocab at most 262144; larger sizes return
+ *    CONFKV_ERR_CAPACITY before anything runs;
+ *  - the first call on a device looks up the array's device address (a
+ *    host-side step, no allocation); make that first call before any stream
+ *    capture;
+ *  - every call shares the one array: calls that overlap on the GPU (on two
+ *    streams, or from two threads) race and give wrong results. Serialise them.
+ * It calls no cudaMalloc, cudaFree or allocating routine. A row with a NaN or
+ * Inf logit gets c = NaN and the larger budget; no error word is kept. */
+CONFKV_API confkv_status confkv_confidence_noalloc(const confkv_params* params, int32_t layers, const float* logits,
+                                                   int32_t batch, int32_t vocab, float* c_out, int32_t* budget_out,
+                                                   void* stream);
+
 /* Static description of a status code. */
 CONFKV_API const char* confkv_status_string(confkv_status s);
 

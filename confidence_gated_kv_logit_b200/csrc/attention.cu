@@ -216,25 +216,19 @@ __device__ __forceinline__ void consume_tile(const Cache& c, const AttnLaunch& a
     float v[C::XPOSE ? C::LPT : G];
 #pragma unroll
     for (int tg = 0; tg < C::TPG; ++tg) {
-      const int tl = stp * C::STEP_TOK + tg * C::NG + gi;
-      const int tok = wb + tl;
-      const bool in = tl < TW && tok < cnt;
-      const int row = in ? tok : wb;      // any staged row; its data is masked below
+      // rows past the tile's end are staged rows of earlier tiles (or zeros): their
+      // scores are computed and discarded below, never masked per element
+      const int row = wb + min(stp * C::STEP_TOK + tg * C::NG + gi, TW - 1);
       float2 x2[8];
       if constexpr (I8) {
-        uint4 w = *reinterpret_cast<const uint4*>(kb + row * ROWB + sub * 16);
-        if (!in) w = make_uint4(0u, 0u, 0u, 0u);
-        i8x4_to_f2x2(w.x ^ (in ? 0u : 0x80808080u), x2[0], x2[1]);
-        i8x4_to_f2x2(w.y ^ (in ? 0u : 0x80808080u), x2[2], x2[3]);
-        i8x4_to_f2x2(w.z ^ (in ? 0u : 0x80808080u), x2[4], x2[5]);
-        i8x4_to_f2x2(w.w ^ (in ? 0u : 0x80808080u), x2[6], x2[7]);
+        const uint4 w = *reinterpret_cast<const uint4*>(kb + row * ROWB + sub * 16);
+        i8x4_to_f2x2(w.x, x2[0], x2[1]);
+        i8x4_to_f2x2(w.y, x2[2], x2[3]);
+        i8x4_to_f2x2(w.z, x2[4], x2[5]);
+        i8x4_to_f2x2(w.w, x2[6], x2[7]);
       } else {
-        uint4 w0 = *reinterpret_cast<const uint4*>(kb + row * ROWB + sub * 32);
-        uint4 w1 = *reinterpret_cast<const uint4*>(kb + row * ROWB + sub * 32 + 16);
-        if (!in) {
-          w0 = make_uint4(0u, 0u, 0u, 0u);
-          w1 = w0;
-        }
+        const uint4 w0 = *reinterpret_cast<const uint4*>(kb + row * ROWB + sub * 32);
+        const uint4 w1 = *reinterpret_cast<const uint4*>(kb + row * ROWB + sub * 32 + 16);
         x2[0] = h2_to_f2(w0.x); x2[1] = h2_to_f2(w0.y); x2[2] = h2_to_f2(w0.z); x2[3] = h2_to_f2(w0.w);
         x2[4] = h2_to_f2(w1.x); x2[5] = h2_to_f2(w1.y); x2[6] = h2_to_f2(w1.z); x2[7] = h2_to_f2(w1.w);
       }
@@ -286,7 +280,7 @@ __device__ __forceinline__ void consume_tile(const Cache& c, const AttnLaunch& a
         sc_base[(size_t)g_own * a.score_stride + col] = sg;
     }
     u_own[stp] = valid ? sg * kLog2e : -CUDART_INF_F;
-    tl_own[stp] = (own && tl < TW) ? tl : -1;
+    tl_own[stp] = (own && tl < TW) ? tl : -1;   // every token < TW gets a probability (0 if invalid)
     lmax = fmaxf(lmax, u_own[stp]);
     if constexpr (!COLD) {
       const uint32_t bal = __ballot_sync(0xffffffffu, valid && g_own == 0);
@@ -328,27 +322,25 @@ __device__ __forceinline__ void consume_tile(const Cache& c, const AttnLaunch& a
       ps[g_own * C::TW_MAX + tl] = p * vscale;
     }
   }
-  const int nv = max(0, min(TW, cnt - wb));   // this warp's staged rows in the tile
-  if (COLD && lane == 0) n_rows += nv;
+  if (COLD && lane == 0) n_rows += max(0, min(TW, cnt - wb));   // this warp's valid rows
   __syncwarp();
 
   // ---- P.V over token pairs: lanes over the head dimension ----
+  // Rows past the tile's end carry probability 0 and finite staged data.
 #pragma unroll
   for (int pp = 0; pp < TW / 2; ++pp) {
-    const int t0 = 2 * pp, t1 = t0 + 1;
-    const bool in0 = t0 < nv, in1 = t1 < nv;
-    float2 x2[E];                     // (token t0, token t1) value pairs per dimension
+    const int t0 = 2 * pp;
+    float2 x2[E];                     // (token t0, token t0+1) value pairs per dimension
     if constexpr (I8) {
       uint32_t w0, w1;
       if constexpr (E == 4) {
-        w0 = *reinterpret_cast<const uint32_t*>(vb + (wb + (in0 ? t0 : 0)) * ROWB + lane * 4);
-        w1 = *reinterpret_cast<const uint32_t*>(vb + (wb + (in1 ? t1 : 0)) * ROWB + lane * 4);
+        w0 = *reinterpret_cast<const uint32_t*>(vb + (wb + t0) * ROWB + lane * 4);
+        w1 = *reinterpret_cast<const uint32_t*>(vb + (wb + t0 + 1) * ROWB + lane * 4);
       } else {
-        w0 = *reinterpret_cast<const uint16_t*>(vb + (wb + (in0 ? t0 : 0)) * ROWB + lane * 2);
-        w1 = *reinterpret_cast<const uint16_t*>(vb + (wb + (in1 ? t1 : 0)) * ROWB + lane * 2);
+        w0 = *reinterpret_cast<const uint16_t*>(vb + (wb + t0) * ROWB + lane * 2);
+        w1 = *reinterpret_cast<const uint16_t*>(vb + (wb + t0 + 1) * ROWB + lane * 2);
       }
-      const uint32_t u0 = in0 ? (w0 ^ 0x80808080u) : 0x80808080u;   // masked rows read as zeros
-      const uint32_t u1 = in1 ? (w1 ^ 0x80808080u) : 0x80808080u;
+      const uint32_t u0 = w0 ^ 0x80808080u, u1 = w1 ^ 0x80808080u;
       const float2 bias = make_float2(-8388736.0f, -8388736.0f);
 #pragma unroll
       for (int e = 0; e < E; ++e) {
@@ -361,26 +353,24 @@ __device__ __forceinline__ void consume_tile(const Cache& c, const AttnLaunch& a
     } else {
       uint32_t w0[E / 2], w1[E / 2];
       if constexpr (E == 4) {
-        const uint2 a0 = *reinterpret_cast<const uint2*>(vb + (wb + (in0 ? t0 : 0)) * ROWB + lane * 8);
-        const uint2 a1 = *reinterpret_cast<const uint2*>(vb + (wb + (in1 ? t1 : 0)) * ROWB + lane * 8);
+        const uint2 a0 = *reinterpret_cast<const uint2*>(vb + (wb + t0) * ROWB + lane * 8);
+        const uint2 a1 = *reinterpret_cast<const uint2*>(vb + (wb + t0 + 1) * ROWB + lane * 8);
         w0[0] = a0.x; w0[1] = a0.y; w1[0] = a1.x; w1[1] = a1.y;
       } else {
-        w0[0] = *reinterpret_cast<const uint32_t*>(vb + (wb + (in0 ? t0 : 0)) * ROWB + lane * 4);
-        w1[0] = *reinterpret_cast<const uint32_t*>(vb + (wb + (in1 ? t1 : 0)) * ROWB + lane * 4);
+        w0[0] = *reinterpret_cast<const uint32_t*>(vb + (wb + t0) * ROWB + lane * 4);
+        w1[0] = *reinterpret_cast<const uint32_t*>(vb + (wb + t0 + 1) * ROWB + lane * 4);
       }
 #pragma unroll
       for (int k = 0; k < E / 2; ++k) {
-        const uint32_t a0 = in0 ? w0[k] : 0u, a1 = in1 ? w1[k] : 0u;
-        x2[2 * k] = h2_to_f2(__byte_perm(a0, a1, 0x5410));       // (t0 dim 2k,   t1 dim 2k)
-        x2[2 * k + 1] = h2_to_f2(__byte_perm(a0, a1, 0x7632));   // (t0 dim 2k+1, t1 dim 2k+1)
+        x2[2 * k] = h2_to_f2(__byte_perm(w0[k], w1[k], 0x5410));       // (t0 dim 2k,   t1 dim 2k)
+        x2[2 * k + 1] = h2_to_f2(__byte_perm(w0[k], w1[k], 0x7632));   // (t0 dim 2k+1, t1 dim 2k+1)
       }
     }
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       const float2 p2 = *reinterpret_cast<const float2*>(ps + g * C::TW_MAX + t0);
-      const float2 pm = make_float2(in0 ? p2.x : 0.0f, in1 ? p2.y : 0.0f);
 #pragma unroll
-      for (int e = 0; e < E; ++e) ws.acc[g][e] = __ffma2_rn(pm, x2[e], ws.acc[g][e]);
+      for (int e = 0; e < E; ++e) ws.acc[g][e] = __ffma2_rn(p2, x2[e], ws.acc[g][e]);
     }
   }
   __syncwarp();
@@ -400,6 +390,11 @@ __global__ void __launch_bounds__(160, (G >= 4 ? CONFKV_G4_MINB : 3)) attn_kerne
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // Zero the stage ring once: rows a tile does not fill then hold zeros or an
+  // earlier tile's finite data, so the tile loops need no per-row masks.
+  for (int i = threadIdx.x; i < C::NSTAGE * C::STAGE_BYTES / 16; i += blockDim.x)
+    reinterpret_cast<uint4*>(stages)[i] = make_uint4(0u, 0u, 0u, 0u);
+  fence_proxy_async_shared();
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NSTAGE; ++i) {
       mbar_init(&full[i], 1);

@@ -46,14 +46,26 @@ class Pair:
         return [(l, b, h) for l in range(self.L) for b in range(self.B) for h in range(self.Hkv)]
 
     def prefill(self, lens, T=None):
+        """Prefill every layer on the GPU; the oracle ingests the host copies of
+        the tracked segments only (the others are never simulated)."""
         T = T or max(max(lens), 1)
         fixed = self.p.mode == "fixed"
         for l in range(self.L):
             k, v = synth.prefill_kv(self.B, self.Hkv, T, self.D, self.gen, self.dev)
             pr = synth.priorities((self.B, self.Hkv, T), self.gen, self.dev) if fixed else None
             self.gpu.prefill(k, v, lens, layer=l, priority=pr)
-            self.orc.prefill(l, k.cpu().numpy(), v.cpu().numpy(), lens,
-                             None if pr is None else pr.cpu().numpy())
+            keys = [key for key in self.segments() if key[0] == l]
+            if keys:
+                kh = np.zeros((self.B, self.Hkv, T, self.D), np.float16)
+                vh = np.zeros_like(kh)
+                ph = np.zeros((self.B, self.Hkv, T), np.float32) if fixed else None
+                for (_, b, h) in keys:
+                    kh[b, h] = k[b, h].cpu().numpy()
+                    vh[b, h] = v[b, h].cpu().numpy()
+                    if fixed:
+                        ph[b, h] = pr[b, h].cpu().numpy()
+                self.orc.prefill(l, kh, vh, lens, ph)
+            del k, v, pr
         torch.cuda.synchronize()
 
     def step_inputs(self, V):
@@ -122,3 +134,39 @@ def assert_segment_equal(g: dict, o, key, exact_scores=True):
         assert np.array_equal(g["score_src"].view(np.uint32), o.score_src.astype(np.float32).view(np.uint32)), key
     else:
         np.testing.assert_allclose(g["score_src"], o.score_src, rtol=RTOL_EMA, atol=ATOL_EMA, err_msg=str(key))
+
+
+def run_synced(pair: Pair, lens, steps, V, T=None, check_every=1):
+    """Step-synchronised parity run: per step, attention (tolerance), EMA
+    (tolerance), confidence and budgets, then -- with the oracle given the
+    GPU's EMA -- the kept set, compaction and INT8 codes bit for bit."""
+    pair.prefill(lens, T)
+    for key in pair.segments():
+        assert_segment_equal(pair.gpu_segment(*key), pair.orc.segment(*key), key)
+    worst = 0.0
+    for step in range(steps):
+        check = (step % check_every == 0) or step == steps - 1
+        q, kn, vn, pn, logits = pair.step_inputs(V)
+        out_g, lse_g, out_o, lse_o = pair.attn(q, kn, vn, pn)
+        for (l, b, h) in pair.segments():
+            sl = slice(h * pair.orc.G, (h + 1) * pair.orc.G)
+            err = float(np.abs(out_g[l, b, sl] - out_o[l, b, sl]).max())
+            worst = max(worst, err)
+            assert err <= ATOL_OUT, (step, l, b, h, err)
+            assert np.abs(lse_g[l, b, sl] - lse_o[l, b, sl]).max() <= ATOL_LSE
+            if check:
+                assert_segment_equal(pair.gpu_segment(l, b, h), pair.orc.segment(l, b, h), (step, l, b, h),
+                                     exact_scores=pair.p.mode == "fixed")
+        if logits is not None:
+            c_g, bud_g, c_o, bud_o, override = pair.confidence(logits)
+            assert np.abs(c_g - c_o).max() <= ATOL_C, (c_g, c_o)
+            assert np.array_equal(bud_g, bud_o), (step, bud_g, bud_o, override)
+        pair.sync_scores_from_gpu()
+        pair.gpu.evict_compact()
+        for l in range(pair.L):
+            pair.orc.evict_compact(l)
+        if check:
+            for key in pair.segments():
+                assert_segment_equal(pair.gpu_segment(*key), pair.orc.segment(*key), (step,) + key)
+    assert pair.gpu.last_error() == 0
+    return worst

@@ -11,39 +11,9 @@ import pytest
 import torch
 
 from oracle.segment import Params
-from parity_util import (ATOL_C, ATOL_LSE, ATOL_OUT, Pair, assert_segment_equal)
+from parity_util import ATOL_C, Pair, run_synced
 
 pytestmark = pytest.mark.gpu
-
-
-def run_synced(pair: Pair, lens, steps, V, T=None):
-    pair.prefill(lens, T)
-    for key in pair.segments():
-        assert_segment_equal(pair.gpu_segment(*key), pair.orc.segment(*key), key)
-    worst = 0.0
-    for step in range(steps):
-        q, kn, vn, pn, logits = pair.step_inputs(V)
-        out_g, lse_g, out_o, lse_o = pair.attn(q, kn, vn, pn)
-        for (l, b, h) in pair.segments():
-            sl = slice(h * pair.orc.G, (h + 1) * pair.orc.G)
-            err = np.abs(out_g[l, b, sl] - out_o[l, b, sl]).max()
-            worst = max(worst, err)
-            assert err <= ATOL_OUT, (step, l, b, h, err)
-            assert np.abs(lse_g[l, b, sl] - lse_o[l, b, sl]).max() <= ATOL_LSE
-            assert_segment_equal(pair.gpu_segment(l, b, h), pair.orc.segment(l, b, h), (step, l, b, h),
-                                 exact_scores=pair.p.mode == "fixed")
-        if logits is not None:
-            c_g, bud_g, c_o, bud_o, override = pair.confidence(logits)
-            assert np.abs(c_g - c_o).max() <= ATOL_C, (c_g, c_o)
-            assert np.array_equal(bud_g, bud_o), (step, bud_g, bud_o, override)
-        pair.sync_scores_from_gpu()
-        pair.gpu.evict_compact()
-        for l in range(pair.L):
-            pair.orc.evict_compact(l)
-        for key in pair.segments():
-            assert_segment_equal(pair.gpu_segment(*key), pair.orc.segment(*key), (step,) + key)
-    assert pair.gpu.last_error() == 0
-    return worst
 
 
 def test_config1_tiny_synced():

@@ -128,30 +128,40 @@ __global__ void __launch_bounds__(NT) confidence_kernel(ConfLaunch a, Policy pol
     is_last = (prev == (unsigned)a.cpr - 1u);
   }
   __syncthreads();
-  if (!is_last || threadIdx.x != 0) return;
+  if (!is_last) return;
 
-  // last CTA of this row: merge every partial (read past L1) and finish
+  // last CTA of this row: every thread loads one partial (read past L1), then
+  // the same warp and block merge as above
   __threadfence();
   ConfPartial acc;
-  {
-    const ConfPartial* pp = a.part + (size_t)row * a.cpr;
-    acc.m = __ldcg(&pp[0].m);
-    acc.S = __ldcg(&pp[0].S);
-    acc.T = __ldcg(&pp[0].T);
-    acc.top1 = __ldcg(&pp[0].top1);
-    acc.top2 = __ldcg(&pp[0].top2);
-    acc.bad = __ldcg(&pp[0].bad);
-    for (int k = 1; k < a.cpr; ++k) {
-      ConfPartial q;
-      q.m = __ldcg(&pp[k].m);
-      q.S = __ldcg(&pp[k].S);
-      q.T = __ldcg(&pp[k].T);
-      q.top1 = __ldcg(&pp[k].top1);
-      q.top2 = __ldcg(&pp[k].top2);
-      q.bad = __ldcg(&pp[k].bad);
-      merge(acc, q);
-    }
+  acc.m = -CUDART_INF_F;
+  acc.S = 0.0f;
+  acc.T = 0.0f;
+  acc.top1 = -CUDART_INF_F;
+  acc.top2 = -CUDART_INF_F;
+  acc.bad = 0;
+  const ConfPartial* pp = a.part + (size_t)row * a.cpr;
+  for (int k = threadIdx.x; k < a.cpr; k += NT) {
+    ConfPartial q;
+    q.m = __ldcg(&pp[k].m);
+    q.S = __ldcg(&pp[k].S);
+    q.T = __ldcg(&pp[k].T);
+    q.top1 = __ldcg(&pp[k].top1);
+    q.top2 = __ldcg(&pp[k].top2);
+    q.bad = __ldcg(&pp[k].bad);
+    merge(acc, q);
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const ConfPartial q = shfl_partial(acc, o);
+    merge(acc, q);
+  }
+  __syncthreads();   // every thread is done with wpart from the first merge
+  if ((threadIdx.x & 31) == 0) wpart[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x != 0) return;
+  acc = wpart[0];
+  for (int w = 1; w < NT / 32; ++w) merge(acc, wpart[w]);
   a.tickets[row] = 0u;   // ready for the next launch
 
   float c;

@@ -18,7 +18,7 @@ namespace {
 
 constexpr uint32_t kMagic = 0xC0F1C0DEu;
 constexpr uint32_t kDead = 0xDEADC0DEu;
-constexpr int kMaxCpr = 32;
+constexpr int kMaxCpr = 128;   // CTAs per logit row (one per ~2048 logits)
 
 struct Buffers {
   std::vector<void*> ptrs;
@@ -403,7 +403,7 @@ confkv_status confkv_confidence(confkv_handle* h, const float* logits, int32_t b
   a.L = h->L;
   a.part = h->cpart;
   a.tickets = h->tickets;
-  a.cpr = std::max(1, std::min(kMaxCpr, (vocab + 8191) / 8192));
+  a.cpr = std::max(1, std::min(kMaxCpr, (vocab + 2047) / 2048));
   a.c_ws = h->c_ws;
   a.budget_ws = h->budget;
   a.c_out = c_out;

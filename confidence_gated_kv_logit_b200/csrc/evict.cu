@@ -57,16 +57,253 @@ __device__ __forceinline__ void move_cold_row(const Cache& c, int s, int src, in
   }
 }
 
-template <int D, bool CI8>
-__global__ void __launch_bounds__(NT) evict_kernel(Cache c, Policy pol, EvictLaunch a) {
-  using R = Rows<D, CI8>;
-  __shared__ SelectSmem<NT> sm;
-  __shared__ int list_h[NT];
-  __shared__ int list_m[NT];
-  __shared__ __align__(16) unsigned char stage[16384];
-  __shared__ int stage_meta[4][64];
+constexpr int kSegsPerCta = NT / 32;     // the fast path gives each warp one segment
+constexpr int kWarpMaxVictims = 4;        // victims one warp handles; more go to the whole CTA
 
-  const int item = blockIdx.x;
+struct WarpCounts {
+  int scanned = 0, moved = 0, requant = 0;
+};
+
+__device__ __forceinline__ unsigned long long warp_min_u64(unsigned long long v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const unsigned long long w = __shfl_xor_sync(0xffffffffu, v, o);
+    v = w < v ? w : v;
+  }
+  return v;
+}
+
+// Keeps the kWarpMaxVictims smallest (key, index) pairs seen by this lane, ascending.
+struct LaneBest {
+  unsigned long long k[kWarpMaxVictims];
+  int i[kWarpMaxVictims];
+  __device__ __forceinline__ void init() {
+#pragma unroll
+    for (int j = 0; j < kWarpMaxVictims; ++j) {
+      k[j] = kNoKey;
+      i[j] = -1;
+    }
+  }
+  __device__ __forceinline__ void offer(unsigned long long key, int idx) {
+    if (key < k[kWarpMaxVictims - 1]) {
+      k[kWarpMaxVictims - 1] = key;
+      i[kWarpMaxVictims - 1] = idx;
+#pragma unroll
+      for (int j = kWarpMaxVictims - 1; j > 0; --j) {
+        if (k[j] < k[j - 1]) {
+          const unsigned long long tk = k[j];
+          k[j] = k[j - 1];
+          k[j - 1] = tk;
+          const int ti = i[j];
+          i[j] = i[j - 1];
+          i[j - 1] = ti;
+        }
+      }
+    }
+  }
+  __device__ __forceinline__ void pop() {
+#pragma unroll
+    for (int j = 0; j < kWarpMaxVictims - 1; ++j) {
+      k[j] = k[j + 1];
+      i[j] = i[j + 1];
+    }
+    k[kWarpMaxVictims - 1] = kNoKey;
+    i[kWarpMaxVictims - 1] = -1;
+  }
+};
+
+// One segment by one warp. Handles the common decode step (at most
+// kWarpMaxVictims victims, hole-fill order) with shuffles only: one pass over
+// the keys in which every lane keeps its own few smallest, a warp merge of the
+// lane lists, the same hole-fill pairing as the whole-CTA path (the k-th
+// hole below the new end gets the k-th survivor above it) and the conversion
+// of the token leaving the window. Returns false, having written nothing,
+// when the segment needs the whole-CTA path (more victims, or stable order).
+template <int D, bool CI8>
+__device__ bool evict_segment_warp(const Cache& c, const Policy& pol, const EvictLaunch& a, int item, int lane,
+                                   WarpCounts* wc) {
+  using R = Rows<D, CI8>;
+  int l, b, h;
+  const int s = seg_of(c, a.r, item, &l, &b, &h);
+  const int t = c.next_pos[s] - 1;
+  const int n_cold = c.n_cold[s];
+  const int W = c.W;
+  if (!(n_cold >= 0 && n_cold <= c.cap && t >= -1)) {
+    if (lane == 0) record_violation(c.err, kSiteEvictSeg, s, n_cold);
+    return true;
+  }
+  const int32_t* pos_c = c.pos_c + (size_t)s * c.cap;
+  const float* sc_c = c.sc_c + (size_t)s * c.cap;
+  int32_t* pos_r = c.pos_r + (size_t)s * c.Wst;
+  const float* sc_r = c.sc_r + (size_t)s * c.Wst;
+
+  int ring_here = 0;
+  for (int slot = lane; slot < W; slot += 32) ring_here += pos_r[slot] >= 0;
+  const int n = n_cold + __reduce_add_sync(0xffffffffu, ring_here);
+  const int budget_eff = pol.mode == 1 ? pol.fixed_budget
+                                       : max(a.budget[(size_t)b * c.L + l], pol.P + pol.n_sink);
+  const int e = n - budget_eff;
+  int n_cold_new = n_cold;
+  int moved = 0;
+
+  if (e > 0 && t >= 0) {
+    if (e > kWarpMaxVictims || a.stable) return false;
+    auto rank = [&](int pos, float sc) -> unsigned long long {
+      if (t - pos < pol.P || pos < pol.n_sink) return kNoKey;
+      return rank_key(pol, sc, pos, t);
+    };
+    LaneBest best;
+    best.init();
+    // cold region, four tokens per lane in flight
+    int i = lane;
+    for (; i + 96 < n_cold; i += 128) {
+      int p4[4];
+      float s4[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        p4[u] = pos_c[i + 32 * u];
+        s4[u] = sc_c[i + 32 * u];
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) best.offer(rank(p4[u], s4[u]), i + 32 * u);
+    }
+    for (; i < n_cold; i += 32) best.offer(rank(pos_c[i], sc_c[i]), i);
+    // window ring (empty slots hold position -1)
+    for (int slot = lane; slot < W; slot += 32) {
+      const int pos = pos_r[slot];
+      if (pos >= 0) best.offer(rank(pos, sc_r[slot]), n_cold + slot);
+    }
+
+    // merge: the e smallest keys of the segment, one per round; cold victims
+    // are collected in v[0..ec) (the same values in every lane)
+    int v[kWarpMaxVictims];
+    int ec = 0;
+#pragma unroll
+    for (int j = 0; j < kWarpMaxVictims; ++j) {
+      v[j] = -1;
+      if (j < e) {
+        const unsigned long long m = warp_min_u64(best.k[0]);
+        if (m != kNoKey) {
+          const unsigned own = __ballot_sync(0xffffffffu, best.k[0] == m);
+          const int src = __ffs(own) - 1;
+          const int vi = __shfl_sync(0xffffffffu, best.i[0], src);
+          if (lane == src) best.pop();
+          if (vi >= n_cold) {
+            if (lane == 0) pos_r[vi - n_cold] = -1;
+          } else {
+#pragma unroll
+            for (int q = 0; q <= j; ++q)
+              if (q == ec) v[q] = vi;
+            ++ec;
+          }
+        }
+      }
+    }
+
+    if (ec > 0) {
+      const int n_keep = n_cold - ec;
+      // holes: victims below n_keep; movers: survivors in [n_keep, n_cold).
+      // Both lists ascending; pair p moves mover p into hole p.
+      int hole_of[kWarpMaxVictims], mover_of[kWarpMaxVictims];
+#pragma unroll
+      for (int p = 0; p < kWarpMaxVictims; ++p) hole_of[p] = mover_of[p] = -1;
+#pragma unroll
+      for (int q = 0; q < kWarpMaxVictims; ++q) {
+        if (q < ec && v[q] < n_keep) {
+          int r = 0;
+#pragma unroll
+          for (int q2 = 0; q2 < kWarpMaxVictims; ++q2) r += (q2 < ec && v[q2] < n_keep && v[q2] < v[q]) ? 1 : 0;
+#pragma unroll
+          for (int p = 0; p < kWarpMaxVictims; ++p)
+            if (p == r) hole_of[p] = v[q];
+        }
+      }
+      int np = 0;
+#pragma unroll
+      for (int d = 0; d < kWarpMaxVictims; ++d) {
+        const int idx = n_keep + d;
+        bool is_victim = false;
+#pragma unroll
+        for (int q = 0; q < kWarpMaxVictims; ++q) is_victim |= (q < ec && v[q] == idx);
+        if (d < ec && !is_victim) {
+#pragma unroll
+          for (int p = 0; p < kWarpMaxVictims; ++p)
+            if (p == np) mover_of[p] = idx;
+          ++np;
+        }
+      }
+      for (int w = lane; w < np * 2 * R::VEC; w += 32) {
+        const int p = w / (2 * R::VEC);
+        int src = -1, dst = -1;
+#pragma unroll
+        for (int q = 0; q < kWarpMaxVictims; ++q)
+          if (q == p) {
+            src = mover_of[q];
+            dst = hole_of[q];
+          }
+        if (kChecked && !guard(dst >= 0 && dst < n_keep && src >= n_keep && src < n_cold, c.err, kSiteEvictPair,
+                               s, src))
+          continue;
+        move_cold_row<D, CI8>(c, s, src, dst, w - p * 2 * R::VEC);
+      }
+      moved = np;
+      n_cold_new = n_keep;
+    }
+  }
+  __syncwarp();   // ring slots freed and rows moved above are visible to every lane
+
+  // the token that the next append would push out of the window becomes INT8
+  int requant = 0;
+  const int leaving = t + 1 - W;
+  if (CI8 && W > 0 && leaving >= 0) {
+    const int slot = (t + 1) % W;
+    const size_t rs = (size_t)s * c.Wst + slot;
+    if (c.pos_r[rs] == leaving) {
+      const int idx = n_cold_new;
+      if (idx >= c.cap || idx < 0) {
+        if (lane == 0) record_violation(c.err, kSiteEvictRequant, s, idx);
+      } else {
+        const size_t cs = (size_t)s * c.cap + idx;
+        warp_quantize_row<D>(c.kr + rs * D, c.k8 + cs * D, c.ks + cs, lane);
+        warp_quantize_row<D>(c.vr + rs * D, c.v8 + cs * D, c.vs + cs, lane);
+        __syncwarp();
+        if (lane == 0) {
+          c.pos_c[cs] = leaving;
+          c.sc_c[cs] = c.sc_r[rs];
+          c.pos_r[rs] = -1;
+        }
+        n_cold_new = idx + 1;
+        requant = 1;
+      }
+    }
+  }
+  if (lane == 0) c.n_cold[s] = n_cold_new;
+  wc->scanned = n;
+  wc->moved = moved;
+  wc->requant = requant;
+  return true;
+}
+
+struct EvictSmem {
+  SelectSmem<NT> sm;
+  int list_h[NT];
+  int list_m[NT];
+  __align__(16) unsigned char stage[16384];
+  int stage_meta[4][64];
+};
+
+// One segment by the whole CTA (all NT threads call it with the same item):
+// any number of victims, both compaction orders.
+template <int D, bool CI8>
+__device__ void evict_segment_block(const Cache& c, const Policy& pol, const EvictLaunch& a, int item,
+                                    EvictSmem& es) {
+  using R = Rows<D, CI8>;
+  SelectSmem<NT>& sm = es.sm;
+  int* list_h = es.list_h;
+  int* list_m = es.list_m;
+  unsigned char* stage = es.stage;
+  int (*stage_meta)[64] = es.stage_meta;
+
   int l, b, h;
   const int s = seg_of(c, a.r, item, &l, &b, &h);
   const int t = c.next_pos[s] - 1;
@@ -255,11 +492,45 @@ __global__ void __launch_bounds__(NT) evict_kernel(Cache c, Policy pol, EvictLau
 }
 
 template <int D, bool CI8>
+__global__ void __launch_bounds__(NT, 4) evict_kernel(Cache c, Policy pol, EvictLaunch a, int items) {
+  __shared__ EvictSmem es;
+  __shared__ int slow_items[kSegsPerCta];
+  __shared__ int n_slow;
+  __shared__ unsigned long long cnt[3];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) n_slow = 0;
+  if (threadIdx.x < 3) cnt[threadIdx.x] = 0;
+  __syncthreads();
+  const int item = blockIdx.x * kSegsPerCta + warp;
+  if (item < items) {
+    WarpCounts wc;
+    if (!evict_segment_warp<D, CI8>(c, pol, a, item, lane, &wc)) {
+      if (lane == 0) slow_items[atomicAdd(&n_slow, 1)] = item;
+    } else if (lane == 0) {
+      if (wc.scanned) atomicAdd(&cnt[0], (unsigned long long)wc.scanned);
+      if (wc.moved) atomicAdd(&cnt[1], (unsigned long long)wc.moved);
+      if (wc.requant) atomicAdd(&cnt[2], (unsigned long long)wc.requant);
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    if (cnt[0]) atomicAdd(&c.counters[kCntEvictScanned], cnt[0]);
+    if (cnt[1]) atomicAdd(&c.counters[kCntMovedRows], cnt[1]);
+    if (cnt[2]) atomicAdd(&c.counters[kCntRequant], cnt[2]);
+  }
+  const int ns = n_slow;
+  for (int k = 0; k < ns; ++k) {
+    __syncthreads();   // the previous segment's shared-memory use is over
+    evict_segment_block<D, CI8>(c, pol, a, slow_items[k], es);
+  }
+}
+
+template <int D, bool CI8>
 cudaError_t run(const Cache& c, const Policy& pol, const EvictLaunch& a, cudaStream_t st, long long* launches,
                 Prof* prof) {
   const int items = a.r.items(c.Hkv);
   ProfScope ps(prof, kKEvict, st);
-  evict_kernel<D, CI8><<<items, NT, 0, st>>>(c, pol, a);
+  evict_kernel<D, CI8><<<(items + kSegsPerCta - 1) / kSegsPerCta, NT, 0, st>>>(c, pol, a, items);
   ++*launches;
   return cudaGetLastError();
 }

@@ -3,32 +3,43 @@
 // FP16/INT8 storage; CONF-KV post, implementation note: INT8 is dequantised
 // inside the attention kernel).
 //
-//   append_kernel     : writes the new token into the FP16 window ring (or the
-//                       cold region when INT8 is off)
-//   attn_kernel       : persistent, warp-specialised split-K attention. One
-//                       producer warp streams K/V tiles and their scales or
-//                       positions into a 3-stage shared-memory ring with 1-D
-//                       TMA bulk copies; four consumer warps compute scores,
-//                       an online softmax with lazy rescaling, and P.V with the
-//                       INT8 codes converted in registers (byte permute into
-//                       the fp32 mantissa) and packed f32x2 FMAs. The per-token
-//                       scale of K multiplies the dot product; the scale of V
-//                       is folded into the probability. No tensor cores: one
-//                       query row per KV head is a GEMV.
-//   combine_kernel    : merges split partials into out and lse
-//   ema_kernel        : second pass with the saved log-sum-exp: per token the
-//                       mean over the G query heads of exp(s - lse) enters the
-//                       attention-mass EMA (CONF-KV post, pseudo-code update_ema)
+//   append_kernel  : writes the new token into the FP16 window ring (or the
+//                    cold region when INT8 is off) and prepares the segment's
+//                    query operands for the tensor cores
+//   attn_kernel    : persistent, warp-specialised split-K attention. One
+//                    producer warp streams K/V tiles with their scales or
+//                    positions into a shared-memory ring with 1-D TMA bulk
+//                    copies; four consumer warps run both contractions on the
+//                    tensor cores (mma.sync) and keep one online softmax per
+//                    CTA.
+//   combine_kernel : merges split partials into out and lse
+//   ema_kernel     : second pass with the saved log-sum-exp: per token the
+//                    mean over the G query heads of exp(s - lse) enters the
+//                    attention-mass EMA (CONF-KV post, pseudo-code update_ema)
+//
+// Arithmetic. The G query heads of one KV head (padded to GP = 4 or 8) make
+// both products small GEMMs:
+//   * INT8 scores S = K8 . q: each query head is written as an integer
+//     Q = q * 2^(27-ex) (ex from the head's max |q|; exact for every fp16 q
+//     above 2^-16 of the maximum) and split into four balanced base-128 digit
+//     planes, so one s8 x s8 MMA with exact int32 accumulation per plane gives
+//     S exactly; the planes are recombined in fp32 and scaled by the token's K
+//     scale and the head's 2^(ex-27)/sqrt(D).
+//   * INT8 P.V: the probabilities times the token's V scale, P' = p * vs, are
+//     written as 31-bit integers relative to the tile's largest V scale and
+//     split into four byte planes (u8 x s8 MMA, exact int32 per tile), then
+//     folded into fp32 accumulators with weights 2^(8k - E).
+//   * FP16 tiles: K and q are fp16, so S comes from an f16 MMA with fp32
+//     accumulation; for P.V each probability is split into fp16 hi + lo
+//     (about 22 significant bits) and multiplied with fp16 V on the f16 MMA.
+// The V codes are stored dimension-major in blocks of 32 tokens so that the
+// token axis (the reduction axis of P.V) is contiguous per dimension.
 #include <math_constants.h>
 
 #include "common.cuh"
 #include "kernels.h"
+#include "mma.cuh"
 #include "tma.cuh"
-
-// CTAs per SM the register budget of the G >= 4 attention kernels targets.
-#ifndef CONFKV_G4_MINB
-#define CONFKV_G4_MINB 2
-#endif
 
 namespace confkv {
 
@@ -37,26 +48,128 @@ namespace {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
+// 2^k for -126 <= k <= 127
+__device__ __forceinline__ float pow2i(int k) { return __int_as_float((k + 127) << 23); }
+
+// Exponent ex with v in [2^(ex-1), 2^ex) for a normal v > 0; 0 for v = 0.
+__device__ __forceinline__ int exp_of(float v) {
+  return v > 0.0f ? (int)((__float_as_uint(v) >> 23) & 0xffu) - 126 : 0;
+}
+
+template <int N>
+__device__ __forceinline__ float sel(const float (&v)[N], int i) {
+  float r = 1.0f;
+#pragma unroll
+  for (int k = 0; k < N; ++k) r = (i == k) ? v[k] : r;
+  return r;
+}
+
+// ---------------------------------------------------------------------------
+// Prepared query operands of one segment (written by append_kernel):
+//   I8 : B fragments of the int8 score MMA, [kb][nb][lane] x 2 words. Column
+//        n of n-block nb is head n/2 + 4*(nb/2), digit plane 2*(nb%2) + n%2.
+//   H  : B fragments of the f16 score MMA, [ks][lane] x 2 words, column = head.
+//   CQ : per head, 2^(ex-27) / sqrt(D) (the int8 scores' scale).
+// ---------------------------------------------------------------------------
+template <int D, int GP>
+struct QF {
+  static constexpr int KB = D / 32, KS = D / 16, NB = GP / 2;
+  static constexpr int I8_OFF = 0;
+  static constexpr int H_OFF = KB * NB * 32 * 8;
+  static constexpr int CQ_OFF = H_OFF + KS * 32 * 8;
+  static constexpr int BYTES = (CQ_OFF + GP * 4 + 255) / 256 * 256;
+};
+
+// Digit `plane` (0..3, least significant first) of the balanced base-128
+// expansion Q = d0 + 128 d1 + 128^2 d2 + 128^3 d3, |d_k| <= 64, |Q| < 2^27.
+__device__ __forceinline__ int q_digit(int Q, int plane) {
+  int d = 0;
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+    d = ((Q + 64) & 127) - 64;
+    if (k == plane) return d;
+    Q = (Q - d) >> 7;
+  }
+  return Q;
+}
+
+template <int D, int GP>
+__device__ __forceinline__ void prepare_query(const Cache& c, const AttnLaunch& a, int s, int l, int b, int h,
+                                              int lane, float qscale) {
+  using Q = QF<D, GP>;
+  const int G = c.G;
+  const __half* qb = a.q + ((size_t)((l - a.r.l0) * a.r.B + b) * c.Hq + (size_t)h * G) * D;
+  unsigned char* out = a.qfrag + (size_t)s * a.qf_stride;
+  float scl[GP];
+#pragma unroll
+  for (int hh = 0; hh < GP; ++hh) {
+    float mx = 0.0f;
+    if (hh < G) {
+#pragma unroll
+      for (int e = 0; e < D / 32; ++e) mx = fmaxf(mx, fabsf(__half2float(qb[(size_t)hh * D + lane * (D / 32) + e])));
+    }
+    mx = warp_max(mx);
+    const int ex = exp_of(mx);
+    scl[hh] = mx > 0.0f ? pow2i(27 - ex) : 1.0f;
+    if (lane == 0) reinterpret_cast<float*>(out + Q::CQ_OFF)[hh] = mx > 0.0f ? qscale * pow2i(ex - 27) : 0.0f;
+  }
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int kb = 0; kb < Q::KB; ++kb) {
+#pragma unroll
+    for (int nb = 0; nb < Q::NB; ++nb) {
+      const int hh = g / 2 + 4 * (nb / 2);
+      const int plane = 2 * (nb % 2) + (g % 2);
+      const float sc = sel(scl, hh);
+      uint32_t r[2];
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int d0 = kb * 32 + half * 16 + 4 * t;
+        uint32_t pk = 0;
+        if (hh < G) {
+          const uint2 w = *reinterpret_cast<const uint2*>(qb + (size_t)hh * D + d0);
+          const float2 f01 = h2_to_f2(w.x), f23 = h2_to_f2(w.y);
+          const float qv[4] = {f01.x, f01.y, f23.x, f23.y};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) pk |= (uint32_t)(q_digit(__float2int_rn(qv[e] * sc), plane) & 0xff) << (8 * e);
+        }
+        r[half] = pk;
+      }
+      reinterpret_cast<uint2*>(out + Q::I8_OFF)[(kb * Q::NB + nb) * 32 + lane] = make_uint2(r[0], r[1]);
+    }
+  }
+#pragma unroll
+  for (int ks = 0; ks < Q::KS; ++ks) {
+    uint32_t r0 = 0, r1 = 0;
+    if (g < G) {
+      r0 = *reinterpret_cast<const uint32_t*>(qb + (size_t)g * D + ks * 16 + 2 * t);
+      r1 = *reinterpret_cast<const uint32_t*>(qb + (size_t)g * D + ks * 16 + 8 + 2 * t);
+    }
+    reinterpret_cast<uint2*>(out + Q::H_OFF)[ks * 32 + lane] = make_uint2(r0, r1);
+  }
+}
+
 // ---------------------------------------------------------------------------
 // append: one warp per segment. If the window slot of the new position still
 // holds a token (a caller skipped eviction), that token is converted to INT8
-// first, exactly as eviction would have done.
+// first, exactly as eviction would have done. Then the segment's query
+// operands are prepared.
 // ---------------------------------------------------------------------------
-template <int D>
-__global__ void __launch_bounds__(256) append_kernel(Cache c, Range r, const __half* __restrict__ k_new,
-                                                     const __half* __restrict__ v_new,
-                                                     const float* __restrict__ prio_new, int fixed_mode) {
+template <int D, int GP>
+__global__ void __launch_bounds__(256) append_kernel(Cache c, AttnLaunch a, int fixed_mode, float qscale) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
+  const Range r = a.r;
   if (warp >= r.items(c.Hkv)) return;
   int l, b, h;
   const int s = seg_of(c, r, warp, &l, &b, &h);
   const int t = c.next_pos[s];
   if (!guard(t >= 0 && c.n_cold[s] >= 0 && c.n_cold[s] <= c.cap, c.err, kSiteAppendSeg, s, t)) return;
   const size_t in_row = ((size_t)((l - r.l0) * r.B + b) * c.Hkv + h);
-  const __half* kn = k_new + in_row * D;
-  const __half* vn = v_new + in_row * D;
-  const float sc_new = fixed_mode ? prio_new[in_row] : 0.0f;
+  const __half* kn = a.k_new + in_row * D;
+  const __half* vn = a.v_new + in_row * D;
+  const float sc_new = fixed_mode ? a.prio_new[in_row] : 0.0f;
+  uint32_t w[D / 64];
   if (c.W > 0) {
     const int slot = t % c.W;
     const size_t rs = (size_t)s * c.Wst + slot;
@@ -67,10 +180,9 @@ __global__ void __launch_bounds__(256) append_kernel(Cache c, Range r, const __h
         if (lane == 0) set_error(c.err, kErrDevice);
         return;
       }
-      const size_t cs = (size_t)s * c.cap + idx;
-      warp_quantize_row<D>(c.kr + rs * D, c.k8 + cs * D, c.ks + cs, lane);
-      warp_quantize_row<D>(c.vr + rs * D, c.v8 + cs * D, c.vs + cs, lane);
+      warp_requant<D>(c, s, slot, idx, lane);
       if (lane == 0) {
+        const size_t cs = (size_t)s * c.cap + idx;
         c.pos_c[cs] = old;
         c.sc_c[cs] = c.sc_r[rs];
         c.n_cold[s] = idx + 1;
@@ -78,8 +190,10 @@ __global__ void __launch_bounds__(256) append_kernel(Cache c, Range r, const __h
       }
       __syncwarp();
     }
-    warp_copy_row_h<D>(kn, c.kr + rs * D, lane);
-    warp_copy_row_h<D>(vn, c.vr + rs * D, lane);
+    row_load_plain<D>(kn, lane, w);
+    row_store_h<D>(c.kr + (size_t)s * c.Wst * D, slot, lane, w);
+    row_load_plain<D>(vn, lane, w);
+    row_store_h<D>(c.vr + (size_t)s * c.Wst * D, slot, lane, w);
     if (lane == 0) {
       c.pos_r[rs] = t;
       c.sc_r[rs] = sc_new;
@@ -91,8 +205,10 @@ __global__ void __launch_bounds__(256) append_kernel(Cache c, Range r, const __h
       return;
     }
     const size_t cs = (size_t)s * c.cap + idx;
-    warp_copy_row_h<D>(kn, c.kc + cs * D, lane);
-    warp_copy_row_h<D>(vn, c.vc + cs * D, lane);
+    row_load_plain<D>(kn, lane, w);
+    row_store_h<D>(c.kc + (size_t)s * c.cap * D, idx, lane, w);
+    row_load_plain<D>(vn, lane, w);
+    row_store_h<D>(c.vc + (size_t)s * c.cap * D, idx, lane, w);
     if (lane == 0) {
       c.pos_c[cs] = t;
       c.sc_c[cs] = sc_new;
@@ -100,45 +216,37 @@ __global__ void __launch_bounds__(256) append_kernel(Cache c, Range r, const __h
     }
   }
   if (lane == 0) c.next_pos[s] = t + 1;
+  prepare_query<D, GP>(c, a, s, l, b, h, lane, qscale);
 }
 
 // ---------------------------------------------------------------------------
 // attention
 // ---------------------------------------------------------------------------
-template <int D, int G, bool CI8>
+template <int D, int GP, bool CI8>
 struct Cfg {
-  static constexpr int LPT = D / 16;              // lanes per token in the score phase (16 dims each)
-  static constexpr int NG = 32 / LPT;             // tokens per warp per score step
-  static constexpr int E = D / 32;                // dims per lane in the value phase
-  static constexpr int ROWB_C = CI8 ? D : 2 * D;  // bytes of one cold row
-  static constexpr int ROWB_R = 2 * D;            // bytes of one window row
-  static constexpr int KV_BYTES = 8192;           // bytes of K (and of V) per stage
-  static constexpr int TT_C = KV_BYTES / ROWB_C;  // tokens per cold tile
-  static constexpr int TT_R = KV_BYTES / ROWB_R;  // tokens per window tile
-  static constexpr int NCW = 4;                   // consumer warps
-  static constexpr int TW_C = TT_C / NCW;         // tokens per consumer warp per tile
-  static constexpr int TW_R = TT_R / NCW;
-  static constexpr int TW_MAX = TW_C > TW_R ? TW_C : TW_R;
-  // Score reduction across the LPT lanes of a token: when G divides LPT, each
-  // lane group scores TPG = LPT/G tokens at once and a transposed (reduce-
-  // scatter) butterfly leaves exactly one (token, head) score in every lane;
-  // otherwise one token per group and a plain butterfly, lanes sub < G keep
-  // one head each.
-  static constexpr bool XPOSE = (LPT % G) == 0;
-  static constexpr int TPG = XPOSE ? LPT / G : 1;
-  static constexpr int STEP_TOK = NG * TPG;       // tokens per warp per score step
-  static constexpr int SPT_C = (TW_C + STEP_TOK - 1) / STEP_TOK;
-  static constexpr int SPT_R = (TW_R + STEP_TOK - 1) / STEP_TOK;
-  static constexpr int MAX_STEPS = SPT_C > SPT_R ? SPT_C : SPT_R;
-  static constexpr int MINB = G >= 4 ? CONFKV_G4_MINB : 3;   // CTAs per SM the register budget is sized for
-  static constexpr int NSTAGE = MINB == 2 ? 4 : 3;
-  static constexpr int AUX_BYTES = 2 * (TT_C > TT_R ? TT_C : TT_R) * 4;
-  static constexpr int STAGE_BYTES = 2 * KV_BYTES + AUX_BYTES;
-  static constexpr int PS_BYTES = NCW * TW_MAX * 8 * 4;          // probabilities [8 heads][TW_MAX] per warp
-  static constexpr int MERGE_BYTES = NCW * G * (D + 2) * 4;
-  static constexpr int SMEM_BYTES = NSTAGE * STAGE_BYTES + PS_BYTES + MERGE_BYTES + 2 * NSTAGE * 8 + 16;
-  static_assert(G <= LPT, "at most head_dim/16 query heads per KV head");
-  static_assert(TW_MAX <= 32, "a warp's share of a tile is at most 32 tokens");
+  static constexpr int NCW = 4;                 // consumer warps
+  static constexpr int TTC = CI8 ? 128 : 64;    // tokens per cold tile
+  static constexpr int TTR = 64;                // tokens per window tile
+  static constexpr int KVB = 128 * D;           // bytes of K (and of V) per stage, either kind
+  static constexpr int AUXB = 1024;             // K and V scales (int8) or positions (window)
+  static constexpr int STAGE = 2 * KVB + AUXB;
+  static constexpr int NSTAGE = D == 128 ? 3 : 4;
+  static constexpr int KB = D / 32;             // k-blocks of the int8 score MMA
+  static constexpr int KS = D / 16;             // k-steps of the f16 score MMA
+  static constexpr int NB = GP / 2;             // n-blocks of the int8 score MMA (GP heads x 4 planes)
+  static constexpr int MB = GP / 4;             // 16-row blocks of the P.V rows
+  static constexpr int NBW = D / 32;            // 8-dimension n-blocks of P.V per consumer warp
+  static constexpr int HPL = GP / 4;            // heads per lane in the int8 score layout
+  static constexpr int PS_OFF = NSTAGE * STAGE;
+  static constexpr int PS_BYTES = NCW * GP * 32 * 4;
+  static constexpr int FB_OFF = PS_OFF + PS_BYTES;
+  static constexpr int FB_ONE = 4 * MB * 32;    // uint4 per buffer
+  static constexpr int FB_BYTES = 2 * FB_ONE * 16;
+  static constexpr int WM_OFF = FB_OFF + FB_BYTES;
+  static constexpr int LS_OFF = WM_OFF + NCW * GP * 4;
+  static constexpr int BAR_OFF = LS_OFF + NCW * GP * 4;
+  static constexpr int FLAG_OFF = BAR_OFF + 2 * NSTAGE * 8;
+  static constexpr int SMEM = FLAG_OFF + 16;
 };
 
 struct Unit {
@@ -147,9 +255,9 @@ struct Unit {
   int tiles_c, t0, t1;
 };
 
-template <int D, int G, bool CI8>
+template <int D, int GP, bool CI8>
 __device__ __forceinline__ Unit make_unit(const Cache& c, const Range& r, int splits, int unit) {
-  using C = Cfg<D, G, CI8>;
+  using C = Cfg<D, GP, CI8>;
   Unit u;
   const int item = unit / splits;
   const int split = unit - item * splits;
@@ -162,8 +270,8 @@ __device__ __forceinline__ Unit make_unit(const Cache& c, const Range& r, int sp
     u.t0 = u.t1 = 0;
     return u;
   }
-  u.tiles_c = (u.n_cold + C::TT_C - 1) / C::TT_C;
-  const int tiles_r = (c.W + C::TT_R - 1) / C::TT_R;
+  u.tiles_c = (u.n_cold + C::TTC - 1) / C::TTC;
+  const int tiles_r = (c.W + C::TTR - 1) / C::TTR;
   const int tiles = u.tiles_c + tiles_r;
   const int per = (tiles + splits - 1) / splits;
   u.t0 = min(tiles, split * per);
@@ -171,228 +279,373 @@ __device__ __forceinline__ Unit make_unit(const Cache& c, const Range& r, int sp
   return u;
 }
 
-
-// Per-warp online-softmax state of one unit.
-template <int D, int G>
-struct WarpState {
-  float m[G];                // running maximum per head (log2 units), uniform in the warp
-  float2 acc[G][D / 32];     // P.V partial sums: .x over even tokens, .y over odd tokens of a pair
-  float l_own;               // this lane's share of the softmax sum of its own head
+// Online-softmax state of one unit, shared by the four consumer warps: the
+// maxima m (log2 units) are the same in every lane. acc holds this lane's
+// rows of the P.V accumulator: rows g and g+8 of each 16-row block, where
+// GP = 4: row r is head r % 4 (int8 digit plane r / 4, or fp16 hi/lo part);
+// GP = 8: row r of block mb is head r % 8 (plane 2 mb + r / 8, or hi/lo in
+// block 0). A head's output is the sum of its rows. lp8 / lp16 are this
+// lane's shares of the softmax sums of the heads it scores in the int8
+// layout (t + 4j) and in the fp16 layout (2t, 2t+1).
+template <int D, int GP>
+struct SoftmaxState {
+  float m[GP];
+  float acc[GP / 4][D / 32][4];
+  float lp8[GP / 4];
+  float lp16[2];
 };
 
-enum TileKind { kTileCold8 = 0, kTileCold16 = 1, kTileRing = 2 };
-
-// One warp's share of one staged tile: scores (with the lane-group reduction),
-// the once-per-tile maximum update, probabilities, then P.V over token pairs.
-// Loops have compile-time trip counts; rows outside the tile are loaded
-// predicated to zero instead of branching.
-template <int D, int G, bool CI8, int KIND>
-__device__ __forceinline__ void consume_tile(const Cache& c, const AttnLaunch& a, const unsigned char* sb,
-                                             const float2 (&q2)[G][8], WarpState<D, G>& ws, float* ps,
-                                             float* sc_base, int s_id, int j0, int cnt, int warp, int lane,
-                                             unsigned long long& n_rows) {
-  using C = Cfg<D, G, CI8>;
-  constexpr bool COLD = KIND != kTileRing;
-  constexpr bool I8 = KIND == kTileCold8;
-  constexpr int TW = COLD ? C::TW_C : C::TW_R;
-  constexpr int ROWB = I8 ? D : 2 * D;
-  constexpr int STEPS = (TW + C::STEP_TOK - 1) / C::STEP_TOK;
-  constexpr int E = D / 32;
-  const int sub = lane % C::LPT;
-  const int gi = lane / C::LPT;
-  const bool own = C::XPOSE || sub < G;
-  const int g_own = C::XPOSE ? sub % G : (sub < G ? sub : 0);
-  const int t_own = C::XPOSE ? sub / G : 0;
-  const int wb = warp * TW;
-  const float* aux = reinterpret_cast<const float*>(sb + 2 * C::KV_BYTES);
-  const unsigned char* kb = sb;
-  const unsigned char* vb = sb + C::KV_BYTES;
-
-  float u_own[STEPS];
-  int tl_own[STEPS];
-  float lmax = -CUDART_INF_F;
+// New running maxima from the four warps' tile maxima; rescale when they grow.
+template <int D, int GP>
+__device__ __forceinline__ void update_max(SoftmaxState<D, GP>& st, const float* wmax, int lane) {
+  float mn[GP];
+  bool grow = false;
 #pragma unroll
-  for (int stp = 0; stp < STEPS; ++stp) {
-    float v[C::XPOSE ? C::LPT : G];
+  for (int h = 0; h < GP; ++h) {
+    float v = st.m[h];
 #pragma unroll
-    for (int tg = 0; tg < C::TPG; ++tg) {
-      // rows past the tile's end are staged rows of earlier tiles (or zeros): their
-      // scores are computed and discarded below, never masked per element
-      const int row = wb + min(stp * C::STEP_TOK + tg * C::NG + gi, TW - 1);
-      float2 x2[8];
-      if constexpr (I8) {
-        const uint4 w = *reinterpret_cast<const uint4*>(kb + row * ROWB + sub * 16);
-        i8x4_to_f2x2(w.x, x2[0], x2[1]);
-        i8x4_to_f2x2(w.y, x2[2], x2[3]);
-        i8x4_to_f2x2(w.z, x2[4], x2[5]);
-        i8x4_to_f2x2(w.w, x2[6], x2[7]);
-      } else {
-        const uint4 w0 = *reinterpret_cast<const uint4*>(kb + row * ROWB + sub * 32);
-        const uint4 w1 = *reinterpret_cast<const uint4*>(kb + row * ROWB + sub * 32 + 16);
-        x2[0] = h2_to_f2(w0.x); x2[1] = h2_to_f2(w0.y); x2[2] = h2_to_f2(w0.z); x2[3] = h2_to_f2(w0.w);
-        x2[4] = h2_to_f2(w1.x); x2[5] = h2_to_f2(w1.y); x2[6] = h2_to_f2(w1.z); x2[7] = h2_to_f2(w1.w);
-      }
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        float2 sa = make_float2(0.0f, 0.0f), sb2 = make_float2(0.0f, 0.0f);
-#pragma unroll
-        for (int i = 0; i < 8; i += 2) {
-          sa = __ffma2_rn(q2[g][i], x2[i], sa);
-          sb2 = __ffma2_rn(q2[g][i + 1], x2[i + 1], sb2);
-        }
-        const float2 t2 = __fadd2_rn(sa, sb2);
-        v[tg * G + g] = t2.x + t2.y;
-      }
-    }
-    float mine;
-    if constexpr (C::XPOSE) {
-#pragma unroll
-      for (int o = C::LPT / 2; o >= 1; o >>= 1) {
-        const bool upper = (sub & o) != 0;
-#pragma unroll
-        for (int k = 0; k < o; ++k) {
-          const float send = upper ? v[k] : v[k + o];
-          const float keep = upper ? v[k + o] : v[k];
-          v[k] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-        }
-      }
-      mine = v[0];                       // value index sub = (token t_own, head g_own)
-    } else {
-#pragma unroll
-      for (int o = 1; o < C::LPT; o <<= 1) {
-#pragma unroll
-        for (int g = 0; g < G; ++g) v[g] += __shfl_xor_sync(0xffffffffu, v[g], o);
-      }
-      mine = v[0];
-#pragma unroll
-      for (int g = 1; g < G; ++g) mine = (sub == g) ? v[g] : mine;
-    }
-    const int tl = stp * C::STEP_TOK + t_own * C::NG + gi;
-    const int tok = wb + tl;
-    const bool in_own = own && tl < TW && tok < cnt;
-    bool valid = in_own;
-    if constexpr (!COLD) valid = valid && reinterpret_cast<const int32_t*>(aux)[in_own ? tok : 0] >= 0;
-    const float kscale = I8 ? aux[in_own ? tok : 0] : 1.0f;
-    const float sg = mine * kscale;
-    if (valid) {
-      const int col = (COLD ? 0 : c.cap) + j0 + tok;
-      if (!kChecked || guard(col >= 0 && col < a.score_stride, c.err, kSiteAttnScore, s_id, col))
-        sc_base[(size_t)g_own * a.score_stride + col] = sg;
-    }
-    u_own[stp] = valid ? sg * kLog2e : -CUDART_INF_F;
-    tl_own[stp] = (own && tl < TW) ? tl : -1;   // every token < TW gets a probability (0 if invalid)
-    lmax = fmaxf(lmax, u_own[stp]);
-    if constexpr (!COLD) {
-      const uint32_t bal = __ballot_sync(0xffffffffu, valid && g_own == 0);
-      if (lane == 0) n_rows += __popc(bal);
-    }
+    for (int w = 0; w < 4; ++w) v = fmaxf(v, wmax[w * GP + h]);
+    mn[h] = v;
+    grow |= v > st.m[h];
   }
-
-  // ---- running maximum: updated once per tile, only when it grows ----
-  float m_own = ws.m[0];
+  if (grow) {
+    const int g = lane >> 2, t = lane & 3;
+    float corr[GP];
 #pragma unroll
-  for (int g = 1; g < G; ++g) m_own = (g_own == g) ? ws.m[g] : m_own;
-  if (__any_sync(0xffffffffu, lmax > m_own)) {
-    float l_scale = 1.0f;
+    for (int h = 0; h < GP; ++h) corr[h] = mn[h] > st.m[h] ? exp2f(st.m[h] - mn[h]) : 1.0f;
+    const float ca = sel(corr, GP == 4 ? (g & 3) : g);
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float hm = warp_max(g_own == g ? lmax : -CUDART_INF_F);
-      if (hm > ws.m[g]) {
-        const float corr = exp2f(ws.m[g] - hm);
+    for (int mb = 0; mb < GP / 4; ++mb)
 #pragma unroll
-        for (int e = 0; e < E; ++e) ws.acc[g][e] = __fmul2_rn(ws.acc[g][e], make_float2(corr, corr));
-        if (g_own == g) l_scale = corr;
-        ws.m[g] = hm;
-      }
-    }
-    ws.l_own *= l_scale;
-    m_own = ws.m[0];
+      for (int nb = 0; nb < D / 32; ++nb)
 #pragma unroll
-    for (int g = 1; g < G; ++g) m_own = (g_own == g) ? ws.m[g] : m_own;
+        for (int k = 0; k < 4; ++k) st.acc[mb][nb][k] *= ca;
+#pragma unroll
+    for (int j = 0; j < GP / 4; ++j) st.lp8[j] *= sel(corr, t + 4 * j);
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) st.lp16[cc] *= sel(corr, 2 * t + cc);
+#pragma unroll
+    for (int h = 0; h < GP; ++h) st.m[h] = mn[h];
   }
-  // probabilities, head-major: ps[g * TW_MAX + token]; the V scale is folded in
-#pragma unroll
-  for (int stp = 0; stp < STEPS; ++stp) {
-    const float uu = u_own[stp];
-    const float p = uu == -CUDART_INF_F ? 0.0f : exp2f(uu - m_own);   // invalid tokens carry nothing
-    ws.l_own += p;
-    const int tl = tl_own[stp];
-    if (tl >= 0) {
-      const float vscale = (I8 && p != 0.0f) ? aux[C::TT_C + wb + tl] : 1.0f;
-      ps[g_own * C::TW_MAX + tl] = p * vscale;
-    }
-  }
-  if (COLD && lane == 0) n_rows += max(0, min(TW, cnt - wb));   // this warp's valid rows
-  __syncwarp();
-
-  // ---- P.V over token pairs: lanes over the head dimension ----
-  // Rows past the tile's end carry probability 0 and finite staged data.
-#pragma unroll
-  for (int pp = 0; pp < TW / 2; ++pp) {
-    const int t0 = 2 * pp;
-    float2 x2[E];                     // (token t0, token t0+1) value pairs per dimension
-    if constexpr (I8) {
-      uint32_t w0, w1;
-      if constexpr (E == 4) {
-        w0 = *reinterpret_cast<const uint32_t*>(vb + (wb + t0) * ROWB + lane * 4);
-        w1 = *reinterpret_cast<const uint32_t*>(vb + (wb + t0 + 1) * ROWB + lane * 4);
-      } else {
-        w0 = *reinterpret_cast<const uint16_t*>(vb + (wb + t0) * ROWB + lane * 2);
-        w1 = *reinterpret_cast<const uint16_t*>(vb + (wb + t0 + 1) * ROWB + lane * 2);
-      }
-      const uint32_t u0 = w0 ^ 0x80808080u, u1 = w1 ^ 0x80808080u;
-      const float2 bias = make_float2(-8388736.0f, -8388736.0f);
-#pragma unroll
-      for (int e = 0; e < E; ++e) {
-        const uint32_t sel = 0x7540u + (uint32_t)e;    // byte e of the word into 2^23's mantissa
-        float2 f;
-        f.x = __uint_as_float(__byte_perm(u0, 0x4B000000u, sel));
-        f.y = __uint_as_float(__byte_perm(u1, 0x4B000000u, sel));
-        x2[e] = __fadd2_rn(f, bias);
-      }
-    } else {
-      uint32_t w0[E / 2], w1[E / 2];
-      if constexpr (E == 4) {
-        const uint2 a0 = *reinterpret_cast<const uint2*>(vb + (wb + t0) * ROWB + lane * 8);
-        const uint2 a1 = *reinterpret_cast<const uint2*>(vb + (wb + t0 + 1) * ROWB + lane * 8);
-        w0[0] = a0.x; w0[1] = a0.y; w1[0] = a1.x; w1[1] = a1.y;
-      } else {
-        w0[0] = *reinterpret_cast<const uint32_t*>(vb + (wb + t0) * ROWB + lane * 4);
-        w1[0] = *reinterpret_cast<const uint32_t*>(vb + (wb + t0 + 1) * ROWB + lane * 4);
-      }
-#pragma unroll
-      for (int k = 0; k < E / 2; ++k) {
-        x2[2 * k] = h2_to_f2(__byte_perm(w0[k], w1[k], 0x5410));       // (t0 dim 2k,   t1 dim 2k)
-        x2[2 * k + 1] = h2_to_f2(__byte_perm(w0[k], w1[k], 0x7632));   // (t0 dim 2k+1, t1 dim 2k+1)
-      }
-    }
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float2 p2 = *reinterpret_cast<const float2*>(ps + g * C::TW_MAX + t0);
-#pragma unroll
-      for (int e = 0; e < E; ++e) ws.acc[g][e] = __ffma2_rn(p2, x2[e], ws.acc[g][e]);
-    }
-  }
-  __syncwarp();
 }
 
-template <int D, int G, bool CI8>
-__global__ void __launch_bounds__(160, (G >= 4 ? CONFKV_G4_MINB : 3)) attn_kernel(Cache c, AttnLaunch a, int splits, int units,
-                                                                  float qscale) {
-  using C = Cfg<D, G, CI8>;
-  extern __shared__ __align__(128) unsigned char smem[];
+// Byte `k` of each of four words, packed into one word (w0 lowest).
+__device__ __forceinline__ uint32_t pack_plane(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, int k) {
+  const uint32_t s = (uint32_t)k | ((uint32_t)(k + 4) << 4);
+  return __byte_perm(__byte_perm(w0, w1, s), __byte_perm(w2, w3, s), 0x5410);
+}
+
+struct TileCtx {
+  const unsigned char* sb;   // the staged tile
+  int j0, cnt;               // first row of the tile in its region; rows present
+  bool ok;                   // the tile arrived
+  float* ps;                 // this warp's probability rows [GP][32]
+  uint4* fb;                 // A operands of P.V for this tile, [k-step][mb][lane]
+  float* wmax;               // [4][GP]
+  volatile int* abort_flag;
+  float* sc_base;            // scores of this segment, [G][score_stride]
+  int warp, lane;
+};
+
+// One INT8 tile (128 tokens): warp w scores tokens 32w..32w+31 and builds the
+// P.V operand of k-step w; every warp then multiplies all four k-steps into
+// its D/4 output dimensions. Returns false when the CTA is aborting.
+template <int D, int GP>
+__device__ __forceinline__ bool consume_i8(const Cache& c, const AttnLaunch& a, const TileCtx& x,
+                                           SoftmaxState<D, GP>& st, const uint2 (&qi)[D / 32][GP / 2],
+                                           const float (&cq8)[GP / 4], unsigned long long& n_rows) {
+  constexpr int KB = D / 32, NB = GP / 2, MB = GP / 4, NBW = D / 32, HPL = GP / 4;
+  const int lane = x.lane, warp = x.warp;
+  const int g = lane >> 2, t = lane & 3;
+  const int G = c.G;
+  const uint32_t kt = smem_addr(x.sb), vt = kt + 128 * D;
+  const float* ksc = reinterpret_cast<const float*>(x.sb + 2 * 128 * D);
+  const float* vsc = ksc + 128;
+
+  // ---- scores: two 16-row blocks, KB k-blocks, NB n-blocks ----
+  float u[2][2][HPL];
+#pragma unroll
+  for (int mb2 = 0; mb2 < 2; ++mb2) {
+    int sacc[NB][4];
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) sacc[nb][k] = 0;
+    const int rb = warp * 32 + mb2 * 16;
+#pragma unroll
+    for (int kb = 0; kb < KB; ++kb) {
+      uint32_t af[4];
+      ldsm_x4(af, kt + (uint32_t)k8_off(rb + (lane & 7) + ((lane >> 3) & 1) * 8, kb * 32 + (lane >> 4) * 16, D));
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) mma_s8s8(sacc[nb], af, qi[kb][nb].x, qi[kb][nb].y);
+    }
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+      const int r = rb + g + 8 * hr;
+      const bool in = r < x.cnt;
+      const float ksr = ksc[r];
+#pragma unroll
+      for (int j = 0; j < HPL; ++j) {
+        const int* p01 = sacc[2 * j];
+        const int* p23 = sacc[2 * j + 1];
+        const float S = fmaf((float)p23[2 * hr + 1], 2097152.0f,
+                             fmaf((float)p23[2 * hr], 16384.0f, fmaf((float)p01[2 * hr + 1], 128.0f, (float)p01[2 * hr])));
+        const float sg = S * (ksr * cq8[j]);
+        const int head = t + 4 * j;
+        const bool valid = in && head < G;
+        if (valid) {
+          const int col = x.j0 + r;
+          if (!kChecked || guard(col < a.score_stride, c.err, kSiteAttnScore, 0, col))
+            x.sc_base[(size_t)head * a.score_stride + col] = sg;
+        }
+        u[mb2][hr][j] = valid ? sg * kLog2e : -CUDART_INF_F;
+      }
+    }
+  }
+  // ---- tile maxima, the tile's largest V scale, then the CTA-wide update ----
+#pragma unroll
+  for (int j = 0; j < HPL; ++j) {
+    float lm = fmaxf(fmaxf(u[0][0][j], u[0][1][j]), fmaxf(u[1][0][j], u[1][1][j]));
+    lm = fmaxf(lm, __shfl_xor_sync(0xffffffffu, lm, 4));
+    lm = fmaxf(lm, __shfl_xor_sync(0xffffffffu, lm, 8));
+    lm = fmaxf(lm, __shfl_xor_sync(0xffffffffu, lm, 16));
+    if (g == 0) x.wmax[warp * GP + t + 4 * j] = lm;
+  }
+  float vm;
+  {
+    const int i0 = lane * 4;
+    const float4 v4 = *reinterpret_cast<const float4*>(vsc + i0);
+    vm = fmaxf(fmaxf(i0 < x.cnt ? v4.x : 0.0f, i0 + 1 < x.cnt ? v4.y : 0.0f),
+               fmaxf(i0 + 2 < x.cnt ? v4.z : 0.0f, i0 + 3 < x.cnt ? v4.w : 0.0f));
+    vm = warp_max(vm);
+  }
+  if (named_barrier_or(1, 128, !x.ok || *x.abort_flag != 0)) return false;
+  update_max<D, GP>(st, x.wmax, lane);
+
+  // ---- probabilities times V scale, into this warp's rows ----
+#pragma unroll
+  for (int j = 0; j < HPL; ++j) {
+    const int head = t + 4 * j;
+    const float mh = sel(st.m, head);
+#pragma unroll
+    for (int mb2 = 0; mb2 < 2; ++mb2)
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr) {
+        const int rl = mb2 * 16 + g + 8 * hr;
+        const float uu = u[mb2][hr][j];
+        const float p = uu == -CUDART_INF_F ? 0.0f : exp2f(uu - mh);
+        st.lp8[j] += p;
+        x.ps[head * 32 + rl] = p == 0.0f ? 0.0f : p * vsc[warp * 32 + rl];
+      }
+  }
+  if (lane == 0) n_rows += max(0, min(32, x.cnt - warp * 32));
+  __syncwarp();
+
+  // ---- P.V operand of k-step `warp`: P' * 2^E as four byte planes ----
+  // P' <= vm < 2^(31 - E), so P' * 2^E < 2^31.
+  const int E = 31 - exp_of(vm);
+  const float sP = pow2i(E);
+  const int ha = GP == 4 ? (g & 3) : g;
+  {
+    const float4 v0 = *reinterpret_cast<const float4*>(x.ps + ha * 32 + 4 * t);
+    const float4 v1 = *reinterpret_cast<const float4*>(x.ps + ha * 32 + 16 + 4 * t);
+    const uint32_t P0 = __float2uint_rn(v0.x * sP), P1 = __float2uint_rn(v0.y * sP);
+    const uint32_t P2 = __float2uint_rn(v0.z * sP), P3 = __float2uint_rn(v0.w * sP);
+    const uint32_t P4 = __float2uint_rn(v1.x * sP), P5 = __float2uint_rn(v1.y * sP);
+    const uint32_t P6 = __float2uint_rn(v1.z * sP), P7 = __float2uint_rn(v1.w * sP);
+#pragma unroll
+    for (int mb = 0; mb < MB; ++mb) {
+      const int pl_lo = GP == 4 ? (g >> 2) : 2 * mb;
+      const int pl_hi = pl_lo + (GP == 4 ? 2 : 1);
+      uint4 f;
+      f.x = pack_plane(P0, P1, P2, P3, pl_lo);
+      f.y = pack_plane(P0, P1, P2, P3, pl_hi);
+      f.z = pack_plane(P4, P5, P6, P7, pl_lo);
+      f.w = pack_plane(P4, P5, P6, P7, pl_hi);
+      x.fb[(warp * MB + mb) * 32 + lane] = f;
+    }
+  }
+  named_barrier_sync(1, 128);
+
+  // ---- P.V: four k-steps of 32 tokens, NBW n-blocks of this warp ----
+  int ia[MB][NBW][4];
+#pragma unroll
+  for (int mb = 0; mb < MB; ++mb)
+#pragma unroll
+    for (int nb = 0; nb < NBW; ++nb)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) ia[mb][nb][k] = 0;
+#pragma unroll
+  for (int ks = 0; ks < 4; ++ks) {
+    uint32_t af[MB][4];
+#pragma unroll
+    for (int mb = 0; mb < MB; ++mb) {
+      const uint4 f = x.fb[(ks * MB + mb) * 32 + lane];
+      af[mb][0] = f.x;
+      af[mb][1] = f.y;
+      af[mb][2] = f.z;
+      af[mb][3] = f.w;
+    }
+#pragma unroll
+    for (int nbp = 0; nbp < NBW / 2; ++nbp) {
+      const int d = warp * (D / 4) + nbp * 16 + (lane & 7) + 8 * (lane >> 4);
+      uint32_t bf[4];
+      ldsm_x4(bf, vt + (uint32_t)swz128((size_t)(ks * D + d) * 32 + 16 * ((lane >> 3) & 1)));
+#pragma unroll
+      for (int mb = 0; mb < MB; ++mb) {
+        mma_u8s8(ia[mb][2 * nbp], af[mb], bf[0], bf[1]);
+        mma_u8s8(ia[mb][2 * nbp + 1], af[mb], bf[2], bf[3]);
+      }
+    }
+  }
+  const float inv = pow2i(-E);
+#pragma unroll
+  for (int mb = 0; mb < MB; ++mb) {
+    const int pl_lo = GP == 4 ? (g >> 2) : 2 * mb;
+    const int pl_hi = pl_lo + (GP == 4 ? 2 : 1);
+    const float wl = inv * pow2i(8 * pl_lo), wh = inv * pow2i(8 * pl_hi);
+#pragma unroll
+    for (int nb = 0; nb < NBW; ++nb) {
+      st.acc[mb][nb][0] = fmaf((float)ia[mb][nb][0], wl, st.acc[mb][nb][0]);
+      st.acc[mb][nb][1] = fmaf((float)ia[mb][nb][1], wl, st.acc[mb][nb][1]);
+      st.acc[mb][nb][2] = fmaf((float)ia[mb][nb][2], wh, st.acc[mb][nb][2]);
+      st.acc[mb][nb][3] = fmaf((float)ia[mb][nb][3], wh, st.acc[mb][nb][3]);
+    }
+  }
+  return true;
+}
+
+// One FP16 tile (64 tokens of the window ring, or of the cold region when
+// INT8 is off): warp w scores tokens 16w..16w+15 and builds k-step w.
+template <int D, int GP, bool RING>
+__device__ __forceinline__ bool consume_h(const Cache& c, const AttnLaunch& a, const TileCtx& x,
+                                          SoftmaxState<D, GP>& st, const uint2 (&qh)[D / 16], float qscale,
+                                          unsigned long long& n_rows) {
+  constexpr int KS = D / 16, MB = GP / 4, NBW = D / 32;
+  const int lane = x.lane, warp = x.warp;
+  const int g = lane >> 2, t = lane & 3;
+  const int G = c.G;
+  const uint32_t kt = smem_addr(x.sb), vt = kt + 128 * D;
+  const int32_t* pos = reinterpret_cast<const int32_t*>(x.sb + 2 * 128 * D);
+  const int rb = warp * 16;
+
+  float f[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+  for (int ks = 0; ks < KS; ++ks) {
+    uint32_t af[4];
+    ldsm_x4(af, kt + (uint32_t)h_off(rb + (lane & 7) + ((lane >> 3) & 1) * 8, ks * 32 + (lane >> 4) * 16, D));
+    mma_f16(f, af, qh[ks].x, qh[ks].y);
+  }
+  float u[2][2];
+  bool tok_valid[2];
+#pragma unroll
+  for (int hr = 0; hr < 2; ++hr) {
+    const int r = rb + g + 8 * hr;
+    bool tv = r < x.cnt;
+    if (RING) tv = tv && pos[r] >= 0;
+    tok_valid[hr] = tv;
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
+      const int head = 2 * t + cc;
+      const bool valid = tv && head < G;
+      const float sg = f[2 * hr + cc] * qscale;
+      if (valid) {
+        const int col = (RING ? c.cap : 0) + x.j0 + r;
+        if (!kChecked || guard(col < a.score_stride, c.err, kSiteAttnScore, 1, col))
+          x.sc_base[(size_t)head * a.score_stride + col] = sg;
+      }
+      u[hr][cc] = valid ? sg * kLog2e : -CUDART_INF_F;
+    }
+  }
+#pragma unroll
+  for (int cc = 0; cc < 2; ++cc) {
+    float lm = fmaxf(u[0][cc], u[1][cc]);
+    lm = fmaxf(lm, __shfl_xor_sync(0xffffffffu, lm, 4));
+    lm = fmaxf(lm, __shfl_xor_sync(0xffffffffu, lm, 8));
+    lm = fmaxf(lm, __shfl_xor_sync(0xffffffffu, lm, 16));
+    if (g == 0 && 2 * t + cc < GP) x.wmax[warp * GP + 2 * t + cc] = lm;
+  }
+  if (named_barrier_or(1, 128, !x.ok || *x.abort_flag != 0)) return false;
+  update_max<D, GP>(st, x.wmax, lane);
+
+#pragma unroll
+  for (int cc = 0; cc < 2; ++cc) {
+    const int head = 2 * t + cc;
+    if (head < GP) {
+      const float mh = sel(st.m, head);
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr) {
+        const float uu = u[hr][cc];
+        const float p = uu == -CUDART_INF_F ? 0.0f : exp2f(uu - mh);
+        st.lp16[cc] += p;
+        x.ps[head * 32 + g + 8 * hr] = p;
+      }
+    }
+  }
+  {
+    const unsigned bal0 = __ballot_sync(0xffffffffu, t == 0 && tok_valid[0]);
+    const unsigned bal1 = __ballot_sync(0xffffffffu, t == 0 && tok_valid[1]);
+    if (lane == 0) n_rows += __popc(bal0) + __popc(bal1);
+  }
+  __syncwarp();
+
+  // ---- P.V operand of k-step `warp`: p = hi + lo in fp16 ----
+  {
+    const int ha = GP == 4 ? (g & 3) : g;
+    const float2 pa = *reinterpret_cast<const float2*>(x.ps + ha * 32 + 2 * t);
+    const float2 pb = *reinterpret_cast<const float2*>(x.ps + ha * 32 + 8 + 2 * t);
+    const __half2 ha2 = __float22half2_rn(pa), hb2 = __float22half2_rn(pb);
+    const float2 fa = __half22float2(ha2), fb2 = __half22float2(hb2);
+    const __half2 la2 = __float22half2_rn(make_float2(pa.x - fa.x, pa.y - fa.y));
+    const __half2 lb2 = __float22half2_rn(make_float2(pb.x - fb2.x, pb.y - fb2.y));
+    const uint32_t uha = *reinterpret_cast<const uint32_t*>(&ha2), uhb = *reinterpret_cast<const uint32_t*>(&hb2);
+    const uint32_t ula = *reinterpret_cast<const uint32_t*>(&la2), ulb = *reinterpret_cast<const uint32_t*>(&lb2);
+    uint4 fr;
+    if (GP == 4) {
+      const bool lo_part = g >= 4;          // rows 0-3: hi parts, rows 4-7: lo parts, rows 8-15: zero
+      fr = make_uint4(lo_part ? ula : uha, 0u, lo_part ? ulb : uhb, 0u);
+    } else {
+      fr = make_uint4(uha, ula, uhb, ulb);  // row g: hi, row g+8: lo
+    }
+    x.fb[(warp * MB) * 32 + lane] = fr;
+  }
+  named_barrier_sync(1, 128);
+
+#pragma unroll
+  for (int ks = 0; ks < 4; ++ks) {
+    const uint4 fr = x.fb[(ks * MB) * 32 + lane];
+    const uint32_t af[4] = {fr.x, fr.y, fr.z, fr.w};
+#pragma unroll
+    for (int nbp = 0; nbp < NBW / 2; ++nbp) {
+      const int d0 = warp * (D / 4) + nbp * 16;
+      uint32_t bf[4];
+      ldsm_x4_t(bf, vt + (uint32_t)h_off(ks * 16 + (lane & 7) + 8 * ((lane >> 3) & 1), 2 * (d0 + 8 * (lane >> 4)), D));
+      mma_f16(st.acc[0][2 * nbp], af, bf[0], bf[1]);
+      mma_f16(st.acc[0][2 * nbp + 1], af, bf[2], bf[3]);
+    }
+  }
+  return true;
+}
+
+template <int D, int GP, bool CI8>
+__global__ void __launch_bounds__(160, 2) attn_kernel(Cache c, AttnLaunch a, int splits, int units, float qscale) {
+  using C = Cfg<D, GP, CI8>;
+  using Q = QF<D, GP>;
+  extern __shared__ __align__(1024) unsigned char smem[];
   unsigned char* stages = smem;
-  float* ps_all = reinterpret_cast<float*>(smem + C::NSTAGE * C::STAGE_BYTES);
-  float* merge = reinterpret_cast<float*>(smem + C::NSTAGE * C::STAGE_BYTES + C::PS_BYTES);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::NSTAGE * C::STAGE_BYTES + C::PS_BYTES + C::MERGE_BYTES);
+  float* ps_all = reinterpret_cast<float*>(smem + C::PS_OFF);
+  uint4* fb_all = reinterpret_cast<uint4*>(smem + C::FB_OFF);
+  float* wmax = reinterpret_cast<float*>(smem + C::WM_OFF);
+  float* lsum = reinterpret_cast<float*>(smem + C::LS_OFF);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   uint64_t* empty = full + C::NSTAGE;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + C::NSTAGE);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::FLAG_OFF);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   // Zero the stage ring once: rows a tile does not fill then hold zeros or an
-  // earlier tile's finite data, so the tile loops need no per-row masks.
-  for (int i = threadIdx.x; i < C::NSTAGE * C::STAGE_BYTES / 16; i += blockDim.x)
+  // earlier tile's data, never uninitialised bits.
+  for (int i = threadIdx.x; i < C::NSTAGE * C::STAGE / 16; i += blockDim.x)
     reinterpret_cast<uint4*>(stages)[i] = make_uint4(0u, 0u, 0u, 0u);
   fence_proxy_async_shared();
   if (threadIdx.x == 0) {
@@ -401,21 +654,19 @@ __global__ void __launch_bounds__(160, (G >= 4 ? CONFKV_G4_MINB : 3)) attn_kerne
       mbar_init(&empty[i], C::NCW);
     }
     abort_flag[0] = 0;
-    abort_flag[1] = 0;
     fence_mbar_init();
   }
   __syncthreads();
 
   if (warp == C::NCW) {
     // ------------------------------ producer -------------------------------
-    // One lane issues every copy; the other lanes go straight to the final
-    // barrier. On a timed-out wait the copies already issued are waited for
-    // (bounded) so that none lands after the CTA has exited.
+    // One lane issues every copy. On a timed-out wait the copies already
+    // issued are waited for (bounded) so that none lands after the CTA exits.
     if (lane == 0) {
       int ctr = 0;
       bool stop = false;
       for (int unit = blockIdx.x; unit < units && !stop; unit += gridDim.x) {
-        const Unit u = make_unit<D, G, CI8>(c, a.r, splits, unit);
+        const Unit u = make_unit<D, GP, CI8>(c, a.r, splits, unit);
         for (int t = u.t0; t < u.t1; ++t) {
           const int st = ctr % C::NSTAGE;
           if (ctr >= C::NSTAGE && !mbar_wait_bounded(&empty[st], ((ctr / C::NSTAGE) - 1) & 1)) {
@@ -426,45 +677,45 @@ __global__ void __launch_bounds__(160, (G >= 4 ? CONFKV_G4_MINB : 3)) attn_kerne
             stop = true;
             break;
           }
-          unsigned char* sb = stages + st * C::STAGE_BYTES;
+          unsigned char* sb = stages + st * C::STAGE;
           const bool cold = t < u.tiles_c;
+          const int j0 = cold ? t * C::TTC : (t - u.tiles_c) * C::TTR;
           if (kChecked) {
-            const int j0 = cold ? t * C::TT_C : (t - u.tiles_c) * C::TT_R;
-            const int cnt = cold ? min(C::TT_C, u.n_cold - j0) : min(C::TT_R, c.W - j0);
+            const int cnt = cold ? min(C::TTC, u.n_cold - j0) : C::TTR;
             const int lim = cold ? c.cap : c.Wst;
-            if (!guard(cnt >= 1 && j0 >= 0 && j0 + ((cnt + 3) & ~3) <= lim, c.err, kSiteAttnTile, u.s, j0)) {
-              *abort_flag = 1;   // consumers give up on their bounded wait for this tile
+            if (!guard(cnt >= 1 && j0 >= 0 && j0 + (cold && CI8 ? ((cnt + 31) & ~31) : C::TTR) <= lim, c.err,
+                       kSiteAttnTile, u.s, j0)) {
+              *abort_flag = 1;
               stop = true;
               break;
             }
           }
-          if (cold) {
-            const int j0 = t * C::TT_C;
-            const int cnt = min(C::TT_C, u.n_cold - j0);
+          if (cold && CI8) {
+            const int cnt = min(C::TTC, u.n_cold - j0);
             const int cnt4 = (cnt + 3) & ~3;
-            const uint32_t kvb = (uint32_t)cnt * C::ROWB_C;
-            const uint32_t aux = CI8 ? 2u * cnt4 * 4u : 0u;
-            mbar_arrive_expect_tx(&full[st], 2 * kvb + aux);
+            const uint32_t kbytes = (uint32_t)(D == 64 ? ((cnt + 1) & ~1) : cnt) * D;   // whole 128-byte lines
+            const uint32_t vbytes = (uint32_t)((cnt + 31) >> 5) * 32 * D;                // whole 32-token blocks
+            mbar_arrive_expect_tx(&full[st], kbytes + vbytes + 2u * cnt4 * 4u);
             const size_t row0 = (size_t)u.s * c.cap + j0;
-            if (CI8) {
-              bulk_g2s(sb, c.k8 + row0 * D, kvb, &full[st]);
-              bulk_g2s(sb + C::KV_BYTES, c.v8 + row0 * D, kvb, &full[st]);
-              bulk_g2s(sb + 2 * C::KV_BYTES, c.ks + row0, cnt4 * 4, &full[st]);
-              bulk_g2s(sb + 2 * C::KV_BYTES + C::TT_C * 4, c.vs + row0, cnt4 * 4, &full[st]);
-            } else {
-              bulk_g2s(sb, c.kc + row0 * D, kvb, &full[st]);
-              bulk_g2s(sb + C::KV_BYTES, c.vc + row0 * D, kvb, &full[st]);
-            }
+            bulk_g2s(sb, c.k8 + row0 * D, kbytes, &full[st]);
+            bulk_g2s(sb + C::KVB, c.v8 + row0 * D, vbytes, &full[st]);
+            bulk_g2s(sb + 2 * C::KVB, c.ks + row0, cnt4 * 4, &full[st]);
+            bulk_g2s(sb + 2 * C::KVB + 512, c.vs + row0, cnt4 * 4, &full[st]);
+          } else if (cold) {
+            // fp16 cold rows: the whole 64-row tile (rows past n_cold hold finite older data or zeros)
+            const uint32_t kvb = (uint32_t)C::TTR * 2 * D;
+            mbar_arrive_expect_tx(&full[st], 2 * kvb);
+            const size_t row0 = (size_t)u.s * c.cap + j0;
+            bulk_g2s(sb, c.kc + row0 * D, kvb, &full[st]);
+            bulk_g2s(sb + C::KVB, c.vc + row0 * D, kvb, &full[st]);
           } else {
-            const int j0 = (t - u.tiles_c) * C::TT_R;
-            const int cnt = min(C::TT_R, c.W - j0);
-            const int cnt4 = (cnt + 3) & ~3;
-            const uint32_t kvb = (uint32_t)cnt * C::ROWB_R;
-            mbar_arrive_expect_tx(&full[st], 2 * kvb + cnt4 * 4);
+            // window ring: the whole 64-slot tile (the ring stride is a multiple of 64)
+            const uint32_t kvb = (uint32_t)C::TTR * 2 * D;
+            mbar_arrive_expect_tx(&full[st], 2 * kvb + C::TTR * 4);
             const size_t row0 = (size_t)u.s * c.Wst + j0;
             bulk_g2s(sb, c.kr + row0 * D, kvb, &full[st]);
-            bulk_g2s(sb + C::KV_BYTES, c.vr + row0 * D, kvb, &full[st]);
-            bulk_g2s(sb + 2 * C::KV_BYTES, c.pos_r + row0, cnt4 * 4, &full[st]);
+            bulk_g2s(sb + C::KVB, c.vr + row0 * D, kvb, &full[st]);
+            bulk_g2s(sb + 2 * C::KVB, c.pos_r + row0, C::TTR * 4, &full[st]);
           }
           ++ctr;
         }
@@ -479,135 +730,137 @@ __global__ void __launch_bounds__(160, (G >= 4 ? CONFKV_G4_MINB : 3)) attn_kerne
   }
 
   // -------------------------------- consumers --------------------------------
-  const int sub = lane % C::LPT;       // which 16-dim slice of a row this lane scores
-  const bool own = C::XPOSE || sub < G;
-  const int g_own = C::XPOSE ? sub % G : (sub < G ? sub : 0);
-  float* ps = ps_all + warp * C::TW_MAX * 8;
-  volatile int* stop_snapshot = abort_flag + 1;
+  const int g = lane >> 2, t = lane & 3;
   int ctr = 0;
-
   for (int unit = blockIdx.x; unit < units; unit += gridDim.x) {
-    const Unit u = make_unit<D, G, CI8>(c, a.r, splits, unit);
-    // query slice of this lane, scaled by 1/sqrt(D)
-    float2 q2[G][8];
-    {
-      const size_t qrow = (size_t)((u.l - a.r.l0) * a.r.B + u.b) * c.Hq + u.h * G;
-      if (kChecked) guard(qrow + G <= (size_t)a.r.items(c.Hkv) * G, c.err, kSiteAttnQ, u.s, (int)qrow);
-      const __half* qp = a.q + qrow * D + sub * 16;
+    const Unit u = make_unit<D, GP, CI8>(c, a.r, splits, unit);
+    const unsigned char* qf = a.qfrag + (size_t)u.s * a.qf_stride;
+    uint2 qi[C::KB][C::NB];
+    float cq8[C::HPL];
+    if constexpr (CI8) {
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const uint4 w0 = *reinterpret_cast<const uint4*>(qp + g * D);
-        const uint4 w1 = *reinterpret_cast<const uint4*>(qp + g * D + 8);
-        const uint32_t ww[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+      for (int kb = 0; kb < C::KB; ++kb)
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float2 f = h2_to_f2(ww[i]);
-          q2[g][i] = make_float2(f.x * qscale, f.y * qscale);
-        }
-      }
+        for (int nb = 0; nb < C::NB; ++nb)
+          qi[kb][nb] = reinterpret_cast<const uint2*>(qf + Q::I8_OFF)[(kb * C::NB + nb) * 32 + lane];
+#pragma unroll
+      for (int j = 0; j < C::HPL; ++j) cq8[j] = reinterpret_cast<const float*>(qf + Q::CQ_OFF)[t + 4 * j];
     }
-    WarpState<D, G> ws;
+    uint2 qh[C::KS];
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      ws.m[g] = -CUDART_INF_F;
-#pragma unroll
-      for (int e = 0; e < C::E; ++e) ws.acc[g][e] = make_float2(0.0f, 0.0f);
-    }
-    ws.l_own = 0.0f;
-    unsigned long long n_rows_c = 0, n_rows_r = 0;
-    float* sc_base = a.scores + (size_t)u.s * G * a.score_stride;
+    for (int ks = 0; ks < C::KS; ++ks) qh[ks] = reinterpret_cast<const uint2*>(qf + Q::H_OFF)[ks * 32 + lane];
 
-    for (int t = u.t0; t < u.t1; ++t) {
-      const int st = ctr % C::NSTAGE;
-      const bool ok = mbar_wait_bounded(&full[st], (ctr / C::NSTAGE) & 1);
-      if (!ok) {
+    SoftmaxState<D, GP> st;
+#pragma unroll
+    for (int h = 0; h < GP; ++h) st.m[h] = -CUDART_INF_F;
+#pragma unroll
+    for (int mb = 0; mb < C::MB; ++mb)
+#pragma unroll
+      for (int nb = 0; nb < C::NBW; ++nb)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) st.acc[mb][nb][k] = 0.0f;
+#pragma unroll
+    for (int j = 0; j < C::HPL; ++j) st.lp8[j] = 0.0f;
+    st.lp16[0] = st.lp16[1] = 0.0f;
+    unsigned long long n_rows_c = 0, n_rows_r = 0;
+
+    TileCtx x;
+    x.ps = ps_all + warp * GP * 32;
+    x.wmax = wmax;
+    x.abort_flag = abort_flag;
+    x.sc_base = a.scores + (size_t)u.s * c.G * a.score_stride;
+    x.warp = warp;
+    x.lane = lane;
+    bool aborted = false;
+    for (int tt = u.t0; tt < u.t1; ++tt) {
+      const int stg = ctr % C::NSTAGE;
+      x.ok = mbar_wait_bounded(&full[stg], (ctr / C::NSTAGE) & 1);
+      if (!x.ok) {
         set_error(c.err, kErrDevice);
         *abort_flag = 1;
       }
-      if (*abort_flag) break;   // every consumer warp still reaches the merge barriers
-      const unsigned char* sb = stages + st * C::STAGE_BYTES;
-      if (t < u.tiles_c) {
-        const int j0 = t * C::TT_C;
-        const int cnt = min(C::TT_C, u.n_cold - j0);
-        if constexpr (CI8)
-          consume_tile<D, G, CI8, kTileCold8>(c, a, sb, q2, ws, ps, sc_base, u.s, j0, cnt, warp, lane, n_rows_c);
-        else
-          consume_tile<D, G, CI8, kTileCold16>(c, a, sb, q2, ws, ps, sc_base, u.s, j0, cnt, warp, lane, n_rows_c);
+      x.sb = stages + stg * C::STAGE;
+      x.fb = fb_all + (ctr & 1) * C::FB_ONE;
+      bool go;
+      if (tt < u.tiles_c) {
+        x.j0 = tt * C::TTC;
+        x.cnt = min(C::TTC, u.n_cold - x.j0);
+        if constexpr (CI8) go = consume_i8<D, GP>(c, a, x, st, qi, cq8, n_rows_c);
+        else go = consume_h<D, GP, false>(c, a, x, st, qh, qscale, n_rows_c);
       } else {
-        const int j0 = (t - u.tiles_c) * C::TT_R;
-        const int cnt = min(C::TT_R, c.W - j0);
-        consume_tile<D, G, CI8, kTileRing>(c, a, sb, q2, ws, ps, sc_base, u.s, j0, cnt, warp, lane, n_rows_r);
+        x.j0 = (tt - u.tiles_c) * C::TTR;
+        x.cnt = min(C::TTR, c.W - x.j0);
+        go = consume_h<D, GP, true>(c, a, x, st, qh, qscale, n_rows_r);
       }
-      if (lane == 0) mbar_arrive(&empty[st]);
+      if (!go) {
+        aborted = true;
+        break;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[stg]);
       ++ctr;
     }
-    // fold the (even token, odd token) halves of the P.V sums
-    float acc[G][C::E];
-#pragma unroll
-    for (int g = 0; g < G; ++g)
-#pragma unroll
-      for (int e = 0; e < C::E; ++e) acc[g][e] = ws.acc[g][e].x + ws.acc[g][e].y;
-    const float* m = ws.m;
-    const float l_own = ws.l_own;
 
-    // ---- merge the four consumer warps of this unit ----
-    float* mg = merge;                                  // [NCW][G] maxima
-    float* lg = merge + C::NCW * G;                     // [NCW][G] sums
-    float* ag = merge + 2 * C::NCW * G;                 // [NCW][G][D] accumulators
+    // ---- softmax sums over the CTA, then this unit's output ----
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float ls = warp_sum((own && g_own == g) ? l_own : 0.0f);
-      if (lane == 0) {
-        mg[warp * G + g] = m[g];
-        lg[warp * G + g] = ls;
-      }
+    for (int h = 0; h < GP; ++h) {
+      float v = 0.0f;
 #pragma unroll
-      for (int e = 0; e < C::E; ++e) ag[(warp * G + g) * D + lane * C::E + e] = acc[g][e];
+      for (int j = 0; j < C::HPL; ++j) v += (t + 4 * j == h) ? st.lp8[j] : 0.0f;
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) v += (2 * t + cc == h) ? st.lp16[cc] : 0.0f;
+      v = warp_sum(v);
+      if (lane == 0) lsum[warp * GP + h] = v;
     }
     if (lane == 0) {
       atomicAdd(&c.counters[kCntAttnInt8], CI8 ? n_rows_c : 0ull);
       atomicAdd(&c.counters[kCntAttnFp16], n_rows_r + (CI8 ? 0ull : n_rows_c));
     }
-    named_barrier_sync(1, C::NCW * 32);
-    if (threadIdx.x == 0) *stop_snapshot = *abort_flag;
+    named_barrier_sync(2, 128);
+    float L[GP];
+#pragma unroll
+    for (int h = 0; h < GP; ++h) L[h] = lsum[h] + lsum[GP + h] + lsum[2 * GP + h] + lsum[3 * GP + h];
     const int item = unit / splits;
     const int split = unit - item * splits;
-    for (int idx = threadIdx.x; idx < G * D; idx += C::NCW * 32) {
-      const int g = idx / D, d = idx - g * D;
-      float M = -CUDART_INF_F;
+    const int ha = GP == 4 ? (g & 3) : g;
+    const bool writer = (GP == 4 ? g < 4 : true) && ha < c.G;
+    const float Lh = sel(L, ha), Mh = sel(st.m, ha);
+    const size_t orow = (size_t)((u.l - a.r.l0) * a.r.B + u.b) * c.Hq + (size_t)u.h * c.G + ha;
+    float* pp = a.part + ((size_t)(item * splits + split) * c.G + ha) * (D + 2);
 #pragma unroll
-      for (int w = 0; w < C::NCW; ++w) M = fmaxf(M, mg[w * G + g]);
-      float L = 0.0f, A = 0.0f;
-      if (M != -CUDART_INF_F) {
-#pragma unroll
-        for (int w = 0; w < C::NCW; ++w) {
-          const float mw = mg[w * G + g];
-          if (mw == -CUDART_INF_F) continue;
-          const float f = exp2f(mw - M);
-          L += lg[w * G + g] * f;
-          A += ag[(w * G + g) * D + d] * f;
-        }
-      }
-      if (splits == 1) {
-        const size_t orow = (size_t)((u.l - a.r.l0) * a.r.B + u.b) * c.Hq + u.h * G + g;
-        if (kChecked && !guard(orow < (size_t)a.r.items(c.Hkv) * G, c.err, kSiteAttnOut, u.s, (int)orow)) continue;
-        a.out[orow * D + d] = A / L;
-        if (d == 0) {
-          const float lse = (M + __log2f(L)) * kLn2;
-          a.lse_ws[(size_t)u.s * G + g] = lse;
-          if (a.lse_out) a.lse_out[orow] = lse;
-        }
+    for (int nb = 0; nb < C::NBW; ++nb) {
+      float o0, o1;
+      if constexpr (GP == 4) {
+        o0 = st.acc[0][nb][0] + st.acc[0][nb][2];
+        o1 = st.acc[0][nb][1] + st.acc[0][nb][3];
+        o0 += __shfl_xor_sync(0xffffffffu, o0, 16);
+        o1 += __shfl_xor_sync(0xffffffffu, o1, 16);
       } else {
-        float* pp = a.part + ((size_t)(item * splits + split) * G + g) * (D + 2);
-        pp[d] = A;
-        if (d == 0) {
-          pp[D] = M;
-          pp[D + 1] = L;
+        o0 = (st.acc[0][nb][0] + st.acc[0][nb][2]) + (st.acc[1][nb][0] + st.acc[1][nb][2]);
+        o1 = (st.acc[0][nb][1] + st.acc[0][nb][3]) + (st.acc[1][nb][1] + st.acc[1][nb][3]);
+      }
+      const int d = warp * (D / 4) + nb * 8 + 2 * t;
+      if (writer && !aborted) {
+        if (splits == 1) {
+          if (kChecked && !guard(orow < (size_t)a.r.items(c.Hkv) * c.G, c.err, kSiteAttnOut, u.s, (int)orow)) continue;
+          *reinterpret_cast<float2*>(a.out + orow * D + d) = make_float2(o0 / Lh, o1 / Lh);
+        } else {
+          *reinterpret_cast<float2*>(pp + d) = make_float2(o0, o1);
         }
       }
     }
-    named_barrier_sync(1, C::NCW * 32);
-    if (*stop_snapshot) break;        // same value for every consumer thread
+    if (writer && !aborted && warp == 0 && t == 0) {
+      if (splits == 1) {
+        const float lse = (Mh + __log2f(Lh)) * kLn2;
+        a.lse_ws[(size_t)u.s * c.G + ha] = lse;
+        if (a.lse_out) a.lse_out[orow] = lse;
+      } else {
+        pp[D] = Mh;
+        pp[D + 1] = Lh;
+      }
+    }
+    // leave together when any warp saw an abort (same answer in every consumer thread)
+    if (named_barrier_or(2, 128, aborted || *abort_flag != 0)) break;
   }
   __syncthreads();
 }
@@ -615,8 +868,9 @@ __global__ void __launch_bounds__(160, (G >= 4 ? CONFKV_G4_MINB : 3)) attn_kerne
 // ---------------------------------------------------------------------------
 // combine split partials: one warp per (item, head)
 // ---------------------------------------------------------------------------
-template <int D, int G>
+template <int D>
 __global__ void __launch_bounds__(256) combine_kernel(Cache c, AttnLaunch a, int splits) {
+  const int G = c.G;
   const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const int items = a.r.items(c.Hkv);
@@ -684,28 +938,55 @@ __global__ void __launch_bounds__(256) ema_kernel(Cache c, AttnLaunch a, Policy 
   }
 }
 
-template <int D, int G, bool CI8>
+template <int G>
+void launch_ema(const Cache& c, const Policy& pol, const AttnLaunch& a, cudaStream_t st) {
+  ema_kernel<G><<<a.r.items(c.Hkv), 256, 0, st>>>(c, a, pol);
+}
+
+cudaError_t run_ema(const Cache& c, const Policy& pol, const AttnLaunch& a, cudaStream_t st) {
+  switch (c.G) {
+    case 1: launch_ema<1>(c, pol, a, st); break;
+    case 2: launch_ema<2>(c, pol, a, st); break;
+    case 3: launch_ema<3>(c, pol, a, st); break;
+    case 4: launch_ema<4>(c, pol, a, st); break;
+    case 5: launch_ema<5>(c, pol, a, st); break;
+    case 6: launch_ema<6>(c, pol, a, st); break;
+    case 7: launch_ema<7>(c, pol, a, st); break;
+    case 8: launch_ema<8>(c, pol, a, st); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaSuccess;
+}
+
+template <int D, int GP, bool CI8>
 cudaError_t run_attn(const Cache& c, const Policy& pol, const AttnLaunch& a, cudaStream_t st, long long* launches,
                      Prof* prof) {
-  using C = Cfg<D, G, CI8>;
+  using C = Cfg<D, GP, CI8>;
   const int items = a.r.items(c.Hkv);
-  cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, G, CI8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       C::SMEM_BYTES);
+  const float qscale = rsqrtf((float)D);
+  {
+    ProfScope ps(prof, kKAppend, st);
+    append_kernel<D, GP><<<(items * 32 + 255) / 256, 256, 0, st>>>(c, a, pol.mode == 1, qscale);
+  }
+  ++*launches;
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(attn_kernel<D, GP, CI8>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   int ctas_per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ctas_per_sm, attn_kernel<D, G, CI8>, 160, C::SMEM_BYTES);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ctas_per_sm, attn_kernel<D, GP, CI8>, 160, C::SMEM);
   if (e != cudaSuccess) return e;
   ctas_per_sm = max(1, ctas_per_sm);
   const int resident = a.num_sms * ctas_per_sm;
-  const int tiles_ub = (a.max_cold_tokens + C::TT_C - 1) / C::TT_C + (c.W + C::TT_R - 1) / C::TT_R;
+  const int tiles_ub = (a.max_cold_tokens + C::TTC - 1) / C::TTC + (c.W + C::TTR - 1) / C::TTR;
   int splits = 1;
   if (items < 2 * resident) {
     // few segments: split the token axis so that every SM has work
     splits = (2 * resident + items - 1) / items;
     splits = min(splits, max(1, tiles_ub / 2));
-  } else if (tiles_ub >= 64) {
+  } else if (tiles_ub >= 32) {
     // long segments: finer units even out the last wave
-    splits = min((16 * resident + items - 1) / items, tiles_ub / 16);
+    splits = min((16 * resident + items - 1) / items, tiles_ub / 8);
     splits = max(1, splits);
   }
   while (splits > 1 && (long long)items * splits > a.part_units) --splits;
@@ -713,61 +994,47 @@ cudaError_t run_attn(const Cache& c, const Policy& pol, const AttnLaunch& a, cud
   const int grid = min(units, resident);
   {
     ProfScope ps(prof, kKAttention, st);
-    attn_kernel<D, G, CI8><<<grid, 160, C::SMEM_BYTES, st>>>(c, a, splits, units, rsqrtf((float)D));
+    attn_kernel<D, GP, CI8><<<grid, 160, C::SMEM, st>>>(c, a, splits, units, qscale);
   }
   ++*launches;
   if (splits > 1) {
-    const int warps = items * G;
+    const int warps = items * c.G;
     ProfScope ps(prof, kKCombine, st);
-    combine_kernel<D, G><<<(warps * 32 + 255) / 256, 256, 0, st>>>(c, a, splits);
+    combine_kernel<D><<<(warps * 32 + 255) / 256, 256, 0, st>>>(c, a, splits);
     ++*launches;
   }
   if (pol.mode == 0) {
     ProfScope ps(prof, kKEma, st);
-    ema_kernel<G><<<items, 256, 0, st>>>(c, a, pol);
+    e = run_ema(c, pol, a, st);
+    if (e != cudaSuccess) return e;
     ++*launches;
   }
   return cudaGetLastError();
 }
 
-template <int D, int G>
-cudaError_t run_attn_g(const Cache& c, const Policy& pol, const AttnLaunch& a, cudaStream_t st, long long* n,
-                       Prof* prof) {
-  return c.cold_int8 ? run_attn<D, G, true>(c, pol, a, st, n, prof) : run_attn<D, G, false>(c, pol, a, st, n, prof);
+template <int D, int GP>
+cudaError_t run_attn_gp(const Cache& c, const Policy& pol, const AttnLaunch& a, cudaStream_t st, long long* n,
+                        Prof* prof) {
+  return c.cold_int8 ? run_attn<D, GP, true>(c, pol, a, st, n, prof) : run_attn<D, GP, false>(c, pol, a, st, n, prof);
 }
 
 }  // namespace
 
+int qfrag_bytes(int D, int G) {
+  if (D == 128) return G <= 4 ? QF<128, 4>::BYTES : QF<128, 8>::BYTES;
+  return G <= 4 ? QF<64, 4>::BYTES : QF<64, 8>::BYTES;
+}
+
 cudaError_t launch_decode_attn(const Cache& c, const Policy& pol, const AttnLaunch& a, cudaStream_t st,
                                long long* launches, Prof* prof) {
-  const int items = a.r.items(c.Hkv);
-  if (items == 0) return cudaSuccess;
-  const int blocks = (items * 32 + 255) / 256;
-  {
-    ProfScope ps(prof, kKAppend, st);
-    if (c.D == 128)
-      append_kernel<128><<<blocks, 256, 0, st>>>(c, a.r, a.k_new, a.v_new, a.prio_new, pol.mode == 1);
-    else
-      append_kernel<64><<<blocks, 256, 0, st>>>(c, a.r, a.k_new, a.v_new, a.prio_new, pol.mode == 1);
-  }
-  ++*launches;
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  if (c.D == 128) {
-    switch (c.G) {
-      case 1: return run_attn_g<128, 1>(c, pol, a, st, launches, prof);
-      case 2: return run_attn_g<128, 2>(c, pol, a, st, launches, prof);
-      case 4: return run_attn_g<128, 4>(c, pol, a, st, launches, prof);
-      case 5: return run_attn_g<128, 5>(c, pol, a, st, launches, prof);
-      case 8: return run_attn_g<128, 8>(c, pol, a, st, launches, prof);
-    }
-  } else {
-    switch (c.G) {
-      case 1: return run_attn_g<64, 1>(c, pol, a, st, launches, prof);
-      case 2: return run_attn_g<64, 2>(c, pol, a, st, launches, prof);
-      case 4: return run_attn_g<64, 4>(c, pol, a, st, launches, prof);
-    }
-  }
+  if (a.r.items(c.Hkv) == 0) return cudaSuccess;
+  if (c.G < 1 || c.G > 8) return cudaErrorInvalidValue;
+  if (c.D == 128)
+    return c.G <= 4 ? run_attn_gp<128, 4>(c, pol, a, st, launches, prof)
+                    : run_attn_gp<128, 8>(c, pol, a, st, launches, prof);
+  if (c.D == 64)
+    return c.G <= 4 ? run_attn_gp<64, 4>(c, pol, a, st, launches, prof)
+                    : run_attn_gp<64, 8>(c, pol, a, st, launches, prof);
   return cudaErrorInvalidValue;
 }
 

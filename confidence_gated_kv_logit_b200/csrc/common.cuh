@@ -18,6 +18,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "layout.cuh"
+
 namespace confkv {
 
 // sticky device error codes (values match confkv_status)
@@ -179,30 +181,63 @@ __device__ __forceinline__ unsigned long long rank_key(const Policy& p, float sc
 constexpr unsigned long long kNoKey = ~0ull;
 
 // ---------------------------------------------------------------------------
-// Symmetric per-row INT8 quantisation by one warp: amax = max |x| over the
-// row, scale = amax / 127 and code = clamp(rint_half_even(x / scale), +-127),
-// both divisions IEEE fp32; a zero row gets scale 0 and codes 0.
+// Row access by one warp: lane l holds the E = D/32 consecutive dimensions
+// E*l .. E*l+E-1 of a row, as D/64 words of fp16 pairs. "region" arguments are
+// the start of one segment's rows; the placement formulas are in layout.cuh.
 // ---------------------------------------------------------------------------
 template <int D>
-__device__ __forceinline__ void warp_quantize_row(const __half* __restrict__ src, int8_t* __restrict__ dst,
-                                                  float* __restrict__ scale_out, int lane) {
-  constexpr int E = D / 32;  // 2 or 4 elements per lane
-  float x[E];
-  if constexpr (E == 4) {
-    const uint2 w = *reinterpret_cast<const uint2*>(src + lane * 4);
-    float2 a = h2_to_f2(w.x), b = h2_to_f2(w.y);
-    x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
+__device__ __forceinline__ void row_load_plain(const __half* __restrict__ row, int lane, uint32_t (&w)[D / 64]) {
+  if constexpr (D == 128) {
+    const uint2 v = reinterpret_cast<const uint2*>(row)[lane];
+    w[0] = v.x;
+    w[1] = v.y;
   } else {
-    const uint32_t w = *reinterpret_cast<const uint32_t*>(src + lane * 2);
-    float2 a = h2_to_f2(w);
-    x[0] = a.x; x[1] = a.y;
+    w[0] = reinterpret_cast<const uint32_t*>(row)[lane];
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void row_load_h(const __half* __restrict__ region, int i, int lane, uint32_t (&w)[D / 64]) {
+  const unsigned char* p = reinterpret_cast<const unsigned char*>(region) + h_off(i, lane * (D / 16), D);
+  if constexpr (D == 128) {
+    const uint2 v = *reinterpret_cast<const uint2*>(p);
+    w[0] = v.x;
+    w[1] = v.y;
+  } else {
+    w[0] = *reinterpret_cast<const uint32_t*>(p);
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void row_store_h(__half* __restrict__ region, int i, int lane, const uint32_t (&w)[D / 64]) {
+  unsigned char* p = reinterpret_cast<unsigned char*>(region) + h_off(i, lane * (D / 16), D);
+  if constexpr (D == 128) {
+    *reinterpret_cast<uint2*>(p) = make_uint2(w[0], w[1]);
+  } else {
+    *reinterpret_cast<uint32_t*>(p) = w[0];
+  }
+}
+
+// Symmetric per-row INT8 quantisation: amax = max |x| over the row, scale =
+// amax / 127 and code = clamp(rint_half_even(x / scale), +-127), both
+// divisions IEEE fp32; a zero row gets scale 0 and codes 0. Returns the scale
+// (the same in every lane) and the lane's E codes packed little-endian.
+template <int D>
+__device__ __forceinline__ float row_quantize(const uint32_t (&w)[D / 64], uint32_t* packed) {
+  constexpr int E = D / 32;
+  float x[E];
+#pragma unroll
+  for (int k = 0; k < D / 64; ++k) {
+    const float2 f = h2_to_f2(w[k]);
+    x[2 * k] = f.x;
+    x[2 * k + 1] = f.y;
   }
   float amax = 0.0f;
 #pragma unroll
   for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(x[e]));
   amax = warp_max(amax);
   const float scale = __fdiv_rn(amax, 127.0f);
-  uint32_t packed = 0;
+  uint32_t pk = 0;
 #pragma unroll
   for (int e = 0; e < E; ++e) {
     int q = 0;
@@ -210,24 +245,39 @@ __device__ __forceinline__ void warp_quantize_row(const __half* __restrict__ src
       q = __float2int_rn(__fdiv_rn(x[e], scale));
       q = max(-127, min(127, q));
     }
-    packed |= ((uint32_t)(q & 0xff)) << (8 * e);
+    pk |= ((uint32_t)(q & 0xff)) << (8 * e);
   }
-  if constexpr (E == 4) {
-    *reinterpret_cast<uint32_t*>(dst + lane * 4) = packed;
-  } else {
-    *reinterpret_cast<uint16_t*>(dst + lane * 2) = (uint16_t)packed;
-  }
-  if (lane == 0) *scale_out = scale;
+  *packed = pk;
+  return scale;
 }
 
-// Copy one fp16 row of D elements by one warp.
 template <int D>
-__device__ __forceinline__ void warp_copy_row_h(const __half* __restrict__ src, __half* __restrict__ dst, int lane) {
-  if constexpr (D == 128) {
-    reinterpret_cast<uint2*>(dst)[lane] = reinterpret_cast<const uint2*>(src)[lane];
-  } else {
-    reinterpret_cast<uint32_t*>(dst)[lane] = reinterpret_cast<const uint32_t*>(src)[lane];
-  }
+__device__ __forceinline__ void row_store_k8(int8_t* __restrict__ region, int i, int lane, uint32_t packed) {
+  int8_t* p = region + k8_off(i, lane * (D / 32), D);
+  if constexpr (D == 128) *reinterpret_cast<uint32_t*>(p) = packed;
+  else *reinterpret_cast<uint16_t*>(p) = (uint16_t)packed;
+}
+
+template <int D>
+__device__ __forceinline__ void row_store_v8(int8_t* __restrict__ region, int i, int lane, uint32_t packed) {
+#pragma unroll
+  for (int e = 0; e < D / 32; ++e) region[v8_off(i, lane * (D / 32) + e, D)] = (int8_t)(packed >> (8 * e));
+}
+
+// Quantise fp16 row `src_i` of a permuted fp16 region (K and V) into cold
+// row `dst_i` (codes and scales); one warp.
+template <int D>
+__device__ __forceinline__ void warp_requant(const Cache& c, int s, int ring_slot, int cold_i, int lane) {
+  const size_t rb = (size_t)s * c.Wst * D, cb = (size_t)s * c.cap * D, cs = (size_t)s * c.cap + cold_i;
+  uint32_t w[D / 64], pk;
+  row_load_h<D>(c.kr + rb, ring_slot, lane, w);
+  float sc = row_quantize<D>(w, &pk);
+  row_store_k8<D>(c.k8 + cb, cold_i, lane, pk);
+  if (lane == 0) c.ks[cs] = sc;
+  row_load_h<D>(c.vr + rb, ring_slot, lane, w);
+  sc = row_quantize<D>(w, &pk);
+  row_store_v8<D>(c.v8 + cb, cold_i, lane, pk);
+  if (lane == 0) c.vs[cs] = sc;
 }
 
 }  // namespace confkv

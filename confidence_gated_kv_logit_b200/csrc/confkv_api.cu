@@ -76,6 +76,8 @@ struct confkv_handle {
   int part_units;
   uint32_t* vmask;
   int mask_words;
+  unsigned char* qfrag;          // [S][qf_stride] query operands of the attention kernel
+  int qf_stride;
   int32_t* keep_list;
   int32_t* keep_count;
   long long launches;
@@ -164,7 +166,7 @@ confkv_status confkv_create(int32_t layers, int32_t kv_heads, int32_t q_heads, i
   if (layers < 1 || kv_heads < 1 || q_heads < 1 || q_heads % kv_heads) return CONFKV_ERR_ARG;
   if (head_dim != 64 && head_dim != 128) return CONFKV_ERR_ARG;
   const int G = q_heads / kv_heads;
-  if (!(G == 1 || G == 2 || G == 4 || G == 5 || G == 8) || G > head_dim / 16) return CONFKV_ERR_ARG;
+  if (G < 1 || G > 8) return CONFKV_ERR_ARG;
   if (p.mode != CONFKV_MODE_CONF && p.mode != CONFKV_MODE_FIXED) return CONFKV_ERR_ARG;
   if (p.gate != CONFKV_GATE_PROSE && p.gate != CONFKV_GATE_LITERAL) return CONFKV_ERR_ARG;
   if (p.compact != CONFKV_COMPACT_HOLEFILL && p.compact != CONFKV_COMPACT_STABLE) return CONFKV_ERR_ARG;
@@ -226,7 +228,7 @@ confkv_status confkv_create(int32_t layers, int32_t kv_heads, int32_t q_heads, i
   c.G = G;
   c.D = head_dim;
   c.W = W;
-  c.Wst = round_up(W, 4);
+  c.Wst = round_up(W, 64);   // whole 64-slot tiles for the attention copies
   c.cap = (int)cap_ll;
   c.cold_int8 = p.int8_enable ? 1 : 0;
 
@@ -282,6 +284,8 @@ confkv_status confkv_create(int32_t layers, int32_t kv_heads, int32_t q_heads, i
   chk(B.alloc(&h->part, (size_t)h->part_units * G * (head_dim + 2)));
   h->mask_words = (c.cap + 31) / 32;
   chk(B.alloc(&h->vmask, S * (size_t)h->mask_words));
+  h->qf_stride = confkv::qfrag_bytes(head_dim, G);
+  chk(B.alloc(&h->qfrag, S * (size_t)h->qf_stride));
   if (p.mode == CONFKV_MODE_FIXED) {
     chk(B.alloc(&h->keep_list, S * (size_t)p.fixed_budget));
     chk(B.alloc(&h->keep_count, S));
@@ -308,6 +312,7 @@ confkv_status confkv_create(int32_t layers, int32_t kv_heads, int32_t q_heads, i
     chk(cudaMemset(c.counters, 0, confkv::kNumCounters * 8));
     chk(cudaMemset(h->tickets, 0, (size_t)p.max_batch * 4));
     chk(cudaMemset(h->scores, 0, S * G * (size_t)h->score_stride * 4));
+    chk(cudaMemset(h->qfrag, 0, S * (size_t)h->qf_stride));
     chk(cudaDeviceSynchronize());
   }
   if (e != cudaSuccess) {
@@ -445,6 +450,8 @@ confkv_status confkv_decode_attn(confkv_handle* h, int32_t layer, const void* q,
   a.part_units = h->part_units;
   a.max_cold_tokens = (int)std::min<long long>(ub, h->c.cap);
   a.num_sms = h->num_sms;
+  a.qfrag = h->qfrag;
+  a.qf_stride = h->qf_stride;
   cudaError_t e =
       confkv::launch_decode_attn(h->c, h->pol, a, static_cast<cudaStream_t>(stream), &h->launches, h->prof_ptr());
   if (e != cudaSuccess) return cuda_status(e);
@@ -564,18 +571,37 @@ confkv_status confkv_export_segment(confkv_handle* h, int32_t layer, int32_t seq
     std::memset(o, 0, n * 8);
   }
   o += n * 8;
-  d2h(o, c.cold_int8 ? (const void*)(c.k8 + cs * c.D) : (const void*)(c.kc + cs * c.D), n * row);
-  o += n * row;
-  d2h(o, c.cold_int8 ? (const void*)(c.v8 + cs * c.D) : (const void*)(c.vc + cs * c.D), n * row);
-  o += n * row;
+  // K and V rows leave the device permuted (see layout.cuh); they are copied
+  // raw and put back in logical row order here
+  const int D = c.D;
+  const size_t nr = (size_t)round_up((long long)n, 32);   // whole 128-byte lines and 32-token blocks
+  std::vector<unsigned char> raw(nr * row);
+  auto unpermute_cold = [&](const void* src, bool v_codes) {
+    d2h(raw.data(), src, nr * row);
+    for (size_t i = 0; i < n; ++i)
+      for (size_t b = 0; b < row; ++b) {
+        size_t off;
+        if (!c.cold_int8) off = confkv::h_off((int)i, (int)b, D);
+        else if (v_codes) off = confkv::v8_off((int)i, (int)b, D);
+        else off = confkv::k8_off((int)i, (int)b, D);
+        o[i * row + b] = raw[off];
+      }
+    o += n * row;
+  };
+  unpermute_cold(c.cold_int8 ? (const void*)(c.k8 + cs * c.D) : (const void*)(c.kc + cs * c.D), false);
+  unpermute_cold(c.cold_int8 ? (const void*)(c.v8 + cs * c.D) : (const void*)(c.vc + cs * c.D), true);
   const size_t rs = s * c.Wst;
   d2h(o, c.pos_r + rs, W * 4);
   o += W * 4;
   d2h(o, c.sc_r + rs, W * 4);
   o += W * 4;
-  d2h(o, c.kr + rs * c.D, W * c.D * 2);
-  o += W * c.D * 2;
-  d2h(o, c.vr + rs * c.D, W * c.D * 2);
+  std::vector<unsigned char> rraw((size_t)c.Wst * c.D * 2);
+  for (int which = 0; which < 2; ++which) {
+    d2h(rraw.data(), which ? (const void*)(c.vr + rs * c.D) : (const void*)(c.kr + rs * c.D), rraw.size());
+    for (size_t i = 0; i < W; ++i)
+      for (size_t b = 0; b < (size_t)c.D * 2; ++b) o[i * c.D * 2 + b] = rraw[confkv::h_off((int)i, (int)b, D)];
+    o += W * c.D * 2;
+  }
   *bytes = need;
   return e == cudaSuccess ? CONFKV_OK : CONFKV_ERR_CUDA;
 }

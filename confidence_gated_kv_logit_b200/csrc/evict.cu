@@ -31,23 +31,63 @@ constexpr int NT = 256;
 
 template <int D, bool CI8>
 struct Rows {
-  static constexpr int ROWB = CI8 ? D : 2 * D;   // bytes of one K (or V) row in the cold region
-  static constexpr int VEC = ROWB / 16;           // uint4 per row
+  static constexpr int ROWB = CI8 ? D : 2 * D;    // bytes of one K (or V) row in the cold region
+  static constexpr int KP = ROWB / 16;            // K parts: 16-byte chunks
+  static constexpr int VP = CI8 ? D / 4 : ROWB / 16;   // V parts: four codes (dims 4q..4q+3), or 16-byte chunks
+  static constexpr int NP = KP + VP;              // parts of one token's K and V
 };
 
-// Move cold row `src` to `dst` (both < cap) with `lanes` threads cooperating.
+// Part p of cold token i's K/V data (placement in layout.cuh). An INT8 V part
+// carries its four codes in .x.
+template <int D, bool CI8>
+__device__ __forceinline__ uint4 load_part(const Cache& c, int s, int i, int p) {
+  using R = Rows<D, CI8>;
+  const size_t base = (size_t)s * c.cap * D;
+  if (p < R::KP) {
+    const unsigned char* k = CI8 ? reinterpret_cast<const unsigned char*>(c.k8 + base)
+                                 : reinterpret_cast<const unsigned char*>(c.kc + base);
+    return *reinterpret_cast<const uint4*>(k + (CI8 ? k8_off(i, 16 * p, D) : h_off(i, 16 * p, D)));
+  }
+  const int q = p - R::KP;
+  if constexpr (CI8) {
+    const unsigned char* v = reinterpret_cast<const unsigned char*>(c.v8 + base);
+    uint32_t w = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) w |= (uint32_t)v[v8_off(i, 4 * q + e, D)] << (8 * e);
+    return make_uint4(w, 0u, 0u, 0u);
+  } else {
+    const unsigned char* v = reinterpret_cast<const unsigned char*>(c.vc + base);
+    return *reinterpret_cast<const uint4*>(v + h_off(i, 16 * q, D));
+  }
+}
+
+template <int D, bool CI8>
+__device__ __forceinline__ void store_part(const Cache& c, int s, int i, int p, uint4 val) {
+  using R = Rows<D, CI8>;
+  const size_t base = (size_t)s * c.cap * D;
+  if (p < R::KP) {
+    unsigned char* k = CI8 ? reinterpret_cast<unsigned char*>(c.k8 + base) : reinterpret_cast<unsigned char*>(c.kc + base);
+    *reinterpret_cast<uint4*>(k + (CI8 ? k8_off(i, 16 * p, D) : h_off(i, 16 * p, D))) = val;
+    return;
+  }
+  const int q = p - R::KP;
+  if constexpr (CI8) {
+    unsigned char* v = reinterpret_cast<unsigned char*>(c.v8 + base);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) v[v8_off(i, 4 * q + e, D)] = (unsigned char)(val.x >> (8 * e));
+  } else {
+    unsigned char* v = reinterpret_cast<unsigned char*>(c.vc + base);
+    *reinterpret_cast<uint4*>(v + h_off(i, 16 * q, D)) = val;
+  }
+}
+
+// Move cold row `src` to `dst` (both < cap), part `part` of Rows::NP; part 0
+// also moves the metadata.
 template <int D, bool CI8>
 __device__ __forceinline__ void move_cold_row(const Cache& c, int s, int src, int dst, int part) {
-  using R = Rows<D, CI8>;
-  const size_t so = (size_t)s * c.cap + src, dO = (size_t)s * c.cap + dst;
-  const uint4* ks = reinterpret_cast<const uint4*>(CI8 ? (const void*)(c.k8 + so * D) : (const void*)(c.kc + so * D));
-  const uint4* vs = reinterpret_cast<const uint4*>(CI8 ? (const void*)(c.v8 + so * D) : (const void*)(c.vc + so * D));
-  uint4* kd = reinterpret_cast<uint4*>(CI8 ? (void*)(c.k8 + dO * D) : (void*)(c.kc + dO * D));
-  uint4* vd = reinterpret_cast<uint4*>(CI8 ? (void*)(c.v8 + dO * D) : (void*)(c.vc + dO * D));
-  // part in [0, 2*VEC): first VEC words of K, then of V; part 0 also moves the metadata
-  if (part < R::VEC) kd[part] = ks[part];
-  else vd[part - R::VEC] = vs[part - R::VEC];
+  store_part<D, CI8>(c, s, dst, part, load_part<D, CI8>(c, s, src, part));
   if (part == 0) {
+    const size_t so = (size_t)s * c.cap + src, dO = (size_t)s * c.cap + dst;
     c.pos_c[dO] = c.pos_c[so];
     c.sc_c[dO] = c.sc_c[so];
     if (CI8) {
@@ -232,8 +272,8 @@ __device__ bool evict_segment_warp(const Cache& c, const Policy& pol, const Evic
           ++np;
         }
       }
-      for (int w = lane; w < np * 2 * R::VEC; w += 32) {
-        const int p = w / (2 * R::VEC);
+      for (int w = lane; w < np * R::NP; w += 32) {
+        const int p = w / R::NP;
         int src = -1, dst = -1;
 #pragma unroll
         for (int q = 0; q < kWarpMaxVictims; ++q)
@@ -244,7 +284,7 @@ __device__ bool evict_segment_warp(const Cache& c, const Policy& pol, const Evic
         if (kChecked && !guard(dst >= 0 && dst < n_keep && src >= n_keep && src < n_cold, c.err, kSiteEvictPair,
                                s, src))
           continue;
-        move_cold_row<D, CI8>(c, s, src, dst, w - p * 2 * R::VEC);
+        move_cold_row<D, CI8>(c, s, src, dst, w - p * R::NP);
       }
       moved = np;
       n_cold_new = n_keep;
@@ -264,8 +304,7 @@ __device__ bool evict_segment_warp(const Cache& c, const Policy& pol, const Evic
         if (lane == 0) record_violation(c.err, kSiteEvictRequant, s, idx);
       } else {
         const size_t cs = (size_t)s * c.cap + idx;
-        warp_quantize_row<D>(c.kr + rs * D, c.k8 + cs * D, c.ks + cs, lane);
-        warp_quantize_row<D>(c.vr + rs * D, c.v8 + cs * D, c.vs + cs, lane);
+        warp_requant<D>(c, s, slot, idx, lane);
         __syncwarp();
         if (lane == 0) {
           c.pos_c[cs] = leaving;
@@ -353,7 +392,7 @@ __device__ void evict_segment_block(const Cache& c, const Policy& pol, const Evi
       } else if (vi >= 0) {
         const int last = n_cold - 1;
         if (vi != last) {
-          for (int w = threadIdx.x; w < 2 * R::VEC; w += NT) move_cold_row<D, CI8>(c, s, last, vi, w);
+          for (int w = threadIdx.x; w < R::NP; w += NT) move_cold_row<D, CI8>(c, s, last, vi, w);
           moved = 1;
         }
         n_cold_new = n_cold - 1;
@@ -389,12 +428,12 @@ __device__ void evict_segment_block(const Cache& c, const Policy& pol, const Evi
         const int nm = block_collect<NT, NT>([&](int i) { return !victim(i); }, &mcur, n_cold, list_m, sm);
         const int np = min(nh, nm);
         if (np == 0) break;
-        for (int w = threadIdx.x; w < np * 2 * R::VEC; w += NT) {
-          const int p = w / (2 * R::VEC);
+        for (int w = threadIdx.x; w < np * R::NP; w += NT) {
+          const int p = w / R::NP;
           if (kChecked && !guard(list_h[p] >= 0 && list_h[p] < n_keep && list_m[p] >= n_keep && list_m[p] < n_cold,
                                  c.err, kSiteEvictPair, s, list_m[p]))
             continue;
-          move_cold_row<D, CI8>(c, s, list_m[p], list_h[p], w - p * 2 * R::VEC);
+          move_cold_row<D, CI8>(c, s, list_m[p], list_h[p], w - p * R::NP);
         }
         moved += np;
         __syncthreads();
@@ -402,7 +441,7 @@ __device__ void evict_segment_block(const Cache& c, const Policy& pol, const Evi
     } else {
       // stable: from the first hole on, every survivor moves down by the number
       // of victims before it, in chunks staged through shared memory
-      constexpr int CH = 16384 / (2 * R::ROWB) < 64 ? 16384 / (2 * R::ROWB) : 64;
+      constexpr int CH = 16384 / (16 * R::NP) < 64 ? 16384 / (16 * R::NP) : 64;
       int dst_base = 0;
       for (int base = 0; base < n_cold; base += CH) {
         const int i = base + (int)threadIdx.x;
@@ -410,16 +449,10 @@ __device__ void evict_segment_block(const Cache& c, const Policy& pol, const Evi
         int total;
         const int r = block_scan_flag<NT>(live, sm, &total);
         // stage this chunk's survivors (rows and metadata), then write them back
-        for (int w = threadIdx.x; w < CH * 2 * R::VEC; w += NT) {
-          const int rr = w / (2 * R::VEC), part = w - rr * 2 * R::VEC;
+        for (int w = threadIdx.x; w < CH * R::NP; w += NT) {
+          const int rr = w / R::NP, part = w - rr * R::NP;
           const int src = base + rr;
-          if (src < n_cold) {
-            const size_t so = (size_t)s * c.cap + src;
-            const uint4* kv = part < R::VEC
-                                  ? reinterpret_cast<const uint4*>(CI8 ? (const void*)(c.k8 + so * D) : (const void*)(c.kc + so * D)) + part
-                                  : reinterpret_cast<const uint4*>(CI8 ? (const void*)(c.v8 + so * D) : (const void*)(c.vc + so * D)) + (part - R::VEC);
-            reinterpret_cast<uint4*>(stage)[w] = *kv;
-          }
+          if (src < n_cold) reinterpret_cast<uint4*>(stage)[w] = load_part<D, CI8>(c, s, src, part);
         }
         if (live) {
           const size_t so = (size_t)s * c.cap + i;
@@ -431,14 +464,11 @@ __device__ void evict_segment_block(const Cache& c, const Policy& pol, const Evi
         }
         if (threadIdx.x < CH) list_h[threadIdx.x] = live ? 1 : 0;
         __syncthreads();
-        for (int w = threadIdx.x; w < CH * 2 * R::VEC; w += NT) {
-          const int rr = w / (2 * R::VEC), part = w - rr * 2 * R::VEC;
+        for (int w = threadIdx.x; w < CH * R::NP; w += NT) {
+          const int rr = w / R::NP, part = w - rr * R::NP;
           if (base + rr < n_cold && list_h[rr]) {
             const size_t dO = (size_t)s * c.cap + list_m[rr];
-            uint4* kv = part < R::VEC
-                            ? reinterpret_cast<uint4*>(CI8 ? (void*)(c.k8 + dO * D) : (void*)(c.kc + dO * D)) + part
-                            : reinterpret_cast<uint4*>(CI8 ? (void*)(c.v8 + dO * D) : (void*)(c.vc + dO * D)) + (part - R::VEC);
-            *kv = reinterpret_cast<const uint4*>(stage)[w];
+            store_part<D, CI8>(c, s, list_m[rr], part, reinterpret_cast<const uint4*>(stage)[w]);
             if (part == 0) {
               c.pos_c[dO] = stage_meta[0][rr];
               c.sc_c[dO] = __int_as_float(stage_meta[1][rr]);
@@ -471,8 +501,7 @@ __device__ void evict_segment_block(const Cache& c, const Policy& pol, const Evi
         if (threadIdx.x == 0) record_violation(c.err, kSiteEvictRequant, s, idx);
       } else {
         const size_t cs = (size_t)s * c.cap + idx;
-        warp_quantize_row<D>(c.kr + rs * D, c.k8 + cs * D, c.ks + cs, threadIdx.x);
-        warp_quantize_row<D>(c.vr + rs * D, c.v8 + cs * D, c.vs + cs, threadIdx.x);
+        warp_requant<D>(c, s, slot, idx, threadIdx.x);
         __syncwarp();
         if (threadIdx.x == 0) {
           c.pos_c[cs] = leaving;

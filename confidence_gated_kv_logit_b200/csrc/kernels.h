@@ -59,9 +59,13 @@ struct AttnLaunch {
   int part_units;         // capacity of part in (item, split) units
   int max_cold_tokens;    // host upper bound of n_cold over the call's segments
   int num_sms;
+  unsigned char* qfrag;   // [S][qf_stride] query operands prepared by the append kernel
+  int qf_stride;
 };
 cudaError_t launch_decode_attn(const Cache& c, const Policy& pol, const AttnLaunch& a, cudaStream_t st,
                                long long* launches, Prof* prof);
+// Bytes of the prepared query operands of one segment (qfrag stride).
+int qfrag_bytes(int D, int G);
 
 // K4 + K5 + K6: select, compaction, conversion of the token leaving the window.
 struct EvictLaunch {

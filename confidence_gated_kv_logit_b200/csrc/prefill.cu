@@ -101,10 +101,14 @@ __global__ void __launch_bounds__(NT) prefill_ingest_kernel(Cache c, PrefillLaun
   const __half* ksrc = a.k + in_row * D;
   const __half* vsrc = a.v + in_row * D;
   const float sc = fixed_mode ? a.prio[in_row] : 0.0f;
+  uint32_t w[D / 64];
   if (c.W > 0 && p > len - c.W) {
-    const size_t rs = (size_t)s * c.Wst + (p % c.W);
-    warp_copy_row_h<D>(ksrc, c.kr + rs * D, lane);
-    warp_copy_row_h<D>(vsrc, c.vr + rs * D, lane);
+    const int slot = p % c.W;
+    const size_t rs = (size_t)s * c.Wst + slot;
+    row_load_plain<D>(ksrc, lane, w);
+    row_store_h<D>(c.kr + (size_t)s * c.Wst * D, slot, lane, w);
+    row_load_plain<D>(vsrc, lane, w);
+    row_store_h<D>(c.vr + (size_t)s * c.Wst * D, slot, lane, w);
     if (lane == 0) {
       c.pos_r[rs] = p;
       c.sc_r[rs] = sc;
@@ -117,12 +121,22 @@ __global__ void __launch_bounds__(NT) prefill_ingest_kernel(Cache c, PrefillLaun
     return;
   }
   const size_t cs = (size_t)s * c.cap + idx;
+  const size_t cb = (size_t)s * c.cap * D;
   if (c.cold_int8) {
-    warp_quantize_row<D>(ksrc, c.k8 + cs * D, c.ks + cs, lane);
-    warp_quantize_row<D>(vsrc, c.v8 + cs * D, c.vs + cs, lane);
+    uint32_t pk;
+    row_load_plain<D>(ksrc, lane, w);
+    float scale = row_quantize<D>(w, &pk);
+    row_store_k8<D>(c.k8 + cb, idx, lane, pk);
+    if (lane == 0) c.ks[cs] = scale;
+    row_load_plain<D>(vsrc, lane, w);
+    scale = row_quantize<D>(w, &pk);
+    row_store_v8<D>(c.v8 + cb, idx, lane, pk);
+    if (lane == 0) c.vs[cs] = scale;
   } else {
-    warp_copy_row_h<D>(ksrc, c.kc + cs * D, lane);
-    warp_copy_row_h<D>(vsrc, c.vc + cs * D, lane);
+    row_load_plain<D>(ksrc, lane, w);
+    row_store_h<D>(c.kc + cb, idx, lane, w);
+    row_load_plain<D>(vsrc, lane, w);
+    row_store_h<D>(c.vc + cb, idx, lane, w);
   }
   if (lane == 0) {
     c.pos_c[cs] = p;

@@ -94,6 +94,18 @@ def attn_traffic(w):
         return None
 
 
+def roofline_table(bytes_per_kernel, ms_per_kernel, peak):
+    """Per kernel: time, algorithmic bytes, achieved GB/s and the fraction of the HBM peak."""
+    out = {}
+    for k, ms in ms_per_kernel.items():
+        if k not in bytes_per_kernel or ms <= 0:
+            continue
+        gbs = bytes_per_kernel[k] / (ms * 1e-3) / 1e9
+        out[k] = {"ms": round(ms, 4), "bytes": int(bytes_per_kernel[k]), "gbs": round(gbs, 1),
+                  "frac": round(gbs / peak, 3)}
+    return out
+
+
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -281,14 +293,18 @@ def main():
         h.confidence(lg, c_out)
         h.evict_compact(ALL_LAYERS)
 
-    # bulk first step, on its own
+    # bulk first step, on its own (per-kernel times from the library's event brackets)
     s0 = h.query()
+    h.profile(True)
+    h.profile_read(reset=True)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     step(0)
     e1.record(stream)
     torch.cuda.synchronize()
     step1_ms = e0.elapsed_time(e1)
+    prof1 = h.profile_read(reset=True)
+    h.profile(False)
     s1 = h.query()
     _report_device_error(h, "first step")
     for i in range(1, 1 + args.warmup):
@@ -345,6 +361,22 @@ def main():
     step_bytes = attn_bytes + ema_bytes + evict_bytes + move_bytes + req_bytes + conf_bytes
     ms_step = elapsed_ms / K
     kernel_ms = {k: round(v["ms"] / K, 4) for k, v in prof.items() if v["launches"]}
+    GP = 4 if G <= 4 else 8
+    qf_bytes = 2 * D * G + (4 * GP + 16) * D + 4 * GP               # q read + prepared operands written
+    append_bytes = L * B * Hkv * (4 * D + 4 * D + qf_bytes)
+    per_kernel_bytes = {"attention": attn_bytes * launches / K, "ema": ema_bytes,
+                        "evict": evict_bytes + move_bytes + req_bytes, "confidence": conf_bytes,
+                        "append": append_bytes}
+    kernels = roofline_table(per_kernel_bytes, kernel_ms, peak)
+    # step 1: the bulk eviction from the prompt down to the budget
+    d1 = {k: s1[k] - s0[k] for k in ("attn_tokens_int8", "attn_tokens_fp16", "evict_tokens", "moved_rows",
+                                     "requant_rows")}
+    step1_bytes = {
+        "attention": d1["attn_tokens_int8"] * (2 * D + 8 + 4 * G) + d1["attn_tokens_fp16"] * (4 * D + 4 * G) + qo,
+        "ema": (d1["attn_tokens_int8"] + d1["attn_tokens_fp16"]) * (4 * G + 8),
+        "evict": d1["evict_tokens"] * 8 + d1["moved_rows"] * 2 * (2 * D + 16) + d1["requant_rows"] * (6 * D + 8),
+        "confidence": conf_bytes, "append": append_bytes}
+    step1_kernels = roofline_table(step1_bytes, {k: v["ms"] for k, v in prof1.items() if v["launches"]}, peak)
 
     # ---- end to end through the public API with pinned host buffers ----
     hpool = []
@@ -409,7 +441,10 @@ def main():
                     "steps": E},
             "gpu_launches": sb["kernel_launches"] - sa["kernel_launches"],
             "clocks": clocks,
+            "kernels": kernels,
             "step1_ms": step1_ms,
+            "step1_kernels": step1_kernels,
+            "step1_counts": d1,
             "step1_attn_tokens": {"int8": s1["attn_tokens_int8"] - s0["attn_tokens_int8"],
                                   "fp16": s1["attn_tokens_fp16"] - s0["attn_tokens_fp16"]},
             "step_hbm_gbs": step_bytes / (ms_step * 1e-3) / 1e9,

@@ -79,6 +79,10 @@ __global__ void __launch_bounds__(NT) confidence_kernel(ConfLaunch a, Policy pol
   p.top1 = -CUDART_INF_F;
   p.top2 = -CUDART_INF_F;
   p.bad = 0;
+  // Each pass loads U logits per thread into registers, then reduces them in
+  // two sweeps: the maximum first, then S and T relative to it (no rescaling
+  // per element), with the top two kept branch-free (counted with
+  // multiplicity: t2 = max(t2, min(t1, x)), t1 = max(t1, x)).
   constexpr int U = 8;
   for (int base = v0; base < v1; base += NT * U) {
     float x[U];
@@ -87,30 +91,36 @@ __global__ void __launch_bounds__(NT) confidence_kernel(ConfLaunch a, Policy pol
       const int i = base + u * NT + threadIdx.x;
       x[u] = i < v1 ? __ldcs(lg + i) : -CUDART_INF_F;
     }
+    float mx = -CUDART_INF_F;
+    int bad = 0;
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int i = base + u * NT + threadIdx.x;
-      if (i >= v1) continue;
-      const float xv = x[u];
-      if (!(fabsf(xv) <= 3.402823466e38f)) {   // NaN or +-Inf
-        p.bad = 1;
-        continue;
-      }
-      if (xv > p.m) {
-        if (p.S > 0.0f) {
-          const float d = p.m - xv;
-          const float f = __expf(d);
-          p.T = f * fmaf(d, p.S, p.T);
-          p.S = f * p.S;
-        }
-        p.m = xv;
-      }
-      const float d = xv - p.m;
-      const float ev = __expf(d);
-      p.S += ev;
-      p.T = fmaf(ev, d, p.T);
-      top2_insert(xv, p.top1, p.top2);
+      const bool finite = fabsf(x[u]) <= 3.402823466e38f;
+      bad |= (i < v1 && !finite) ? 1 : 0;
+      if (!finite) x[u] = -CUDART_INF_F;        // out of range or non-finite: no contribution
+      mx = fmaxf(mx, x[u]);
+      p.top2 = fmaxf(p.top2, fminf(p.top1, x[u]));
+      p.top1 = fmaxf(p.top1, x[u]);
     }
+    p.bad |= bad;
+    if (mx == -CUDART_INF_F) continue;
+    float S = 0.0f, T = 0.0f;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const float d = x[u] - mx;                // -inf for the excluded elements
+      const float ev = __expf(d);               // 0 for them
+      S += ev;
+      T = fmaf(ev, ev > 0.0f ? d : 0.0f, T);
+    }
+    ConfPartial q;
+    q.m = mx;
+    q.S = S;
+    q.T = T;
+    q.top1 = -CUDART_INF_F;
+    q.top2 = -CUDART_INF_F;
+    q.bad = 0;
+    merge(p, q);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {

@@ -177,42 +177,63 @@ __device__ bool evict_segment_warp(const Cache& c, const Policy& pol, const Evic
   int32_t* pos_r = c.pos_r + (size_t)s * c.Wst;
   const float* sc_r = c.sc_r + (size_t)s * c.Wst;
 
-  int ring_here = 0;
-  for (int slot = lane; slot < W; slot += 32) ring_here += pos_r[slot] >= 0;
-  const int n = n_cold + __reduce_add_sync(0xffffffffu, ring_here);
   const int budget_eff = pol.mode == 1 ? pol.fixed_budget
                                        : max(a.budget[(size_t)b * c.L + l], pol.P + pol.n_sink);
+  auto rank = [&](int pos, float sc) -> unsigned long long {
+    if (t - pos < pol.P || pos < pol.n_sink) return kNoKey;
+    return rank_key(pol, sc, pos, t);
+  };
+  // One pass over the segment counts the occupied window slots and keeps
+  // each lane's kWarpMaxVictims smallest keys; the keys are computed before
+  // the victim count is known (it needs the slot count) and are simply
+  // unused when nothing is evicted. Loads are 16 bytes (four tokens) per lane.
+  LaneBest best;
+  best.init();
+  int ring_here = 0;
+  for (int s0 = 4 * lane; s0 < W; s0 += 128) {   // the ring stride is a multiple of 64 slots
+    const int4 p4 = *reinterpret_cast<const int4*>(pos_r + s0);
+    const float4 f4 = *reinterpret_cast<const float4*>(sc_r + s0);
+    const int pp[4] = {p4.x, p4.y, p4.z, p4.w};
+    const float ff[4] = {f4.x, f4.y, f4.z, f4.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (s0 + q < W && pp[q] >= 0) {
+        ++ring_here;
+        best.offer(rank(pp[q], ff[q]), n_cold + s0 + q);
+      }
+    }
+  }
+  for (int base = 0; base < n_cold; base += 256) {   // cap is a multiple of 64 tokens
+    int4 P[2];
+    float4 F[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int i0 = base + 128 * u + 4 * lane;
+      P[u] = make_int4(-1, -1, -1, -1);
+      F[u] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      if (i0 < n_cold) {
+        P[u] = *reinterpret_cast<const int4*>(pos_c + i0);
+        F[u] = *reinterpret_cast<const float4*>(sc_c + i0);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int pp[4] = {P[u].x, P[u].y, P[u].z, P[u].w};
+      const float ff[4] = {F[u].x, F[u].y, F[u].z, F[u].w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int i = base + 128 * u + 4 * lane + q;
+        if (i < n_cold) best.offer(rank(pp[q], ff[q]), i);
+      }
+    }
+  }
+  const int n = n_cold + __reduce_add_sync(0xffffffffu, ring_here);
   const int e = n - budget_eff;
   int n_cold_new = n_cold;
   int moved = 0;
 
   if (e > 0 && t >= 0) {
     if (e > kWarpMaxVictims || a.stable) return false;
-    auto rank = [&](int pos, float sc) -> unsigned long long {
-      if (t - pos < pol.P || pos < pol.n_sink) return kNoKey;
-      return rank_key(pol, sc, pos, t);
-    };
-    LaneBest best;
-    best.init();
-    // cold region, four tokens per lane in flight
-    int i = lane;
-    for (; i + 96 < n_cold; i += 128) {
-      int p4[4];
-      float s4[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        p4[u] = pos_c[i + 32 * u];
-        s4[u] = sc_c[i + 32 * u];
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) best.offer(rank(p4[u], s4[u]), i + 32 * u);
-    }
-    for (; i < n_cold; i += 32) best.offer(rank(pos_c[i], sc_c[i]), i);
-    // window ring (empty slots hold position -1)
-    for (int slot = lane; slot < W; slot += 32) {
-      const int pos = pos_r[slot];
-      if (pos >= 0) best.offer(rank(pos, sc_r[slot]), n_cold + slot);
-    }
 
     // merge: the e smallest keys of the segment, one per round; cold victims
     // are collected in v[0..ec) (the same values in every lane)
@@ -530,7 +551,10 @@ __global__ void __launch_bounds__(NT, 4) evict_kernel(Cache c, Policy pol, Evict
   if (threadIdx.x == 0) n_slow = 0;
   if (threadIdx.x < 3) cnt[threadIdx.x] = 0;
   __syncthreads();
-  const int item = blockIdx.x * kSegsPerCta + warp;
+  // segments are dealt to CTAs round-robin, so that the segments of one
+  // sequence (which share a budget, and so need the whole-CTA path at the
+  // same steps) spread over many CTAs
+  const int item = warp * gridDim.x + blockIdx.x;
   if (item < items) {
     WarpCounts wc;
     if (!evict_segment_warp<D, CI8>(c, pol, a, item, lane, &wc)) {

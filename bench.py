@@ -353,8 +353,9 @@ def main():
     achieved = attn_bytes / (attn_ms * 1e-3) / 1e9
     traffic = attn_traffic(w)
     # whole-step algorithmic bytes: attention + EMA pass + confidence + eviction scan/moves
-    ema_bytes = (n8 + n16) * (4 * G + 8) / K
-    evict_bytes = (sb["evict_tokens"] - sa["evict_tokens"]) * 8 / K
+    cand_bytes = L * B * Hkv * 208                                # eviction candidates, written and read once
+    ema_bytes = (n8 + n16) * (4 * G + 12) / K + cand_bytes          # scores, EMA r/w, positions
+    evict_bytes = (sb["evict_tokens"] - sa["evict_tokens"]) * 8 / K + cand_bytes
     move_bytes = (sb["moved_rows"] - sa["moved_rows"]) * 2 * (2 * D + 16) / K
     req_bytes = (sb["requant_rows"] - sa["requant_rows"]) * (6 * D + 8) / K
     conf_bytes = B * V * 4
@@ -373,7 +374,7 @@ def main():
                                      "requant_rows")}
     step1_bytes = {
         "attention": d1["attn_tokens_int8"] * (2 * D + 8 + 4 * G) + d1["attn_tokens_fp16"] * (4 * D + 4 * G) + qo,
-        "ema": (d1["attn_tokens_int8"] + d1["attn_tokens_fp16"]) * (4 * G + 8),
+        "ema": (d1["attn_tokens_int8"] + d1["attn_tokens_fp16"]) * (4 * G + 12) + cand_bytes,
         "evict": d1["evict_tokens"] * 8 + d1["moved_rows"] * 2 * (2 * D + 16) + d1["requant_rows"] * (6 * D + 8),
         "confidence": conf_bytes, "append": append_bytes}
     step1_kernels = roofline_table(step1_bytes, {k: v["ms"] for k, v in prof1.items() if v["launches"]}, peak)
@@ -442,6 +443,7 @@ def main():
             "gpu_launches": sb["kernel_launches"] - sa["kernel_launches"],
             "clocks": clocks,
             "kernels": kernels,
+            "evict_block_segments_per_step": (sb["evict_block_segments"] - sa["evict_block_segments"]) / K,
             "step1_ms": step1_ms,
             "step1_kernels": step1_kernels,
             "step1_counts": d1,

@@ -57,7 +57,7 @@ class Stats(ctypes.Structure):
                 ("max_len", ctypes.c_int32), ("attn_tokens_int8", ctypes.c_int64),
                 ("attn_tokens_fp16", ctypes.c_int64), ("evict_tokens", ctypes.c_int64),
                 ("moved_rows", ctypes.c_int64), ("requant_rows", ctypes.c_int64),
-                ("kernel_launches", ctypes.c_int64)]
+                ("kernel_launches", ctypes.c_int64), ("evict_block_segments", ctypes.c_int64)]
 
 
 class Profile(ctypes.Structure):

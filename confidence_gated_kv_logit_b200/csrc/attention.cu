@@ -80,17 +80,15 @@ struct QF {
   static constexpr int BYTES = (CQ_OFF + GP * 4 + 255) / 256 * 256;
 };
 
-// Digit `plane` (0..3, least significant first) of the balanced base-128
-// expansion Q = d0 + 128 d1 + 128^2 d2 + 128^3 d3, |d_k| <= 64, |Q| < 2^27.
-__device__ __forceinline__ int q_digit(int Q, int plane) {
-  int d = 0;
+// The balanced base-128 digits of Q (least significant first):
+// Q = d0 + 128 d1 + 128^2 d2 + 128^3 d3 with |d_k| <= 64 for |Q| < 2^27.
+__device__ __forceinline__ void q_digits(int Q, int (&d)[4]) {
 #pragma unroll
   for (int k = 0; k < 3; ++k) {
-    d = ((Q + 64) & 127) - 64;
-    if (k == plane) return d;
-    Q = (Q - d) >> 7;
+    d[k] = ((Q + 64) & 127) - 64;
+    Q = (Q - d[k]) >> 7;
   }
-  return Q;
+  d[3] = Q;
 }
 
 template <int D, int GP>
@@ -114,28 +112,34 @@ __device__ __forceinline__ void prepare_query(const Cache& c, const AttnLaunch& 
     if (lane == 0) reinterpret_cast<float*>(out + Q::CQ_OFF)[hh] = mx > 0.0f ? qscale * pow2i(ex - 27) : 0.0f;
   }
   const int g = lane >> 2, t = lane & 3;
+  // column g of n-block nb = 2*hs + p2 is head g/2 + 4*hs, digit plane 2*p2 + g%2
 #pragma unroll
   for (int kb = 0; kb < Q::KB; ++kb) {
 #pragma unroll
-    for (int nb = 0; nb < Q::NB; ++nb) {
-      const int hh = g / 2 + 4 * (nb / 2);
-      const int plane = 2 * (nb % 2) + (g % 2);
+    for (int hs = 0; hs < GP / 4; ++hs) {
+      const int hh = g / 2 + 4 * hs;
       const float sc = sel(scl, hh);
-      uint32_t r[2];
+      uint32_t r[2][2] = {{0u, 0u}, {0u, 0u}};   // [p2][half]
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
-        const int d0 = kb * 32 + half * 16 + 4 * t;
-        uint32_t pk = 0;
         if (hh < G) {
-          const uint2 w = *reinterpret_cast<const uint2*>(qb + (size_t)hh * D + d0);
+          const uint2 w = *reinterpret_cast<const uint2*>(qb + (size_t)hh * D + kb * 32 + half * 16 + 4 * t);
           const float2 f01 = h2_to_f2(w.x), f23 = h2_to_f2(w.y);
           const float qv[4] = {f01.x, f01.y, f23.x, f23.y};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) pk |= (uint32_t)(q_digit(__float2int_rn(qv[e] * sc), plane) & 0xff) << (8 * e);
+          for (int e = 0; e < 4; ++e) {
+            int d[4];
+            q_digits(__float2int_rn(qv[e] * sc), d);
+            const int lo = (g & 1) ? d[1] : d[0], hi = (g & 1) ? d[3] : d[2];
+            r[0][half] |= (uint32_t)(lo & 0xff) << (8 * e);
+            r[1][half] |= (uint32_t)(hi & 0xff) << (8 * e);
+          }
         }
-        r[half] = pk;
       }
-      reinterpret_cast<uint2*>(out + Q::I8_OFF)[(kb * Q::NB + nb) * 32 + lane] = make_uint2(r[0], r[1]);
+#pragma unroll
+      for (int p2 = 0; p2 < 2; ++p2)
+        reinterpret_cast<uint2*>(out + Q::I8_OFF)[(kb * Q::NB + 2 * hs + p2) * 32 + lane] =
+            make_uint2(r[p2][0], r[p2][1]);
     }
   }
 #pragma unroll
@@ -905,42 +909,123 @@ __global__ void __launch_bounds__(256) combine_kernel(Cache c, AttnLaunch a, int
 }
 
 // ---------------------------------------------------------------------------
-// attention-mass EMA: one CTA per segment
+// attention-mass EMA: one warp per segment, eight segments per CTA. Each lane
+// takes four consecutive tokens per 128 with 16-byte loads of the G score rows
+// and of the EMA values, two such groups in flight at a time.
 // ---------------------------------------------------------------------------
 template <int G>
+__device__ __forceinline__ float4 ema_update4(const float* __restrict__ sb, int stride, int col, float4 e,
+                                              const float (&lse)[G], const Policy& pol) {
+  float sum[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const float4 v = *reinterpret_cast<const float4*>(sb + (size_t)g * stride + col);
+    sum[0] += __expf(v.x - lse[g]);
+    sum[1] += __expf(v.y - lse[g]);
+    sum[2] += __expf(v.z - lse[g]);
+    sum[3] += __expf(v.w - lse[g]);
+  }
+  const float invG = 1.0f / G;
+  e.x = fmaf(pol.beta, e.x, pol.one_minus_beta * (sum[0] * invG));
+  e.y = fmaf(pol.beta, e.y, pol.one_minus_beta * (sum[1] * invG));
+  e.z = fmaf(pol.beta, e.z, pol.one_minus_beta * (sum[2] * invG));
+  e.w = fmaf(pol.beta, e.w, pol.one_minus_beta * (sum[3] * invG));
+  return e;
+}
+
+// The pass also computes every token's eviction key from its new EMA value
+// and leaves the segment's kCandMax smallest keys, with the window slot count,
+// in a.cand for the eviction kernel (which then need not rescan the segment).
+template <int G>
 __global__ void __launch_bounds__(256) ema_kernel(Cache c, AttnLaunch a, Policy pol) {
-  const int item = blockIdx.x;
+  const int lane = threadIdx.x & 31;
+  const int item = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (item >= a.r.items(c.Hkv)) return;
   int l, b, h;
   const int s = seg_of(c, a.r, item, &l, &b, &h);
   float lse[G];
 #pragma unroll
   for (int g = 0; g < G; ++g) lse[g] = a.lse_ws[(size_t)s * G + g];
   const int n_cold = c.n_cold[s];
-  if (!guard(n_cold >= 0 && n_cold <= c.cap, c.err, kSiteEmaSeg, s, n_cold)) return;
+  const int t = c.next_pos[s] - 1;
+  if (!(n_cold >= 0 && n_cold <= c.cap)) {
+    if (lane == 0) record_violation(c.err, kSiteEmaSeg, s, n_cold);
+    return;
+  }
   const float* sb = a.scores + (size_t)s * G * a.score_stride;
-  const float invG = 1.0f / G;
-  for (int i = threadIdx.x; i < n_cold + c.W; i += blockDim.x) {
-    float* scp;
-    int col;
-    if (i < n_cold) {
-      scp = c.sc_c + (size_t)s * c.cap + i;
-      col = i;
-    } else {
-      const int slot = i - n_cold;
-      if (c.pos_r[(size_t)s * c.Wst + slot] < 0) continue;
-      scp = c.sc_r + (size_t)s * c.Wst + slot;
-      col = c.cap + slot;
-    }
-    float sum = 0.0f;
+  float* scc = c.sc_c + (size_t)s * c.cap;
+  const int32_t* pc = c.pos_c + (size_t)s * c.cap;
+  LaneBest best;
+  best.init();
+  const bool use_bound = pol.one_minus_alpha >= 0x1p-60f;
+  const float t1_over_oma = use_bound ? (float)(t + 1) / pol.one_minus_alpha : 0.0f;
+  auto offer = [&](int pos, float ema, int idx) {
+    if (pos + 1 > best.pos_bound) return;
+    if (t - pos < pol.P || pos < pol.n_sink) return;   // protected: never a victim
+    best.offer(rank_key(pol, ema, pos, t), idx);
+    if (use_bound) best.update_bound(t1_over_oma);
+  };
+  // cold region [0, n_cold): the region and the score rows are multiples of 64 long
+  for (int base = 0; base < n_cold; base += 256) {
 #pragma unroll
-    for (int g = 0; g < G; ++g) sum += __expf(sb[(size_t)g * a.score_stride + col] - lse[g]);
-    *scp = fmaf(pol.beta, *scp, pol.one_minus_beta * (sum * invG));
+    for (int u = 0; u < 2; ++u) {
+      const int i0 = base + 128 * u + 4 * lane;
+      if (i0 < n_cold) {
+        const float4 e = ema_update4<G>(sb, a.score_stride, i0, *reinterpret_cast<const float4*>(scc + i0), lse, pol);
+        const int4 p4 = *reinterpret_cast<const int4*>(pc + i0);
+        if (i0 + 3 < n_cold) {
+          *reinterpret_cast<float4*>(scc + i0) = e;
+        } else {
+          scc[i0] = e.x;
+          if (i0 + 1 < n_cold) scc[i0 + 1] = e.y;
+          if (i0 + 2 < n_cold) scc[i0 + 2] = e.z;
+        }
+        offer(p4.x, e.x, i0);
+        if (i0 + 1 < n_cold) offer(p4.y, e.y, i0 + 1);
+        if (i0 + 2 < n_cold) offer(p4.z, e.z, i0 + 2);
+        if (i0 + 3 < n_cold) offer(p4.w, e.w, i0 + 3);
+      }
+    }
+  }
+  // window ring: occupied slots only (the ring stride is a multiple of 64)
+  const int32_t* pr = c.pos_r + (size_t)s * c.Wst;
+  float* scr = c.sc_r + (size_t)s * c.Wst;
+  int ring_here = 0;
+  for (int s0 = 4 * lane; s0 < c.W; s0 += 128) {
+    const int4 p4 = *reinterpret_cast<const int4*>(pr + s0);
+    const float4 e = ema_update4<G>(sb, a.score_stride, c.cap + s0, *reinterpret_cast<const float4*>(scr + s0), lse, pol);
+    const int pp[4] = {p4.x, p4.y, p4.z, p4.w};
+    const float ee[4] = {e.x, e.y, e.z, e.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (s0 + q < c.W && pp[q] >= 0) {
+        scr[s0 + q] = ee[q];
+        ++ring_here;
+        offer(pp[q], ee[q], n_cold + s0 + q);
+      }
+    }
+  }
+  if (a.cand == nullptr) return;
+  const int n_ring = __reduce_add_sync(0xffffffffu, ring_here);
+  unsigned long long mk;
+  int mi, cnt, safe;
+  warp_merge_smallest(best, lane, kCandMax, &mk, &mi, &cnt, &safe);
+  EvictCand* cd = a.cand + s;
+  if (lane < kCandMax) {
+    cd->key[lane] = mk;
+    cd->idx[lane] = mi;
+  }
+  if (lane == 0) {
+    cd->n_ring = n_ring;
+    cd->safe = safe;
+    cd->n_cold = n_cold;
+    cd->stamp = t + 1;
   }
 }
 
 template <int G>
 void launch_ema(const Cache& c, const Policy& pol, const AttnLaunch& a, cudaStream_t st) {
-  ema_kernel<G><<<a.r.items(c.Hkv), 256, 0, st>>>(c, a, pol);
+  ema_kernel<G><<<(a.r.items(c.Hkv) + 7) / 8, 256, 0, st>>>(c, a, pol);
 }
 
 cudaError_t run_ema(const Cache& c, const Policy& pol, const AttnLaunch& a, cudaStream_t st) {

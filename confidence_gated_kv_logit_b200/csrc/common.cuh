@@ -33,6 +33,7 @@ enum Counter {
   kCntEvictScanned = 2,
   kCntMovedRows = 3,
   kCntRequant = 4,
+  kCntEvictBlock = 5,
   kNumCounters = 8
 };
 

@@ -18,7 +18,7 @@ namespace {
 
 constexpr uint32_t kMagic = 0xC0F1C0DEu;
 constexpr uint32_t kDead = 0xDEADC0DEu;
-constexpr int kMaxCpr = 128;   // CTAs per logit row (one per ~2048 logits)
+constexpr int kMaxCpr = 128;   // CTAs per logit row (one per ~8192 logits)
 
 struct Buffers {
   std::vector<void*> ptrs;
@@ -78,6 +78,7 @@ struct confkv_handle {
   int mask_words;
   unsigned char* qfrag;          // [S][qf_stride] query operands of the attention kernel
   int qf_stride;
+  confkv::EvictCand* cand;       // [S] eviction candidates from the EMA pass
   int32_t* keep_list;
   int32_t* keep_count;
   long long launches;
@@ -286,6 +287,7 @@ confkv_status confkv_create(int32_t layers, int32_t kv_heads, int32_t q_heads, i
   chk(B.alloc(&h->vmask, S * (size_t)h->mask_words));
   h->qf_stride = confkv::qfrag_bytes(head_dim, G);
   chk(B.alloc(&h->qfrag, S * (size_t)h->qf_stride));
+  chk(B.alloc(&h->cand, S));
   if (p.mode == CONFKV_MODE_FIXED) {
     chk(B.alloc(&h->keep_list, S * (size_t)p.fixed_budget));
     chk(B.alloc(&h->keep_count, S));
@@ -313,6 +315,7 @@ confkv_status confkv_create(int32_t layers, int32_t kv_heads, int32_t q_heads, i
     chk(cudaMemset(h->tickets, 0, (size_t)p.max_batch * 4));
     chk(cudaMemset(h->scores, 0, S * G * (size_t)h->score_stride * 4));
     chk(cudaMemset(h->qfrag, 0, S * (size_t)h->qf_stride));
+    chk(cudaMemset(h->cand, 0xff, S * sizeof(confkv::EvictCand)));   // stamp -1: no record
     chk(cudaDeviceSynchronize());
   }
   if (e != cudaSuccess) {
@@ -384,6 +387,7 @@ confkv_status confkv_prefill(confkv_handle* h, int32_t layer, int32_t batch, con
   a.prio = priority;
   a.keep_list = h->keep_list;
   a.keep_count = h->keep_count;
+  a.cand = h->cand;
   e = confkv::launch_prefill(h->c, h->pol, a, st, &h->launches, h->prof_ptr());
   if (e != cudaSuccess) return CONFKV_ERR_CUDA;
   // the host copy of lens must stay valid until the copy has been consumed
@@ -408,7 +412,7 @@ confkv_status confkv_confidence(confkv_handle* h, const float* logits, int32_t b
   a.L = h->L;
   a.part = h->cpart;
   a.tickets = h->tickets;
-  a.cpr = std::max(1, std::min(kMaxCpr, (vocab + 2047) / 2048));
+  a.cpr = std::max(1, std::min(kMaxCpr, (vocab + 8191) / 8192));
   a.c_ws = h->c_ws;
   a.budget_ws = h->budget;
   a.c_out = c_out;
@@ -452,6 +456,7 @@ confkv_status confkv_decode_attn(confkv_handle* h, int32_t layer, const void* q,
   a.num_sms = h->num_sms;
   a.qfrag = h->qfrag;
   a.qf_stride = h->qf_stride;
+  a.cand = h->cand;
   cudaError_t e =
       confkv::launch_decode_attn(h->c, h->pol, a, static_cast<cudaStream_t>(stream), &h->launches, h->prof_ptr());
   if (e != cudaSuccess) return cuda_status(e);
@@ -472,6 +477,7 @@ confkv_status confkv_evict_compact(confkv_handle* h, int32_t layer, void* stream
   a.vmask = h->vmask;
   a.mask_words = h->mask_words;
   a.stable = h->p.compact == CONFKV_COMPACT_STABLE;
+  a.cand = h->cand;
   cudaError_t e =
       confkv::launch_evict_compact(h->c, h->pol, a, static_cast<cudaStream_t>(stream), &h->launches, h->prof_ptr());
   if (e != cudaSuccess) return cuda_status(e);
@@ -495,6 +501,7 @@ confkv_status confkv_query(confkv_handle* h, confkv_stats* out) {
   out->moved_rows = (int64_t)cnt[confkv::kCntMovedRows];
   out->requant_rows = (int64_t)cnt[confkv::kCntRequant];
   out->kernel_launches = h->launches;
+  out->evict_block_segments = (int64_t)cnt[confkv::kCntEvictBlock];
   out->bytes_capacity = (int64_t)h->buf.bytes;
   out->min_len = 0;
   out->max_len = 0;

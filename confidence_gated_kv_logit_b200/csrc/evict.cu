@@ -22,6 +22,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "select.cuh"
+#include "warp_select.cuh"
 
 namespace confkv {
 
@@ -98,58 +99,8 @@ __device__ __forceinline__ void move_cold_row(const Cache& c, int s, int src, in
 }
 
 constexpr int kSegsPerCta = NT / 32;     // the fast path gives each warp one segment
-constexpr int kWarpMaxVictims = 4;        // victims one warp handles; more go to the whole CTA
-
 struct WarpCounts {
   int scanned = 0, moved = 0, requant = 0;
-};
-
-__device__ __forceinline__ unsigned long long warp_min_u64(unsigned long long v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const unsigned long long w = __shfl_xor_sync(0xffffffffu, v, o);
-    v = w < v ? w : v;
-  }
-  return v;
-}
-
-// Keeps the kWarpMaxVictims smallest (key, index) pairs seen by this lane, ascending.
-struct LaneBest {
-  unsigned long long k[kWarpMaxVictims];
-  int i[kWarpMaxVictims];
-  __device__ __forceinline__ void init() {
-#pragma unroll
-    for (int j = 0; j < kWarpMaxVictims; ++j) {
-      k[j] = kNoKey;
-      i[j] = -1;
-    }
-  }
-  __device__ __forceinline__ void offer(unsigned long long key, int idx) {
-    if (key < k[kWarpMaxVictims - 1]) {
-      k[kWarpMaxVictims - 1] = key;
-      i[kWarpMaxVictims - 1] = idx;
-#pragma unroll
-      for (int j = kWarpMaxVictims - 1; j > 0; --j) {
-        if (k[j] < k[j - 1]) {
-          const unsigned long long tk = k[j];
-          k[j] = k[j - 1];
-          k[j - 1] = tk;
-          const int ti = i[j];
-          i[j] = i[j - 1];
-          i[j - 1] = ti;
-        }
-      }
-    }
-  }
-  __device__ __forceinline__ void pop() {
-#pragma unroll
-    for (int j = 0; j < kWarpMaxVictims - 1; ++j) {
-      k[j] = k[j + 1];
-      i[j] = i[j + 1];
-    }
-    k[kWarpMaxVictims - 1] = kNoKey;
-    i[kWarpMaxVictims - 1] = -1;
-  }
 };
 
 // One segment by one warp. Handles the common decode step (at most
@@ -158,10 +109,12 @@ struct LaneBest {
 // lane lists, the same hole-fill pairing as the whole-CTA path (the k-th
 // hole below the new end gets the k-th survivor above it) and the conversion
 // of the token leaving the window. Returns false, having written nothing,
-// when the segment needs the whole-CTA path (more victims, or stable order).
+// when the segment needs the whole-CTA path (more victims, stable order, or
+// a lane list that may have dropped a victim). ws_pairs: 2*kWarpMaxVictims
+// ints of shared memory owned by this warp.
 template <int D, bool CI8>
 __device__ bool evict_segment_warp(const Cache& c, const Policy& pol, const EvictLaunch& a, int item, int lane,
-                                   WarpCounts* wc) {
+                                   WarpCounts* wc, int* ws_pairs) {
   using R = Rows<D, CI8>;
   int l, b, h;
   const int s = seg_of(c, a.r, item, &l, &b, &h);
@@ -183,134 +136,131 @@ __device__ bool evict_segment_warp(const Cache& c, const Policy& pol, const Evic
     if (t - pos < pol.P || pos < pol.n_sink) return kNoKey;
     return rank_key(pol, sc, pos, t);
   };
-  // One pass over the segment counts the occupied window slots and keeps
-  // each lane's kWarpMaxVictims smallest keys; the keys are computed before
+  // This step's EMA pass may have left the segment's smallest keys and its
+  // window slot count (confidence mode): then nothing needs rescanning.
+  EvictCand* cd = a.cand != nullptr ? a.cand + s : nullptr;
+  bool have = false;
+  int n_ring = 0, count = 0, safe = 0;
+  unsigned long long my_key = kNoKey;
+  int my_idx = -1;
+  if (cd != nullptr && pol.mode == 0 && !a.stable && cd->stamp == t + 1 && cd->n_cold == n_cold) {
+    have = true;
+    n_ring = cd->n_ring;
+    safe = cd->safe;
+    if (lane < kCandMax) {
+      my_key = cd->key[lane];
+      my_idx = cd->idx[lane];
+    }
+    count = __popc(__ballot_sync(0xffffffffu, lane < kCandMax && my_key != kNoKey));
+  }
+  // Otherwise one pass over the segment counts the occupied window slots and
+  // keeps each lane's kLaneKeep smallest keys; the keys are computed before
   // the victim count is known (it needs the slot count) and are simply
   // unused when nothing is evicted. Loads are 16 bytes (four tokens) per lane.
   LaneBest best;
   best.init();
-  int ring_here = 0;
-  for (int s0 = 4 * lane; s0 < W; s0 += 128) {   // the ring stride is a multiple of 64 slots
-    const int4 p4 = *reinterpret_cast<const int4*>(pos_r + s0);
-    const float4 f4 = *reinterpret_cast<const float4*>(sc_r + s0);
-    const int pp[4] = {p4.x, p4.y, p4.z, p4.w};
-    const float ff[4] = {f4.x, f4.y, f4.z, f4.w};
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      if (s0 + q < W && pp[q] >= 0) {
-        ++ring_here;
-        best.offer(rank(pp[q], ff[q]), n_cold + s0 + q);
-      }
-    }
-  }
-  for (int base = 0; base < n_cold; base += 256) {   // cap is a multiple of 64 tokens
-    int4 P[2];
-    float4 F[2];
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int i0 = base + 128 * u + 4 * lane;
-      P[u] = make_int4(-1, -1, -1, -1);
-      F[u] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-      if (i0 < n_cold) {
-        P[u] = *reinterpret_cast<const int4*>(pos_c + i0);
-        F[u] = *reinterpret_cast<const float4*>(sc_c + i0);
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int pp[4] = {P[u].x, P[u].y, P[u].z, P[u].w};
-      const float ff[4] = {F[u].x, F[u].y, F[u].z, F[u].w};
+  if (!have) {
+    const bool use_bound = pol.mode == 0 && pol.one_minus_alpha >= 0x1p-60f;
+    const float t1_over_oma = use_bound ? (float)(t + 1) / pol.one_minus_alpha : 0.0f;
+    int ring_here = 0;
+    for (int s0 = 4 * lane; s0 < W; s0 += 128) {   // the ring stride is a multiple of 64 slots
+      const int4 p4 = *reinterpret_cast<const int4*>(pos_r + s0);
+      const float4 f4 = *reinterpret_cast<const float4*>(sc_r + s0);
+      const int pp[4] = {p4.x, p4.y, p4.z, p4.w};
+      const float ff[4] = {f4.x, f4.y, f4.z, f4.w};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const int i = base + 128 * u + 4 * lane + q;
-        if (i < n_cold) best.offer(rank(pp[q], ff[q]), i);
+        if (s0 + q < W && pp[q] >= 0) {
+          ++ring_here;
+          if (pp[q] + 1 <= best.pos_bound) {
+            best.offer(rank(pp[q], ff[q]), n_cold + s0 + q);
+            if (use_bound) best.update_bound(t1_over_oma);
+          }
+        }
       }
     }
+    for (int base = 0; base < n_cold; base += 256) {   // cap is a multiple of 64 tokens
+      int4 P[2];
+      float4 F[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int i0 = base + 128 * u + 4 * lane;
+        P[u] = make_int4(-1, -1, -1, -1);
+        F[u] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        if (i0 < n_cold) {
+          P[u] = *reinterpret_cast<const int4*>(pos_c + i0);
+          F[u] = *reinterpret_cast<const float4*>(sc_c + i0);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int pp[4] = {P[u].x, P[u].y, P[u].z, P[u].w};
+        const float ff[4] = {F[u].x, F[u].y, F[u].z, F[u].w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int i = base + 128 * u + 4 * lane + q;
+          if (i < n_cold && pp[q] + 1 <= best.pos_bound) {
+            best.offer(rank(pp[q], ff[q]), i);
+            if (use_bound) best.update_bound(t1_over_oma);
+          }
+        }
+      }
+    }
+    n_ring = __reduce_add_sync(0xffffffffu, ring_here);
   }
-  const int n = n_cold + __reduce_add_sync(0xffffffffu, ring_here);
+  const int n = n_cold + n_ring;
   const int e = n - budget_eff;
   int n_cold_new = n_cold;
   int moved = 0;
 
   if (e > 0 && t >= 0) {
     if (e > kWarpMaxVictims || a.stable) return false;
+    // the e smallest keys: victim j's index in lane j; nothing is written
+    // before the completeness check (see warp_merge_smallest)
+    if (!have) warp_merge_smallest(best, lane, e, &my_key, &my_idx, &count, &safe);
+    if (count < e || safe < e) return false;
+    const int my_victim = lane < e ? my_idx : -1;
 
-    // merge: the e smallest keys of the segment, one per round; cold victims
-    // are collected in v[0..ec) (the same values in every lane)
-    int v[kWarpMaxVictims];
-    int ec = 0;
-#pragma unroll
-    for (int j = 0; j < kWarpMaxVictims; ++j) {
-      v[j] = -1;
-      if (j < e) {
-        const unsigned long long m = warp_min_u64(best.k[0]);
-        if (m != kNoKey) {
-          const unsigned own = __ballot_sync(0xffffffffu, best.k[0] == m);
-          const int src = __ffs(own) - 1;
-          const int vi = __shfl_sync(0xffffffffu, best.i[0], src);
-          if (lane == src) best.pop();
-          if (vi >= n_cold) {
-            if (lane == 0) pos_r[vi - n_cold] = -1;
-          } else {
-#pragma unroll
-            for (int q = 0; q <= j; ++q)
-              if (q == ec) v[q] = vi;
-            ++ec;
-          }
-        }
-      }
-    }
-
+    const bool is_v = my_victim >= 0;
+    if (is_v && my_victim >= n_cold) pos_r[my_victim - n_cold] = -1;   // window victims free their slot
+    const bool cold_v = is_v && my_victim < n_cold;
+    const int ec = __popc(__ballot_sync(0xffffffffu, cold_v));
     if (ec > 0) {
       const int n_keep = n_cold - ec;
-      // holes: victims below n_keep; movers: survivors in [n_keep, n_cold).
-      // Both lists ascending; pair p moves mover p into hole p.
-      int hole_of[kWarpMaxVictims], mover_of[kWarpMaxVictims];
-#pragma unroll
-      for (int p = 0; p < kWarpMaxVictims; ++p) hole_of[p] = mover_of[p] = -1;
+      // holes: cold victims below n_keep; movers: survivors in [n_keep, n_cold).
+      // Pair p moves the p-th mover (ascending) into the p-th hole (ascending).
+      const bool hole = cold_v && my_victim < n_keep;
+      int hole_rank = 0;
+      bool idx_is_victim = false;
+      const int idx = n_keep + lane;                  // mover candidate of this lane (lane < ec)
 #pragma unroll
       for (int q = 0; q < kWarpMaxVictims; ++q) {
-        if (q < ec && v[q] < n_keep) {
-          int r = 0;
-#pragma unroll
-          for (int q2 = 0; q2 < kWarpMaxVictims; ++q2) r += (q2 < ec && v[q2] < n_keep && v[q2] < v[q]) ? 1 : 0;
-#pragma unroll
-          for (int p = 0; p < kWarpMaxVictims; ++p)
-            if (p == r) hole_of[p] = v[q];
-        }
+        const int vq = __shfl_sync(0xffffffffu, my_victim, q);
+        const bool cq = __shfl_sync(0xffffffffu, cold_v, q);
+        hole_rank += (cq && vq < n_keep && vq < my_victim) ? 1 : 0;
+        idx_is_victim |= cq && vq == idx;
       }
-      int np = 0;
-#pragma unroll
-      for (int d = 0; d < kWarpMaxVictims; ++d) {
-        const int idx = n_keep + d;
-        bool is_victim = false;
-#pragma unroll
-        for (int q = 0; q < kWarpMaxVictims; ++q) is_victim |= (q < ec && v[q] == idx);
-        if (d < ec && !is_victim) {
-#pragma unroll
-          for (int p = 0; p < kWarpMaxVictims; ++p)
-            if (p == np) mover_of[p] = idx;
-          ++np;
-        }
-      }
+      const bool mover = lane < ec && !idx_is_victim;
+      const unsigned mb = __ballot_sync(0xffffffffu, mover);
+      const int np = __popc(mb);
+      int* holes = ws_pairs;
+      int* movers = ws_pairs + kWarpMaxVictims;
+      if (hole) holes[hole_rank] = my_victim;
+      if (mover) movers[__popc(mb & ((1u << lane) - 1u))] = idx;
+      __syncwarp();
       for (int w = lane; w < np * R::NP; w += 32) {
-        const int p = w / R::NP;
-        int src = -1, dst = -1;
-#pragma unroll
-        for (int q = 0; q < kWarpMaxVictims; ++q)
-          if (q == p) {
-            src = mover_of[q];
-            dst = hole_of[q];
-          }
+        const int pr = w / R::NP;
+        const int src = movers[pr], dst = holes[pr];
         if (kChecked && !guard(dst >= 0 && dst < n_keep && src >= n_keep && src < n_cold, c.err, kSiteEvictPair,
                                s, src))
           continue;
-        move_cold_row<D, CI8>(c, s, src, dst, w - p * R::NP);
+        move_cold_row<D, CI8>(c, s, src, dst, w - pr * R::NP);
       }
       moved = np;
       n_cold_new = n_keep;
     }
   }
+  if (cd != nullptr && lane == 0) cd->stamp = -1;   // the record described the segment before this call
   __syncwarp();   // ring slots freed and rows moved above are visible to every lane
 
   // the token that the next append would push out of the window becomes INT8
@@ -338,7 +288,7 @@ __device__ bool evict_segment_warp(const Cache& c, const Policy& pol, const Evic
     }
   }
   if (lane == 0) c.n_cold[s] = n_cold_new;
-  wc->scanned = n;
+  wc->scanned = have ? 0 : n;   // tokens whose keys this call read
   wc->moved = moved;
   wc->requant = requant;
   return true;
@@ -536,6 +486,8 @@ __device__ void evict_segment_block(const Cache& c, const Policy& pol, const Evi
   }
   if (threadIdx.x == 0) {
     c.n_cold[s] = n_cold_new;
+    atomicAdd(&c.counters[kCntEvictBlock], 1ull);
+    if (a.cand != nullptr) a.cand[s].stamp = -1;
     atomicAdd(&c.counters[kCntEvictScanned], (unsigned long long)n);
     if (moved > 0) atomicAdd(&c.counters[kCntMovedRows], (unsigned long long)moved);
   }
@@ -547,17 +499,20 @@ __global__ void __launch_bounds__(NT, 4) evict_kernel(Cache c, Policy pol, Evict
   __shared__ int slow_items[kSegsPerCta];
   __shared__ int n_slow;
   __shared__ unsigned long long cnt[3];
+  __shared__ int pairs[kSegsPerCta][2 * kWarpMaxVictims];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) n_slow = 0;
   if (threadIdx.x < 3) cnt[threadIdx.x] = 0;
   __syncthreads();
-  // segments are dealt to CTAs round-robin, so that the segments of one
-  // sequence (which share a budget, and so need the whole-CTA path at the
-  // same steps) spread over many CTAs
-  const int item = warp * gridDim.x + blockIdx.x;
+  // Segments are dealt to warps through a multiplicative bijection of
+  // [0, items) (the multiplier is a prime above any item count), so that the
+  // segments of one sequence, which share a budget and so need the whole-CTA
+  // path at the same steps, land in different CTAs.
+  const int slot = blockIdx.x * kSegsPerCta + warp;
+  const int item = slot < items ? (int)(((unsigned long long)slot * 2654435761ull) % (unsigned long long)items) : items;
   if (item < items) {
     WarpCounts wc;
-    if (!evict_segment_warp<D, CI8>(c, pol, a, item, lane, &wc)) {
+    if (!evict_segment_warp<D, CI8>(c, pol, a, item, lane, &wc, pairs[warp])) {
       if (lane == 0) slow_items[atomicAdd(&n_slow, 1)] = item;
     } else if (lane == 0) {
       if (wc.scanned) atomicAdd(&cnt[0], (unsigned long long)wc.scanned);

@@ -5,6 +5,7 @@
 
 #include "common.cuh"
 #include "prof.h"
+#include "warp_select.cuh"
 
 namespace confkv {
 
@@ -39,6 +40,7 @@ struct PrefillLaunch {
   const float* prio;      // [nl][B][Hkv][t_stride] (fixed mode) or null
   int32_t* keep_list;     // fixed mode: [items][fixed_budget] positions kept (ascending)
   int32_t* keep_count;    // fixed mode: [items]
+  EvictCand* cand;        // [S] eviction candidates, invalidated for the segments ingested
 };
 cudaError_t launch_prefill(const Cache& c, const Policy& pol, const PrefillLaunch& a, cudaStream_t st,
                            long long* launches, Prof* prof);
@@ -61,6 +63,7 @@ struct AttnLaunch {
   int num_sms;
   unsigned char* qfrag;   // [S][qf_stride] query operands prepared by the append kernel
   int qf_stride;
+  EvictCand* cand;        // [S] eviction candidates written by the EMA pass (confidence mode)
 };
 cudaError_t launch_decode_attn(const Cache& c, const Policy& pol, const AttnLaunch& a, cudaStream_t st,
                                long long* launches, Prof* prof);
@@ -74,6 +77,7 @@ struct EvictLaunch {
   uint32_t* vmask;        // [S][mask_words] victim bitmask scratch
   int mask_words;
   int stable;             // 1: order-preserving compaction
+  EvictCand* cand;        // [S] candidates from this step's EMA pass (used when their stamp matches)
 };
 cudaError_t launch_evict_compact(const Cache& c, const Policy& pol, const EvictLaunch& a, cudaStream_t st,
                                  long long* launches, Prof* prof);

@@ -30,6 +30,7 @@ __global__ void __launch_bounds__(NT) prefill_meta_kernel(Cache c, PrefillLaunch
   if (threadIdx.x == 0) {
     c.n_cold[s] = c.W > 0 ? max(0, len - c.W + 1) : len;
     c.next_pos[s] = len;
+    if (a.cand) a.cand[s].stamp = -1;
   }
 }
 
@@ -74,6 +75,7 @@ __global__ void __launch_bounds__(NT) prefill_select_kernel(Cache c, Policy pol,
     a.keep_count[item] = min(kept, pol.fixed_budget);
     c.n_cold[s] = cold;
     c.next_pos[s] = len;
+    if (a.cand) a.cand[s].stamp = -1;
   }
 }
 

@@ -105,6 +105,7 @@ typedef struct {
   int64_t moved_rows;         /* cumulative rows moved by compaction */
   int64_t requant_rows;       /* cumulative tokens converted FP16 -> INT8 */
   int64_t kernel_launches;    /* cumulative kernels launched by this handle */
+  int64_t evict_block_segments; /* cumulative segments evicted by the whole-CTA path (many victims) */
 } confkv_stats;
 
 /* Fill *p with the defaults: CONF mode, N_low 256, N_high 512, tau 0.6,

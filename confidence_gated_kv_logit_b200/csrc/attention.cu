@@ -242,7 +242,8 @@ struct Cfg {
   static constexpr int NBW = D / 32;            // 8-dimension n-blocks of P.V per consumer warp
   static constexpr int HPL = GP / 4;            // heads per lane in the int8 score layout
   static constexpr int PS_OFF = NSTAGE * STAGE;
-  static constexpr int PS_BYTES = NCW * GP * 32 * 4;
+  static constexpr int PSTR = 40;               // floats per probability row (conflict-free stores)
+  static constexpr int PS_BYTES = NCW * GP * PSTR * 4;
   static constexpr int FB_OFF = PS_OFF + PS_BYTES;
   static constexpr int FB_ONE = 4 * MB * 32;    // uint4 per buffer
   static constexpr int FB_BYTES = 2 * FB_ONE * 16;
@@ -250,7 +251,9 @@ struct Cfg {
   static constexpr int LS_OFF = WM_OFF + NCW * GP * 4;
   static constexpr int BAR_OFF = LS_OFF + NCW * GP * 4;
   static constexpr int FLAG_OFF = BAR_OFF + 2 * NSTAGE * 8;
-  static constexpr int SMEM = FLAG_OFF + 16;
+  static constexpr int UQ = 8;                  // unit-id queue entries (> NSTAGE)
+  static constexpr int UQ_OFF = FLAG_OFF + 16;
+  static constexpr int SMEM = UQ_OFF + UQ * 4;
 };
 
 struct Unit {
@@ -333,22 +336,56 @@ __device__ __forceinline__ void update_max(SoftmaxState<D, GP>& st, const float*
   }
 }
 
+// Floats per row of a warp's probability buffer: 40 (not 32) puts the rows of
+// the four heads a lane group writes at once in different banks.
+constexpr int kPstr = 40;
+
 // Byte `k` of each of four words, packed into one word (w0 lowest).
 __device__ __forceinline__ uint32_t pack_plane(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, int k) {
   const uint32_t s = (uint32_t)k | ((uint32_t)(k + 4) << 4);
   return __byte_perm(__byte_perm(w0, w1, s), __byte_perm(w2, w3, s), 0x5410);
 }
 
+// Per-lane offsets of the ldmatrix row addresses within a staged tile; they
+// depend only on the lane and the warp, so they are computed once. With rows
+// starting at multiples of 8 and the placement of layout.cuh, the chunk XOR of
+// a row is (lane & 7) for every tile.
+struct LaneOffsets {
+  uint32_t k8_row;     // INT8 K: row (warp*32 + r0) * D, r0 = (lane&7) + 8*((lane>>3)&1)
+  uint32_t kx;         // chunk bits (lane>>4) XOR (lane&7), as a byte offset
+  uint32_t h_row;      // fp16 K: row (warp*16 + r0) * 2D
+  uint32_t v8[2];      // INT8 V: offset of this lane's 16 bytes for n-block pair 0/1, k-step 0
+  uint32_t hv[2];      // fp16 V (.trans): offset for n-block pair 0/1, k-step 0
+};
+
+template <int D>
+__device__ __forceinline__ LaneOffsets lane_offsets(int warp, int lane) {
+  LaneOffsets o;
+  const int r0 = (lane & 7) + 8 * ((lane >> 3) & 1);
+  o.k8_row = (uint32_t)((warp * 32 + r0) * D);
+  o.kx = (uint32_t)((((lane >> 4) ^ (lane & 7)) & 7) << 4);
+  o.h_row = (uint32_t)((warp * 16 + r0) * 2 * D);
+#pragma unroll
+  for (int nbp = 0; nbp < 2; ++nbp) {
+    const int d = warp * (D / 4) + nbp * 16 + (lane & 7) + 8 * (lane >> 4);
+    o.v8[nbp] = (uint32_t)swz128((size_t)d * 32 + 16 * ((lane >> 3) & 1));
+    const int dh = warp * (D / 4) + nbp * 16 + 8 * (lane >> 4);
+    o.hv[nbp] = (uint32_t)h_off(r0, 2 * dh, D);
+  }
+  return o;
+}
+
 struct TileCtx {
   const unsigned char* sb;   // the staged tile
   int j0, cnt;               // first row of the tile in its region; rows present
   bool ok;                   // the tile arrived
-  float* ps;                 // this warp's probability rows [GP][32]
+  float* ps;                 // this warp's probability rows [GP][kPstr]
   uint4* fb;                 // A operands of P.V for this tile, [k-step][mb][lane]
   float* wmax;               // [4][GP]
   volatile int* abort_flag;
   float* sc_base;            // scores of this segment, [G][score_stride]
   int warp, lane;
+  LaneOffsets lo;
 };
 
 // One INT8 tile (128 tokens): warp w scores tokens 32w..32w+31 and builds the
@@ -379,7 +416,10 @@ __device__ __forceinline__ bool consume_i8(const Cache& c, const AttnLaunch& a, 
 #pragma unroll
     for (int kb = 0; kb < KB; ++kb) {
       uint32_t af[4];
-      ldsm_x4(af, kt + (uint32_t)k8_off(rb + (lane & 7) + ((lane >> 3) & 1) * 8, kb * 32 + (lane >> 4) * 16, D));
+      if constexpr (D == 128)   // 128-byte rows: the chunk XOR is the row index mod 8 = lane & 7
+        ldsm_x4(af, kt + x.lo.k8_row + mb2 * 16 * D + (((uint32_t)kb << 5) ^ x.lo.kx));
+      else
+        ldsm_x4(af, kt + (uint32_t)k8_off(rb + (lane & 7) + ((lane >> 3) & 1) * 8, kb * 32 + (lane >> 4) * 16, D));
 #pragma unroll
       for (int nb = 0; nb < NB; ++nb) mma_s8s8(sacc[nb], af, qi[kb][nb].x, qi[kb][nb].y);
     }
@@ -439,7 +479,7 @@ __device__ __forceinline__ bool consume_i8(const Cache& c, const AttnLaunch& a, 
         const float uu = u[mb2][hr][j];
         const float p = uu == -CUDART_INF_F ? 0.0f : exp2f(uu - mh);
         st.lp8[j] += p;
-        x.ps[head * 32 + rl] = p == 0.0f ? 0.0f : p * vsc[warp * 32 + rl];
+        x.ps[head * kPstr + rl] = p == 0.0f ? 0.0f : p * vsc[warp * 32 + rl];
       }
   }
   if (lane == 0) n_rows += max(0, min(32, x.cnt - warp * 32));
@@ -451,8 +491,8 @@ __device__ __forceinline__ bool consume_i8(const Cache& c, const AttnLaunch& a, 
   const float sP = pow2i(E);
   const int ha = GP == 4 ? (g & 3) : g;
   {
-    const float4 v0 = *reinterpret_cast<const float4*>(x.ps + ha * 32 + 4 * t);
-    const float4 v1 = *reinterpret_cast<const float4*>(x.ps + ha * 32 + 16 + 4 * t);
+    const float4 v0 = *reinterpret_cast<const float4*>(x.ps + ha * kPstr + 4 * t);
+    const float4 v1 = *reinterpret_cast<const float4*>(x.ps + ha * kPstr + 16 + 4 * t);
     const uint32_t P0 = __float2uint_rn(v0.x * sP), P1 = __float2uint_rn(v0.y * sP);
     const uint32_t P2 = __float2uint_rn(v0.z * sP), P3 = __float2uint_rn(v0.w * sP);
     const uint32_t P4 = __float2uint_rn(v1.x * sP), P5 = __float2uint_rn(v1.y * sP);
@@ -492,9 +532,8 @@ __device__ __forceinline__ bool consume_i8(const Cache& c, const AttnLaunch& a, 
     }
 #pragma unroll
     for (int nbp = 0; nbp < NBW / 2; ++nbp) {
-      const int d = warp * (D / 4) + nbp * 16 + (lane & 7) + 8 * (lane >> 4);
       uint32_t bf[4];
-      ldsm_x4(bf, vt + (uint32_t)swz128((size_t)(ks * D + d) * 32 + 16 * ((lane >> 3) & 1)));
+      ldsm_x4(bf, vt + (uint32_t)(ks * 32 * D) + x.lo.v8[nbp]);   // ks*32*D is a multiple of 2 KB
 #pragma unroll
       for (int mb = 0; mb < MB; ++mb) {
         mma_u8s8(ia[mb][2 * nbp], af[mb], bf[0], bf[1]);
@@ -537,7 +576,7 @@ __device__ __forceinline__ bool consume_h(const Cache& c, const AttnLaunch& a, c
 #pragma unroll
   for (int ks = 0; ks < KS; ++ks) {
     uint32_t af[4];
-    ldsm_x4(af, kt + (uint32_t)h_off(rb + (lane & 7) + ((lane >> 3) & 1) * 8, ks * 32 + (lane >> 4) * 16, D));
+    ldsm_x4(af, kt + x.lo.h_row + (((uint32_t)ks << 5) ^ x.lo.kx));
     mma_f16(f, af, qh[ks].x, qh[ks].y);
   }
   float u[2][2];
@@ -582,7 +621,7 @@ __device__ __forceinline__ bool consume_h(const Cache& c, const AttnLaunch& a, c
         const float uu = u[hr][cc];
         const float p = uu == -CUDART_INF_F ? 0.0f : exp2f(uu - mh);
         st.lp16[cc] += p;
-        x.ps[head * 32 + g + 8 * hr] = p;
+        x.ps[head * kPstr + g + 8 * hr] = p;
       }
     }
   }
@@ -596,8 +635,8 @@ __device__ __forceinline__ bool consume_h(const Cache& c, const AttnLaunch& a, c
   // ---- P.V operand of k-step `warp`: p = hi + lo in fp16 ----
   {
     const int ha = GP == 4 ? (g & 3) : g;
-    const float2 pa = *reinterpret_cast<const float2*>(x.ps + ha * 32 + 2 * t);
-    const float2 pb = *reinterpret_cast<const float2*>(x.ps + ha * 32 + 8 + 2 * t);
+    const float2 pa = *reinterpret_cast<const float2*>(x.ps + ha * kPstr + 2 * t);
+    const float2 pb = *reinterpret_cast<const float2*>(x.ps + ha * kPstr + 8 + 2 * t);
     const __half2 ha2 = __float22half2_rn(pa), hb2 = __float22half2_rn(pb);
     const float2 fa = __half22float2(ha2), fb2 = __half22float2(hb2);
     const __half2 la2 = __float22half2_rn(make_float2(pa.x - fa.x, pa.y - fa.y));
@@ -621,9 +660,8 @@ __device__ __forceinline__ bool consume_h(const Cache& c, const AttnLaunch& a, c
     const uint32_t af[4] = {fr.x, fr.y, fr.z, fr.w};
 #pragma unroll
     for (int nbp = 0; nbp < NBW / 2; ++nbp) {
-      const int d0 = warp * (D / 4) + nbp * 16;
       uint32_t bf[4];
-      ldsm_x4_t(bf, vt + (uint32_t)h_off(ks * 16 + (lane & 7) + 8 * ((lane >> 3) & 1), 2 * (d0 + 8 * (lane >> 4)), D));
+      ldsm_x4_t(bf, vt + (uint32_t)(ks * 16 * 2 * D) + x.lo.hv[nbp]);   // 16 rows: a multiple of the XOR period
       mma_f16(st.acc[0][2 * nbp], af, bf[0], bf[1]);
       mma_f16(st.acc[0][2 * nbp + 1], af, bf[2], bf[3]);
     }
@@ -644,6 +682,7 @@ __global__ void __launch_bounds__(160, 2) attn_kernel(Cache c, AttnLaunch a, int
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   uint64_t* empty = full + C::NSTAGE;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::FLAG_OFF);
+  volatile int* uq = reinterpret_cast<volatile int*>(smem + C::UQ_OFF);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -667,20 +706,45 @@ __global__ void __launch_bounds__(160, 2) attn_kernel(Cache c, AttnLaunch a, int
     // One lane issues every copy. On a timed-out wait the copies already
     // issued are waited for (bounded) so that none lands after the CTA exits.
     if (lane == 0) {
+      // Units are claimed one at a time from a launch-wide counter, so CTAs
+      // that drew short segments take more of them (no static tail). Each
+      // claimed unit id goes into the queue uq before the unit's first stage
+      // is published; a unit without tiles, and the end, are published as a
+      // stage without data.
       int ctr = 0;
       bool stop = false;
-      for (int unit = blockIdx.x; unit < units && !stop; unit += gridDim.x) {
+      auto next_stage = [&]() -> int {
+        const int st = ctr % C::NSTAGE;
+        if (ctr >= C::NSTAGE && !mbar_wait_bounded(&empty[st], ((ctr / C::NSTAGE) - 1) & 1)) {
+          set_error(c.err, kErrDevice);
+          *abort_flag = 1;
+        }
+        if (*abort_flag) stop = true;
+        return st;
+      };
+      for (int k = 0; !stop; ++k) {
+        const int unit = atomicAdd(a.sched, 1);
+        if (unit >= units) {
+          const int st = next_stage();
+          uq[k % C::UQ] = -1;                       // the end
+          if (!stop) {
+            mbar_arrive(&full[st]);
+            ++ctr;
+          }
+          break;
+        }
         const Unit u = make_unit<D, GP, CI8>(c, a.r, splits, unit);
+        uq[k % C::UQ] = unit;
+        if (u.t0 == u.t1) {
+          const int st = next_stage();
+          if (stop) break;
+          mbar_arrive(&full[st]);                   // no data: the consumers only close the unit
+          ++ctr;
+          continue;
+        }
         for (int t = u.t0; t < u.t1; ++t) {
-          const int st = ctr % C::NSTAGE;
-          if (ctr >= C::NSTAGE && !mbar_wait_bounded(&empty[st], ((ctr / C::NSTAGE) - 1) & 1)) {
-            set_error(c.err, kErrDevice);
-            *abort_flag = 1;
-          }
-          if (*abort_flag) {
-            stop = true;
-            break;
-          }
+          const int st = next_stage();
+          if (stop) break;
           unsigned char* sb = stages + st * C::STAGE;
           const bool cold = t < u.tiles_c;
           const int j0 = cold ? t * C::TTC : (t - u.tiles_c) * C::TTR;
@@ -735,8 +799,19 @@ __global__ void __launch_bounds__(160, 2) attn_kernel(Cache c, AttnLaunch a, int
 
   // -------------------------------- consumers --------------------------------
   const int g = lane >> 2, t = lane & 3;
+  const LaneOffsets lane_offs = lane_offsets<D>(warp, lane);
   int ctr = 0;
-  for (int unit = blockIdx.x; unit < units; unit += gridDim.x) {
+  for (int k = 0;; ++k) {
+    // the next unit: its id is published with its first stage
+    {
+      const bool ok = mbar_wait_bounded(&full[ctr % C::NSTAGE], (ctr / C::NSTAGE) & 1);
+      if (!ok) {
+        set_error(c.err, kErrDevice);
+        *abort_flag = 1;
+      }
+    }
+    const int unit = uq[k % C::UQ];
+    if (named_barrier_or(2, 128, unit < 0 || *abort_flag != 0)) break;   // the end, or an abort
     const Unit u = make_unit<D, GP, CI8>(c, a.r, splits, unit);
     const unsigned char* qf = a.qfrag + (size_t)u.s * a.qf_stride;
     uint2 qi[C::KB][C::NB];
@@ -769,13 +844,19 @@ __global__ void __launch_bounds__(160, 2) attn_kernel(Cache c, AttnLaunch a, int
     unsigned long long n_rows_c = 0, n_rows_r = 0;
 
     TileCtx x;
-    x.ps = ps_all + warp * GP * 32;
+    x.ps = ps_all + warp * GP * kPstr;
     x.wmax = wmax;
     x.abort_flag = abort_flag;
     x.sc_base = a.scores + (size_t)u.s * c.G * a.score_stride;
     x.warp = warp;
     x.lane = lane;
+    x.lo = lane_offs;
     bool aborted = false;
+    if (u.t0 == u.t1) {   // a stage without data: release it and close the unit
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[ctr % C::NSTAGE]);
+      ++ctr;
+    }
     for (int tt = u.t0; tt < u.t1; ++tt) {
       const int stg = ctr % C::NSTAGE;
       x.ok = mbar_wait_bounded(&full[stg], (ctr / C::NSTAGE) & 1);
@@ -867,6 +948,11 @@ __global__ void __launch_bounds__(160, 2) attn_kernel(Cache c, AttnLaunch a, int
     if (named_barrier_or(2, 128, aborted || *abort_flag != 0)) break;
   }
   __syncthreads();
+  // the last CTA to finish resets the unit counter for the next launch
+  if (threadIdx.x == 0 && atomicAdd(a.sched + 1, 1) == (int)gridDim.x - 1) {
+    a.sched[0] = 0;
+    a.sched[1] = 0;
+  }
 }
 
 // ---------------------------------------------------------------------------

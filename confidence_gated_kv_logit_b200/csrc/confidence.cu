@@ -72,18 +72,23 @@ __global__ void __launch_bounds__(NT) confidence_kernel(ConfLaunch a, Policy pol
   const int v1 = min(a.V, v0 + chunk);
   const float* lg = a.logits + (size_t)row * a.V;
 
-  ConfPartial p;
-  p.m = -CUDART_INF_F;
-  p.S = 0.0f;
-  p.T = 0.0f;
-  p.top1 = -CUDART_INF_F;
-  p.top2 = -CUDART_INF_F;
-  p.bad = 0;
-  // Each pass loads U logits per thread into registers, then reduces them in
-  // two sweeps: the maximum first, then S and T relative to it (no rescaling
-  // per element), with the top two kept branch-free (counted with
-  // multiplicity: t2 = max(t2, min(t1, x)), t1 = max(t1, x)).
-  constexpr int U = 8;
+  // Each pass loads U logits per thread into registers (a CTA's whole chunk
+  // in one pass when the row is split vocab/4096 ways). The CTA first agrees on
+  // the pass maximum M, so every thread sums S = sum e^(l-M) and
+  // T = sum e^(l-M)(l-M) against the same M and the block reductions are plain
+  // sums; the top two are kept branch-free, counted with multiplicity
+  // (t2 = max(t2, min(t1, x)), t1 = max(t1, x)).
+  __shared__ float red[NT / 32][4];
+  __shared__ int red_bad[NT / 32];
+  constexpr int U = 16;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  ConfPartial cta;   // meaningful in thread 0
+  cta.m = -CUDART_INF_F;
+  cta.S = 0.0f;
+  cta.T = 0.0f;
+  cta.top1 = -CUDART_INF_F;
+  cta.top2 = -CUDART_INF_F;
+  cta.bad = 0;
   for (int base = v0; base < v1; base += NT * U) {
     float x[U];
 #pragma unroll
@@ -91,48 +96,74 @@ __global__ void __launch_bounds__(NT) confidence_kernel(ConfLaunch a, Policy pol
       const int i = base + u * NT + threadIdx.x;
       x[u] = i < v1 ? __ldcs(lg + i) : -CUDART_INF_F;
     }
-    float mx = -CUDART_INF_F;
-    int bad = 0;
+    float mx = -CUDART_INF_F, t1 = -CUDART_INF_F, t2 = -CUDART_INF_F;
+    bool bad = false;
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int i = base + u * NT + threadIdx.x;
       const bool finite = fabsf(x[u]) <= 3.402823466e38f;
-      bad |= (i < v1 && !finite) ? 1 : 0;
+      bad |= i < v1 && !finite;
       if (!finite) x[u] = -CUDART_INF_F;        // out of range or non-finite: no contribution
       mx = fmaxf(mx, x[u]);
-      p.top2 = fmaxf(p.top2, fminf(p.top1, x[u]));
-      p.top1 = fmaxf(p.top1, x[u]);
+      t2 = fmaxf(t2, fminf(t1, x[u]));
+      t1 = fmaxf(t1, x[u]);
     }
-    p.bad |= bad;
-    if (mx == -CUDART_INF_F) continue;
+    mx = warp_max(mx);
+    if (lane == 0) red[wid][0] = mx;
+    __syncthreads();
+    float M = red[0][0];
+#pragma unroll
+    for (int w = 1; w < NT / 32; ++w) M = fmaxf(M, red[w][0]);
     float S = 0.0f, T = 0.0f;
+    if (M != -CUDART_INF_F) {
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const float d = x[u] - mx;                // -inf for the excluded elements
-      const float ev = __expf(d);               // 0 for them
-      S += ev;
-      T = fmaf(ev, ev > 0.0f ? d : 0.0f, T);
+      for (int u = 0; u < U; ++u) {
+        const float d = x[u] - M;                 // -inf for the excluded elements
+        const float ev = __expf(d);               // 0 for them
+        S += ev;
+        T = fmaf(ev, ev > 0.0f ? d : 0.0f, T);
+      }
     }
-    ConfPartial q;
-    q.m = mx;
-    q.S = S;
-    q.T = T;
-    q.top1 = -CUDART_INF_F;
-    q.top2 = -CUDART_INF_F;
-    q.bad = 0;
-    merge(p, q);
-  }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const ConfPartial q = shfl_partial(p, o);
-    merge(p, q);
+    for (int o = 16; o > 0; o >>= 1) {
+      S += __shfl_xor_sync(0xffffffffu, S, o);
+      T += __shfl_xor_sync(0xffffffffu, T, o);
+      const float o1 = __shfl_xor_sync(0xffffffffu, t1, o), o2 = __shfl_xor_sync(0xffffffffu, t2, o);
+      t2 = fmaxf(fminf(t1, o1), fmaxf(t2, o2));
+      t1 = fmaxf(t1, o1);
+    }
+    const bool wbad = __any_sync(0xffffffffu, bad);
+    __syncthreads();   // every thread has read red[.][0]
+    if (lane == 0) {
+      red[wid][0] = S;
+      red[wid][1] = T;
+      red[wid][2] = t1;   // the warp's top two
+      red[wid][3] = t2;
+      red_bad[wid] = wbad ? 1 : 0;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      ConfPartial q;
+      q.m = M;
+      q.S = 0.0f;
+      q.T = 0.0f;
+      q.top1 = -CUDART_INF_F;
+      q.top2 = -CUDART_INF_F;
+      q.bad = 0;
+      for (int w = 0; w < NT / 32; ++w) {
+        q.S += red[w][0];
+        q.T += red[w][1];
+        q.bad |= red_bad[w];
+        q.top2 = fmaxf(fminf(q.top1, red[w][2]), fmaxf(q.top2, red[w][3]));
+        q.top1 = fmaxf(q.top1, red[w][2]);
+      }
+      if (M == -CUDART_INF_F) q.S = 0.0f;
+      merge(cta, q);
+    }
+    __syncthreads();   // red is reused by the next pass
   }
-  if ((threadIdx.x & 31) == 0) wpart[threadIdx.x >> 5] = p;
-  __syncthreads();
   if (threadIdx.x == 0) {
-    ConfPartial acc = wpart[0];
-    for (int w = 1; w < NT / 32; ++w) merge(acc, wpart[w]);
-    a.part[(size_t)row * a.cpr + blockIdx.x] = acc;
+    a.part[(size_t)row * a.cpr + blockIdx.x] = cta;
     __threadfence();
     const unsigned prev = atomicAdd(&a.tickets[row], 1u);
     is_last = (prev == (unsigned)a.cpr - 1u);
@@ -169,32 +200,37 @@ __global__ void __launch_bounds__(NT) confidence_kernel(ConfLaunch a, Policy pol
   __syncthreads();   // every thread is done with wpart from the first merge
   if ((threadIdx.x & 31) == 0) wpart[threadIdx.x >> 5] = acc;
   __syncthreads();
-  if (threadIdx.x != 0) return;
-  acc = wpart[0];
-  for (int w = 1; w < NT / 32; ++w) merge(acc, wpart[w]);
-  a.tickets[row] = 0u;   // ready for the next launch
-
-  float c;
-  int N;
-  const int larger = max(pol.n_low, pol.n_high);
-  if (acc.bad || !(acc.S > 0.0f)) {
-    c = CUDART_NAN_F;
-    N = larger;
-    set_error(a.err, kErrNonfinite);
-  } else {
-    const float H = logf(acc.S) - acc.T / acc.S;
-    const float norm_entropy = H / logf((float)a.V);
-    const float margin = acc.top1 - acc.top2;
-    const float sig = 1.0f / (1.0f + expf(-margin));
-    const float p_max = 1.0f / acc.S;
-    c = 0.4f * (1.0f - norm_entropy) + 0.3f * sig + 0.3f * p_max;
-    const bool confident = c >= pol.tau;
-    if (pol.gate == 0) N = confident ? pol.n_low : pol.n_high;
-    else N = confident ? pol.n_high : pol.n_low;
+  __shared__ int n_sh;
+  if (threadIdx.x == 0) {
+    acc = wpart[0];
+    for (int w = 1; w < NT / 32; ++w) merge(acc, wpart[w]);
+    a.tickets[row] = 0u;   // ready for the next launch
+    float c;
+    int N;
+    const int larger = max(pol.n_low, pol.n_high);
+    if (acc.bad || !(acc.S > 0.0f)) {
+      c = CUDART_NAN_F;
+      N = larger;
+      set_error(a.err, kErrNonfinite);
+    } else {
+      const float H = logf(acc.S) - acc.T / acc.S;
+      const float norm_entropy = H / logf((float)a.V);
+      const float margin = acc.top1 - acc.top2;
+      const float sig = 1.0f / (1.0f + expf(-margin));
+      const float p_max = 1.0f / acc.S;
+      c = 0.4f * (1.0f - norm_entropy) + 0.3f * sig + 0.3f * p_max;
+      const bool confident = c >= pol.tau;
+      if (pol.gate == 0) N = confident ? pol.n_low : pol.n_high;
+      else N = confident ? pol.n_high : pol.n_low;
+    }
+    a.c_ws[row] = c;
+    if (a.c_out) a.c_out[row] = c;
+    n_sh = N;
   }
-  a.c_ws[row] = c;
-  if (a.c_out) a.c_out[row] = c;
-  for (int l = 0; l < a.L; ++l) {
+  __syncthreads();
+  // the per-layer budgets, one layer per thread
+  const int N = n_sh;
+  for (int l = threadIdx.x; l < a.L; l += NT) {
     int bl = N;
     if (pol.pyramidal && a.L > 1) {
       const long long L1 = a.L - 1;

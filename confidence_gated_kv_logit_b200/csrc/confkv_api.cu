@@ -18,7 +18,7 @@ namespace {
 
 constexpr uint32_t kMagic = 0xC0F1C0DEu;
 constexpr uint32_t kDead = 0xDEADC0DEu;
-constexpr int kMaxCpr = 128;   // CTAs per logit row (one per ~8192 logits)
+constexpr int kMaxCpr = 128;   // CTAs per logit row (one per ~4096 logits)
 
 struct Buffers {
   std::vector<void*> ptrs;
@@ -79,6 +79,9 @@ struct confkv_handle {
   unsigned char* qfrag;          // [S][qf_stride] query operands of the attention kernel
   int qf_stride;
   confkv::EvictCand* cand;       // [S] eviction candidates from the EMA pass
+  uint32_t* kscratch;            // evict scratch, per CTA of the largest evict grid
+  int* sched;                    // attention unit counters (zero between launches)
+  int scratch_stride;
   int32_t* keep_list;
   int32_t* keep_count;
   long long launches;
@@ -288,6 +291,9 @@ confkv_status confkv_create(int32_t layers, int32_t kv_heads, int32_t q_heads, i
   h->qf_stride = confkv::qfrag_bytes(head_dim, G);
   chk(B.alloc(&h->qfrag, S * (size_t)h->qf_stride));
   chk(B.alloc(&h->cand, S));
+  chk(B.alloc(&h->sched, 2));
+  h->scratch_stride = 3 * c.cap + c.Wst;
+  chk(B.alloc(&h->kscratch, (size_t)confkv::evict_grid((int)S) * h->scratch_stride));
   if (p.mode == CONFKV_MODE_FIXED) {
     chk(B.alloc(&h->keep_list, S * (size_t)p.fixed_budget));
     chk(B.alloc(&h->keep_count, S));
@@ -316,6 +322,7 @@ confkv_status confkv_create(int32_t layers, int32_t kv_heads, int32_t q_heads, i
     chk(cudaMemset(h->scores, 0, S * G * (size_t)h->score_stride * 4));
     chk(cudaMemset(h->qfrag, 0, S * (size_t)h->qf_stride));
     chk(cudaMemset(h->cand, 0xff, S * sizeof(confkv::EvictCand)));   // stamp -1: no record
+    chk(cudaMemset(h->sched, 0, 2 * sizeof(int)));
     chk(cudaDeviceSynchronize());
   }
   if (e != cudaSuccess) {
@@ -412,7 +419,7 @@ confkv_status confkv_confidence(confkv_handle* h, const float* logits, int32_t b
   a.L = h->L;
   a.part = h->cpart;
   a.tickets = h->tickets;
-  a.cpr = std::max(1, std::min(kMaxCpr, (vocab + 8191) / 8192));
+  a.cpr = std::max(1, std::min(kMaxCpr, (vocab + 4095) / 4096));
   a.c_ws = h->c_ws;
   a.budget_ws = h->budget;
   a.c_out = c_out;
@@ -457,6 +464,7 @@ confkv_status confkv_decode_attn(confkv_handle* h, int32_t layer, const void* q,
   a.qfrag = h->qfrag;
   a.qf_stride = h->qf_stride;
   a.cand = h->cand;
+  a.sched = h->sched;
   cudaError_t e =
       confkv::launch_decode_attn(h->c, h->pol, a, static_cast<cudaStream_t>(stream), &h->launches, h->prof_ptr());
   if (e != cudaSuccess) return cuda_status(e);
@@ -478,6 +486,9 @@ confkv_status confkv_evict_compact(confkv_handle* h, int32_t layer, void* stream
   a.mask_words = h->mask_words;
   a.stable = h->p.compact == CONFKV_COMPACT_STABLE;
   a.cand = h->cand;
+  a.kscratch = h->kscratch;
+  a.scratch_stride = h->scratch_stride;
+  a.scratch_keys = h->c.cap + h->c.Wst;
   cudaError_t e =
       confkv::launch_evict_compact(h->c, h->pol, a, static_cast<cudaStream_t>(stream), &h->launches, h->prof_ptr());
   if (e != cudaSuccess) return cuda_status(e);

@@ -294,6 +294,67 @@ __device__ bool evict_segment_warp(const Cache& c, const Policy& pol, const Evic
   return true;
 }
 
+// Pairs p in [0, np): move cold row movers[p] into holes[p] (all holes are
+// below n_keep, all movers at or above it, so no move reads a row another
+// writes). Called by every thread of the CTA.
+template <int D, bool CI8>
+__device__ __forceinline__ void move_pairs_warp(const Cache& c, int s, const int* __restrict__ holes,
+                                                const int* __restrict__ movers, int np, int n_keep, int n_cold) {
+  using R = Rows<D, CI8>;
+  const int lane = threadIdx.x & 31;
+  const size_t base = (size_t)s * c.cap * D;
+  for (int p0 = threadIdx.x & ~31; p0 < np; p0 += NT) {
+    const int p = p0 + lane;
+    const bool on = p < np;
+    const int src = on ? movers[p] : 0, dst = on ? holes[p] : 0;
+    if (kChecked && on && !guard(dst >= 0 && dst < n_keep && src >= n_keep && src < n_cold, c.err, kSiteEvictPair,
+                                 s, src))
+      continue;
+    // K (or fp16 K and V) rows: 16-byte chunks, four in flight
+    constexpr int CH = CI8 ? R::KP : R::NP;   // fp16 rows move K and V by chunks
+#pragma unroll
+    for (int c0 = 0; c0 < CH; c0 += 4) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (on && c0 + u < CH) v[u] = load_part<D, CI8>(c, s, src, c0 + u);
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (on && c0 + u < CH) store_part<D, CI8>(c, s, dst, c0 + u, v[u]);
+    }
+    if constexpr (CI8) {
+      // V codes: dimension-major, one byte per dimension, 16 dimensions in flight
+      const unsigned char* vsrc = reinterpret_cast<const unsigned char*>(c.v8 + base);
+      unsigned char* vdst = reinterpret_cast<unsigned char*>(c.v8 + base);
+#pragma unroll 1
+      for (int d0 = 0; d0 < D; d0 += 16) {
+        unsigned char b[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) b[u] = on ? vsrc[v8_off(src, d0 + u, D)] : 0;
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+          if (on) vdst[v8_off(dst, d0 + u, D)] = b[u];
+      }
+    }
+    if (on) {
+      const size_t so = (size_t)s * c.cap + src, dO = (size_t)s * c.cap + dst;
+      const int pv = c.pos_c[so];
+      const float sv = c.sc_c[so];
+      float kv = 0.0f, vv = 0.0f;
+      if (CI8) {
+        kv = c.ks[so];
+        vv = c.vs[so];
+      }
+      c.pos_c[dO] = pv;
+      c.sc_c[dO] = sv;
+      if (CI8) {
+        c.ks[dO] = kv;
+        c.vs[dO] = vv;
+      }
+    }
+  }
+}
+
 struct EvictSmem {
   SelectSmem<NT> sm;
   int list_h[NT];
@@ -336,6 +397,7 @@ __device__ void evict_segment_block(const Cache& c, const Policy& pol, const Evi
   int moved = 0;
 
   if (e > 0 && t >= 0) {
+    auto pos_of = [&](int i) -> int { return i < n_cold ? pos_c[i] : pos_r[i - n_cold]; };
     auto key = [&](int i) -> unsigned long long {
       int pos;
       float sc;
@@ -354,8 +416,8 @@ __device__ void evict_segment_block(const Cache& c, const Policy& pol, const Evi
     uint32_t* vm = a.vmask + (size_t)s * a.mask_words;
     auto victim = [&](int i) -> bool { return (vm[i >> 5] >> (i & 31)) & 1u; };
     if (e == 1 && !a.stable) {
-      // steady state: one victim; its index comes with the argmin, and at most
-      // one row (the last cold row) moves into its place
+      // one victim; its index comes with the argmin, and at most one row (the
+      // last cold row) moves into its place
       int vi;
       block_argmin_idx<NT>(key, span, sm, &vi);
       if (vi >= n_cold) {
@@ -370,45 +432,120 @@ __device__ void evict_segment_block(const Cache& c, const Policy& pol, const Evi
       }
       __syncthreads();
     } else {
-    const SelectResult sel = block_select_smallest<NT>(key, span, e, sm);
-
-    // victim bitmask of the cold region (one ballot per 32 tokens), and count
-    int ecold_here = 0;
-    for (int base = 0; base < n_cold; base += NT) {
-      const int i = base + (int)threadIdx.x;
-      const bool v = i < n_cold && is_selected(key(i), sel);
-      const unsigned bal = __ballot_sync(0xffffffffu, v);
-      if ((threadIdx.x & 31) == 0 && i < n_cold) {
-        vm[i >> 5] = bal;
-        ecold_here += __popc(bal);
+    // High halves of the keys (ordered score bits; 0xFFFFFFFF = never a
+    // victim) into this CTA's scratch, four tokens per thread in flight.
+    uint32_t* __restrict__ khi = a.kscratch + (size_t)blockIdx.x * a.scratch_stride;
+    auto hi_of = [&](int pos, float sc) -> uint32_t {
+      const bool none = pos < 0 || t - pos < pol.P || pos < pol.n_sink;
+      return none ? 0xFFFFFFFFu : (uint32_t)(rank_key(pol, sc, pos, t) >> 32);
+    };
+    // cold region: 8 tokens per thread per step in two 16-byte loads each of
+    // positions and EMA values (the region is a multiple of 64 tokens long)
+    for (int i0 = 8 * threadIdx.x; i0 < n_cold; i0 += 8 * NT) {
+      const int4 p0 = reinterpret_cast<const int4*>(pos_c + i0)[0];
+      const int4 p1 = reinterpret_cast<const int4*>(pos_c + i0)[1];
+      const float4 f0 = reinterpret_cast<const float4*>(sc_c + i0)[0];
+      const float4 f1 = reinterpret_cast<const float4*>(sc_c + i0)[1];
+      const int pp[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+      const float ff[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+      uint32_t hv[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) hv[j] = i0 + j < n_cold ? hi_of(pp[j], ff[j]) : 0xFFFFFFFFu;
+      if (i0 + 8 <= n_cold) {
+        reinterpret_cast<uint4*>(khi + i0)[0] = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+        reinterpret_cast<uint4*>(khi + i0)[1] = make_uint4(hv[4], hv[5], hv[6], hv[7]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (i0 + j < n_cold) khi[i0 + j] = hv[j];
       }
+    }
+    for (int slot = threadIdx.x; slot < W; slot += NT) khi[n_cold + slot] = hi_of(pos_r[slot], sc_r[slot]);
+    __syncthreads();
+    const SelectResult sel = block_select_smallest_hi<NT>(khi, pos_of, span, e, sm);
+    const bool sel_lo = (sel.mask & 0xffffffffull) != 0;   // the low half (position) decides ties
+    auto is_victim = [&](int i) -> bool {
+      const uint32_t hv = khi[i];
+      if (hv == 0xFFFFFFFFu) return false;
+      const unsigned long long k64 = ((unsigned long long)hv << 32) | (sel_lo ? (uint32_t)pos_of(i) : 0u);
+      return is_selected(k64, sel);
+    };
+
+    // victim bitmask of the cold region: each thread builds whole 32-token
+    // words from eight 16-byte loads of the key scratch
+    int ecold_here = 0;
+    for (int w = threadIdx.x; w < ((n_cold + 31) >> 5); w += NT) {
+      uint4 q[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) q[u] = reinterpret_cast<const uint4*>(khi + 32 * w)[u];
+      uint32_t bits = 0u;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const uint32_t hv[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int i = 32 * w + 4 * u + j;
+          if (i < n_cold && hv[j] != 0xFFFFFFFFu) {
+            const unsigned long long k64 = ((unsigned long long)hv[j] << 32) | (sel_lo ? (uint32_t)pos_c[i] : 0u);
+            if (is_selected(k64, sel)) bits |= 1u << (4 * u + j);
+          }
+        }
+      }
+      vm[w] = bits;
+      ecold_here += __popc(bits);
     }
     // window victims free their slot (each thread reads and writes only its own slots)
     for (int slot = threadIdx.x; slot < W; slot += NT)
-      if (is_selected(key(n_cold + slot), sel)) pos_r[slot] = -1;
+      if (is_victim(n_cold + slot)) pos_r[slot] = -1;
     const int e_cold = block_sum_int<NT>(ecold_here, sm);   // includes a block barrier: vm is visible
     const int n_keep = n_cold - e_cold;
 
     if (e_cold == 0) {
       // every victim was in the window ring: the cold region is unchanged
     } else if (!a.stable) {
-      // hole-fill: pair the k-th hole below n_keep with the k-th survivor above it
-      int hcur = 0, mcur = n_keep;
-      while (true) {
-        const int nh = block_collect<NT, NT>([&](int i) { return victim(i); }, &hcur, n_keep, list_h, sm);
-        const int nm = block_collect<NT, NT>([&](int i) { return !victim(i); }, &mcur, n_cold, list_m, sm);
-        const int np = min(nh, nm);
-        if (np == 0) break;
-        for (int w = threadIdx.x; w < np * R::NP; w += NT) {
-          const int p = w / R::NP;
-          if (kChecked && !guard(list_h[p] >= 0 && list_h[p] < n_keep && list_m[p] >= n_keep && list_m[p] < n_cold,
-                                 c.err, kSiteEvictPair, s, list_m[p]))
-            continue;
-          move_cold_row<D, CI8>(c, s, list_m[p], list_h[p], w - p * R::NP);
+      // Hole-fill: the k-th hole below n_keep receives the k-th survivor at or
+      // above it. Both lists come from one pass over the mask words (popcount
+      // and a block scan) into this CTA's scratch.
+      int* __restrict__ holes = reinterpret_cast<int*>(khi + a.scratch_keys);
+      int* __restrict__ movers = holes + c.cap;
+      const int words = (n_cold + 31) >> 5;
+      int hole_base = 0, mover_base = 0;
+      for (int w0 = 0; w0 < words; w0 += NT) {
+        const int w = w0 + (int)threadIdx.x;
+        uint32_t hb = 0u, mb = 0u;
+        const int lo_i = w << 5;
+        if (w < words) {
+          const uint32_t bits = vm[w];
+          const uint32_t valid = lo_i + 32 <= n_cold ? 0xffffffffu : ((1u << (n_cold - lo_i)) - 1u);
+          const uint32_t below = lo_i + 32 <= n_keep ? 0xffffffffu
+                                 : (lo_i >= n_keep ? 0u : ((1u << (n_keep - lo_i)) - 1u));
+          hb = bits & below & valid;
+          mb = ~bits & ~below & valid;
         }
-        moved += np;
-        __syncthreads();
+        int htot, mtot;
+        int ho = hole_base + block_excl_scan_int<NT>(__popc(hb), sm, &htot);
+        int mo = mover_base + block_excl_scan_int<NT>(__popc(mb), sm, &mtot);
+        while (hb) {
+          holes[ho++] = lo_i + __ffs(hb) - 1;
+          hb &= hb - 1u;
+        }
+        while (mb) {
+          movers[mo++] = lo_i + __ffs(mb) - 1;
+          mb &= mb - 1u;
+        }
+        hole_base += htot;
+        mover_base += mtot;
       }
+      __syncthreads();   // the lists are complete and visible
+      const int np = min(hole_base, mover_base);
+      // moves: each warp takes 32 consecutive pairs, lane j the j-th; K rows
+      // move as 16-byte chunks, and V codes one dimension at a time, so that
+      // a warp instruction reads and writes 32 neighbouring bytes of a
+      // dimension-major row whenever the holes and the movers run in order
+      // (as they do in bulk evictions).
+      move_pairs_warp<D, CI8>(c, s, holes, movers, np, n_keep, n_cold);
+      moved = np;
+      __syncthreads();
     } else {
       // stable: from the first hole on, every survivor moves down by the number
       // of victims before it, in chunks staged through shared memory
@@ -538,12 +675,14 @@ cudaError_t run(const Cache& c, const Policy& pol, const EvictLaunch& a, cudaStr
                 Prof* prof) {
   const int items = a.r.items(c.Hkv);
   ProfScope ps(prof, kKEvict, st);
-  evict_kernel<D, CI8><<<(items + kSegsPerCta - 1) / kSegsPerCta, NT, 0, st>>>(c, pol, a, items);
+  evict_kernel<D, CI8><<<evict_grid(items), NT, 0, st>>>(c, pol, a, items);
   ++*launches;
   return cudaGetLastError();
 }
 
 }  // namespace
+
+int evict_grid(int items) { return (items + kSegsPerCta - 1) / kSegsPerCta; }
 
 cudaError_t launch_evict_compact(const Cache& c, const Policy& pol, const EvictLaunch& a, cudaStream_t st,
                                  long long* launches, Prof* prof) {

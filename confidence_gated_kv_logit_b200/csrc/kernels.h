@@ -64,6 +64,7 @@ struct AttnLaunch {
   unsigned char* qfrag;   // [S][qf_stride] query operands prepared by the append kernel
   int qf_stride;
   EvictCand* cand;        // [S] eviction candidates written by the EMA pass (confidence mode)
+  int* sched;             // [2] unit counter and finished-CTA counter of the attention kernel (zero between launches)
 };
 cudaError_t launch_decode_attn(const Cache& c, const Policy& pol, const AttnLaunch& a, cudaStream_t st,
                                long long* launches, Prof* prof);
@@ -78,8 +79,13 @@ struct EvictLaunch {
   int mask_words;
   int stable;             // 1: order-preserving compaction
   EvictCand* cand;        // [S] candidates from this step's EMA pass (used when their stamp matches)
+  uint32_t* kscratch;     // per CTA of the evict grid: key high halves [cap + Wst], then hole and mover lists [cap] each
+  int scratch_stride;     // uint32 words per CTA
+  int scratch_keys;       // offset of the hole list (= cap + Wst)
 };
 cudaError_t launch_evict_compact(const Cache& c, const Policy& pol, const EvictLaunch& a, cudaStream_t st,
                                  long long* launches, Prof* prof);
+// CTAs the evict kernel uses for `items` segments (the scratch is per CTA).
+int evict_grid(int items);
 
 }  // namespace confkv

@@ -209,6 +209,117 @@ __device__ SelectResult block_select_smallest(KeyFn kf, int n, int k, SelectSmem
   return r;
 }
 
+// Exclusive prefix of an int over the block; *total receives the sum.
+template <int NT>
+__device__ __forceinline__ int block_excl_scan_int(int v, SelectSmem<NT>& sm, int* total) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int x = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += x;
+  }
+  if (lane == 31) sm.warp_tot[w] = incl;
+  __syncthreads();
+  int off = 0, tot = 0;
+#pragma unroll
+  for (int i = 0; i < NT / 32; ++i) {
+    const int x = sm.warp_tot[i];
+    off += (i < w) ? x : 0;
+    tot += x;
+  }
+  __syncthreads();
+  *total = tot;
+  return off + incl - v;
+}
+
+// The k smallest of the 64-bit keys (hi[i] << 32) | lo(i), i < n, where
+// hi[i] == 0xFFFFFFFF marks an absent key (1 <= k <= number of present
+// keys): MSD radix select with 8-bit digits, stopping once the bucket holding
+// the k-th key is entirely selected. The high halves come from memory the
+// caller filled once; lo(i) is evaluated only in the passes over the low half
+// (when the high halves alone do not separate the k-th key). Histograms take
+// one shared-memory atomic per distinct digit of a warp (__match_any_sync).
+template <int NT, class LoFn>
+__device__ SelectResult block_select_smallest_hi(const uint32_t* __restrict__ hi, LoFn lo, int n, int k,
+                                                 SelectSmem<NT>& sm) {
+  if (threadIdx.x == 0) {
+    sm.prefix = 0;
+    sm.mask = 0;
+    sm.rem = k;
+    sm.done = 0;
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int wbase = threadIdx.x & ~31;
+  for (int shift = 56; shift >= 0; shift -= 8) {
+    for (int i = threadIdx.x; i < 256; i += NT) sm.hist[i] = 0;
+    __syncthreads();
+    const unsigned long long prefix = sm.prefix, mask = sm.mask;
+    const bool need_lo = shift < 32;
+    // eight keys per thread per step, all loaded before any is counted
+    for (int base = wbase * 8; base < n; base += NT * 8) {   // whole warps step together
+      uint32_t hv[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = base + u * 32 + lane;
+        hv[u] = i < n ? hi[i] : 0xFFFFFFFFu;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = base + u * 32 + lane;
+        unsigned bin = 256u;
+        if (hv[u] != 0xFFFFFFFFu) {
+          unsigned long long key = (unsigned long long)hv[u] << 32;
+          if (need_lo) key |= (uint32_t)lo(i);
+          if ((key & mask) == prefix) bin = (unsigned)((key >> shift) & 255u);
+        }
+        const unsigned peers = __match_any_sync(0xffffffffu, bin);
+        if (bin != 256u && lane == __ffs(peers) - 1) atomicAdd(&sm.hist[bin], (unsigned)__popc(peers));
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      unsigned cnt[8];
+      unsigned tot = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        cnt[j] = sm.hist[lane * 8 + j];
+        tot += cnt[j];
+      }
+      unsigned incl = tot;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      const unsigned excl = incl - tot;
+      const unsigned rem = (unsigned)sm.rem;
+      __syncwarp();
+      if (excl < rem && rem <= incl) {
+        unsigned below = excl;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (below + cnt[j] >= rem) {
+            const unsigned nrem = rem - below;
+            sm.prefix = prefix | ((unsigned long long)(lane * 8 + j) << shift);
+            sm.mask = mask | (0xffull << shift);
+            sm.rem = (int)nrem;
+            sm.done = (cnt[j] == nrem) ? 1 : 0;
+            break;
+          }
+          below += cnt[j];
+        }
+      }
+    }
+    __syncthreads();
+    if (sm.done) break;
+  }
+  SelectResult r{sm.prefix, sm.mask};
+  __syncthreads();
+  return r;
+}
+
 __device__ __forceinline__ bool is_selected(unsigned long long key, const SelectResult& r) {
   return key != kNoKey && (key & r.mask) <= r.prefix;
 }

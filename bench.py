@@ -94,6 +94,22 @@ def attn_traffic(w):
         return None
 
 
+def max_over_ranks(ms: float, device) -> float:
+    """The slowest rank's time (every rank gets the same answer); the identity on one process."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return ms
+    t = torch.tensor([ms], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world: int, batch: int, steps: int, ms: float) -> float:
+    """Tokens per second of the whole job: every rank decodes `batch` sequences for `steps` steps."""
+    return world * batch * steps / (ms / 1e3)
+
+
 def roofline_table(bytes_per_kernel, ms_per_kernel, peak):
     """Per kernel: time, algorithmic bytes, achieved GB/s and the fraction of the HBM peak."""
     out = {}
@@ -335,12 +351,9 @@ def main():
     prof = h.profile_read(reset=True)
     h.profile(False)
     sb = h.query()
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, dev)
     K = args.steps
-    value = world * B * K / (elapsed_ms / 1e3)
+    value = whole_job_rate(world, B, K, elapsed_ms)
 
     # ---- roofline of the dominant kernel (attention) ----
     n8 = sb["attn_tokens_int8"] - sa["attn_tokens_int8"]
@@ -436,11 +449,8 @@ def main():
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
     _report_device_error(h, "end-to-end region")
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * B * E / (e2e_ms / 1e3)
+    e2e_ms = max_over_ranks(e2e_ms, dev)
+    e2e_value = whole_job_rate(world, B, E, e2e_ms)
 
     stats = h.query()
     full_cache = L * B * Hkv * (T + 1 + args.warmup + K + E) * 4 * D

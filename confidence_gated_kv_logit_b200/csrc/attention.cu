@@ -51,6 +51,14 @@ constexpr float kLn2 = 0.6931471805599453f;
 // 2^k for -126 <= k <= 127
 __device__ __forceinline__ float pow2i(int k) { return __int_as_float((k + 127) << 23); }
 
+// 2^x with the SFU's approximation (relative error about 2^-22; results below
+// 2^-126 flush to zero): the softmax weights and the EMA terms.
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Exponent ex with v in [2^(ex-1), 2^ex) for a normal v > 0; 0 for v = 0.
 __device__ __forceinline__ int exp_of(float v) {
   return v > 0.0f ? (int)((__float_as_uint(v) >> 23) & 0xffu) - 126 : 0;
@@ -98,42 +106,64 @@ __device__ __forceinline__ void prepare_query(const Cache& c, const AttnLaunch& 
   const int G = c.G;
   const __half* qb = a.q + ((size_t)((l - a.r.l0) * a.r.B + b) * c.Hq + (size_t)h * G) * D;
   unsigned char* out = a.qfrag + (size_t)s * a.qf_stride;
-  float scl[GP];
-#pragma unroll
-  for (int hh = 0; hh < GP; ++hh) {
-    float mx = 0.0f;
-    if (hh < G) {
-#pragma unroll
-      for (int e = 0; e < D / 32; ++e) mx = fmaxf(mx, fabsf(__half2float(qb[(size_t)hh * D + lane * (D / 32) + e])));
-    }
-    mx = warp_max(mx);
-    const int ex = exp_of(mx);
-    scl[hh] = mx > 0.0f ? pow2i(27 - ex) : 1.0f;
-    if (lane == 0) reinterpret_cast<float*>(out + Q::CQ_OFF)[hh] = mx > 0.0f ? qscale * pow2i(ex - 27) : 0.0f;
-  }
   const int g = lane >> 2, t = lane & 3;
-  // column g of n-block nb = 2*hs + p2 is head g/2 + 4*hs, digit plane 2*p2 + g%2
+  // Every load is issued first. Lane (g, t) holds, for head g/2 + 4*hs, the
+  // 8 dims kb*32 + half*16 + 4t .. +3 of every k-block (32 values), which are
+  // also what its digit planes need; the eight lanes of one head (t and g&1)
+  // cover all D dims, so three shuffles give the head's max |q|.
+  uint2 w[GP / 4][Q::KB][2];
 #pragma unroll
-  for (int kb = 0; kb < Q::KB; ++kb) {
+  for (int hs = 0; hs < GP / 4; ++hs) {
+    const int hh = g / 2 + 4 * hs;
 #pragma unroll
-    for (int hs = 0; hs < GP / 4; ++hs) {
-      const int hh = g / 2 + 4 * hs;
-      const float sc = sel(scl, hh);
+    for (int kb = 0; kb < Q::KB; ++kb)
+#pragma unroll
+      for (int half = 0; half < 2; ++half)
+        w[hs][kb][half] = hh < G ? *reinterpret_cast<const uint2*>(qb + (size_t)hh * D + kb * 32 + half * 16 + 4 * t)
+                                 : make_uint2(0u, 0u);
+  }
+  uint32_t hq[Q::KS][2];
+#pragma unroll
+  for (int ks = 0; ks < Q::KS; ++ks) {
+    hq[ks][0] = g < G ? *reinterpret_cast<const uint32_t*>(qb + (size_t)g * D + ks * 16 + 2 * t) : 0u;
+    hq[ks][1] = g < G ? *reinterpret_cast<const uint32_t*>(qb + (size_t)g * D + ks * 16 + 8 + 2 * t) : 0u;
+  }
+#pragma unroll
+  for (int ks = 0; ks < Q::KS; ++ks)
+    reinterpret_cast<uint2*>(out + Q::H_OFF)[ks * 32 + lane] = make_uint2(hq[ks][0], hq[ks][1]);
+
+#pragma unroll
+  for (int hs = 0; hs < GP / 4; ++hs) {
+    const int hh = g / 2 + 4 * hs;
+    float mx = 0.0f;
+#pragma unroll
+    for (int kb = 0; kb < Q::KB; ++kb)
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const float2 f01 = h2_to_f2(w[hs][kb][half].x), f23 = h2_to_f2(w[hs][kb][half].y);
+        mx = fmaxf(fmaxf(mx, fmaxf(fabsf(f01.x), fabsf(f01.y))), fmaxf(fabsf(f23.x), fabsf(f23.y)));
+      }
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+    const int ex = exp_of(mx);
+    const float sc = mx > 0.0f ? pow2i(27 - ex) : 1.0f;
+    if ((lane & 7) == 0) reinterpret_cast<float*>(out + Q::CQ_OFF)[hh] = mx > 0.0f ? qscale * pow2i(ex - 27) : 0.0f;
+    // column g of n-block nb = 2*hs + p2 is head g/2 + 4*hs, digit plane 2*p2 + g%2
+#pragma unroll
+    for (int kb = 0; kb < Q::KB; ++kb) {
       uint32_t r[2][2] = {{0u, 0u}, {0u, 0u}};   // [p2][half]
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
-        if (hh < G) {
-          const uint2 w = *reinterpret_cast<const uint2*>(qb + (size_t)hh * D + kb * 32 + half * 16 + 4 * t);
-          const float2 f01 = h2_to_f2(w.x), f23 = h2_to_f2(w.y);
-          const float qv[4] = {f01.x, f01.y, f23.x, f23.y};
+        const float2 f01 = h2_to_f2(w[hs][kb][half].x), f23 = h2_to_f2(w[hs][kb][half].y);
+        const float qv[4] = {f01.x, f01.y, f23.x, f23.y};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            int d[4];
-            q_digits(__float2int_rn(qv[e] * sc), d);
-            const int lo = (g & 1) ? d[1] : d[0], hi = (g & 1) ? d[3] : d[2];
-            r[0][half] |= (uint32_t)(lo & 0xff) << (8 * e);
-            r[1][half] |= (uint32_t)(hi & 0xff) << (8 * e);
-          }
+        for (int e = 0; e < 4; ++e) {
+          int d[4];
+          q_digits(__float2int_rn(qv[e] * sc), d);
+          const int lo = (g & 1) ? d[1] : d[0], hi = (g & 1) ? d[3] : d[2];
+          r[0][half] |= (uint32_t)(lo & 0xff) << (8 * e);
+          r[1][half] |= (uint32_t)(hi & 0xff) << (8 * e);
         }
       }
 #pragma unroll
@@ -141,15 +171,6 @@ __device__ __forceinline__ void prepare_query(const Cache& c, const AttnLaunch& 
         reinterpret_cast<uint2*>(out + Q::I8_OFF)[(kb * Q::NB + 2 * hs + p2) * 32 + lane] =
             make_uint2(r[p2][0], r[p2][1]);
     }
-  }
-#pragma unroll
-  for (int ks = 0; ks < Q::KS; ++ks) {
-    uint32_t r0 = 0, r1 = 0;
-    if (g < G) {
-      r0 = *reinterpret_cast<const uint32_t*>(qb + (size_t)g * D + ks * 16 + 2 * t);
-      r1 = *reinterpret_cast<const uint32_t*>(qb + (size_t)g * D + ks * 16 + 8 + 2 * t);
-    }
-    reinterpret_cast<uint2*>(out + Q::H_OFF)[ks * 32 + lane] = make_uint2(r0, r1);
   }
 }
 
@@ -167,6 +188,7 @@ __global__ void __launch_bounds__(256) append_kernel(Cache c, AttnLaunch a, int 
   if (warp >= r.items(c.Hkv)) return;
   int l, b, h;
   const int s = seg_of(c, r, warp, &l, &b, &h);
+  prepare_query<D, GP>(c, a, s, l, b, h, lane, qscale);   // independent of the cache state: first
   const int t = c.next_pos[s];
   if (!guard(t >= 0 && c.n_cold[s] >= 0 && c.n_cold[s] <= c.cap, c.err, kSiteAppendSeg, s, t)) return;
   const size_t in_row = ((size_t)((l - r.l0) * r.B + b) * c.Hkv + h);
@@ -220,7 +242,6 @@ __global__ void __launch_bounds__(256) append_kernel(Cache c, AttnLaunch a, int 
     }
   }
   if (lane == 0) c.next_pos[s] = t + 1;
-  prepare_query<D, GP>(c, a, s, l, b, h, lane, qscale);
 }
 
 // ---------------------------------------------------------------------------
@@ -319,7 +340,7 @@ __device__ __forceinline__ void update_max(SoftmaxState<D, GP>& st, const float*
     const int g = lane >> 2, t = lane & 3;
     float corr[GP];
 #pragma unroll
-    for (int h = 0; h < GP; ++h) corr[h] = mn[h] > st.m[h] ? exp2f(st.m[h] - mn[h]) : 1.0f;
+    for (int h = 0; h < GP; ++h) corr[h] = mn[h] > st.m[h] ? ex2(st.m[h] - mn[h]) : 1.0f;
     const float ca = sel(corr, GP == 4 ? (g & 3) : g);
 #pragma unroll
     for (int mb = 0; mb < GP / 4; ++mb)
@@ -437,12 +458,13 @@ __device__ __forceinline__ bool consume_i8(const Cache& c, const AttnLaunch& a, 
         const float sg = S * (ksr * cq8[j]);
         const int head = t + 4 * j;
         const bool valid = in && head < G;
+        const float ul = sg * kLog2e;
         if (valid) {
           const int col = x.j0 + r;
           if (!kChecked || guard(col < a.score_stride, c.err, kSiteAttnScore, 0, col))
-            x.sc_base[(size_t)head * a.score_stride + col] = sg;
+            x.sc_base[(size_t)head * a.score_stride + col] = ul;   // scores are kept in log2 units
         }
-        u[mb2][hr][j] = valid ? sg * kLog2e : -CUDART_INF_F;
+        u[mb2][hr][j] = valid ? ul : -CUDART_INF_F;
       }
     }
   }
@@ -477,7 +499,7 @@ __device__ __forceinline__ bool consume_i8(const Cache& c, const AttnLaunch& a, 
       for (int hr = 0; hr < 2; ++hr) {
         const int rl = mb2 * 16 + g + 8 * hr;
         const float uu = u[mb2][hr][j];
-        const float p = uu == -CUDART_INF_F ? 0.0f : exp2f(uu - mh);
+        const float p = uu == -CUDART_INF_F ? 0.0f : ex2(uu - mh);
         st.lp8[j] += p;
         x.ps[head * kPstr + rl] = p == 0.0f ? 0.0f : p * vsc[warp * 32 + rl];
       }
@@ -591,13 +613,13 @@ __device__ __forceinline__ bool consume_h(const Cache& c, const AttnLaunch& a, c
     for (int cc = 0; cc < 2; ++cc) {
       const int head = 2 * t + cc;
       const bool valid = tv && head < G;
-      const float sg = f[2 * hr + cc] * qscale;
+      const float ul = f[2 * hr + cc] * qscale * kLog2e;
       if (valid) {
         const int col = (RING ? c.cap : 0) + x.j0 + r;
         if (!kChecked || guard(col < a.score_stride, c.err, kSiteAttnScore, 1, col))
-          x.sc_base[(size_t)head * a.score_stride + col] = sg;
+          x.sc_base[(size_t)head * a.score_stride + col] = ul;   // scores are kept in log2 units
       }
-      u[hr][cc] = valid ? sg * kLog2e : -CUDART_INF_F;
+      u[hr][cc] = valid ? ul : -CUDART_INF_F;
     }
   }
 #pragma unroll
@@ -619,7 +641,7 @@ __device__ __forceinline__ bool consume_h(const Cache& c, const AttnLaunch& a, c
 #pragma unroll
       for (int hr = 0; hr < 2; ++hr) {
         const float uu = u[hr][cc];
-        const float p = uu == -CUDART_INF_F ? 0.0f : exp2f(uu - mh);
+        const float p = uu == -CUDART_INF_F ? 0.0f : ex2(uu - mh);
         st.lp16[cc] += p;
         x.ps[head * kPstr + g + 8 * hr] = p;
       }
@@ -1005,11 +1027,11 @@ __device__ __forceinline__ float4 ema_update4(const float* __restrict__ sb, int 
   float sum[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
   for (int g = 0; g < G; ++g) {
-    const float4 v = *reinterpret_cast<const float4*>(sb + (size_t)g * stride + col);
-    sum[0] += __expf(v.x - lse[g]);
-    sum[1] += __expf(v.y - lse[g]);
-    sum[2] += __expf(v.z - lse[g]);
-    sum[3] += __expf(v.w - lse[g]);
+    const float4 v = *reinterpret_cast<const float4*>(sb + (size_t)g * stride + col);   // log2 units
+    sum[0] += ex2(v.x - lse[g]);
+    sum[1] += ex2(v.y - lse[g]);
+    sum[2] += ex2(v.z - lse[g]);
+    sum[3] += ex2(v.w - lse[g]);
   }
   const float invG = 1.0f / G;
   e.x = fmaf(pol.beta, e.x, pol.one_minus_beta * (sum[0] * invG));
@@ -1031,7 +1053,7 @@ __global__ void __launch_bounds__(256) ema_kernel(Cache c, AttnLaunch a, Policy 
   const int s = seg_of(c, a.r, item, &l, &b, &h);
   float lse[G];
 #pragma unroll
-  for (int g = 0; g < G; ++g) lse[g] = a.lse_ws[(size_t)s * G + g];
+  for (int g = 0; g < G; ++g) lse[g] = a.lse_ws[(size_t)s * G + g] * kLog2e;   // log2 units, like the scores
   const int n_cold = c.n_cold[s];
   const int t = c.next_pos[s] - 1;
   if (!(n_cold >= 0 && n_cold <= c.cap)) {

@@ -136,6 +136,23 @@ __device__ bool evict_segment_warp(const Cache& c, const Policy& pol, const Evic
     if (t - pos < pol.P || pos < pol.n_sink) return kNoKey;
     return rank_key(pol, sc, pos, t);
   };
+  // Everything the conversion of the window's leaving token needs is loaded
+  // now, in parallel with the candidate record (it does not depend on the
+  // victims, except that the token may itself be one: checked below).
+  const int leaving = t + 1 - W;
+  const bool may_req = CI8 && W > 0 && leaving >= 0;
+  const int rq_slot = may_req ? (t + 1) % W : 0;
+  int rq_pos = -1;
+  float rq_sc = 0.0f;
+  uint32_t rq_k[D / 64], rq_v[D / 64];
+  if (may_req) {
+    rq_pos = pos_r[rq_slot];
+    rq_sc = sc_r[rq_slot];
+    row_load_h<D>(c.kr + (size_t)s * c.Wst * D, rq_slot, lane, rq_k);
+    row_load_h<D>(c.vr + (size_t)s * c.Wst * D, rq_slot, lane, rq_v);
+  }
+  bool leaving_evicted = false;
+
   // This step's EMA pass may have left the segment's smallest keys and its
   // window slot count (confidence mode): then nothing needs rescanning.
   EvictCand* cd = a.cand != nullptr ? a.cand + s : nullptr;
@@ -223,6 +240,7 @@ __device__ bool evict_segment_warp(const Cache& c, const Policy& pol, const Evic
 
     const bool is_v = my_victim >= 0;
     if (is_v && my_victim >= n_cold) pos_r[my_victim - n_cold] = -1;   // window victims free their slot
+    leaving_evicted = __any_sync(0xffffffffu, may_req && is_v && my_victim == n_cold + rq_slot);
     const bool cold_v = is_v && my_victim < n_cold;
     const int ec = __popc(__ballot_sync(0xffffffffu, cold_v));
     if (ec > 0) {
@@ -265,26 +283,27 @@ __device__ bool evict_segment_warp(const Cache& c, const Policy& pol, const Evic
 
   // the token that the next append would push out of the window becomes INT8
   int requant = 0;
-  const int leaving = t + 1 - W;
-  if (CI8 && W > 0 && leaving >= 0) {
-    const int slot = (t + 1) % W;
-    const size_t rs = (size_t)s * c.Wst + slot;
-    if (c.pos_r[rs] == leaving) {
-      const int idx = n_cold_new;
-      if (idx >= c.cap || idx < 0) {
-        if (lane == 0) record_violation(c.err, kSiteEvictRequant, s, idx);
-      } else {
-        const size_t cs = (size_t)s * c.cap + idx;
-        warp_requant<D>(c, s, slot, idx, lane);
-        __syncwarp();
-        if (lane == 0) {
-          c.pos_c[cs] = leaving;
-          c.sc_c[cs] = c.sc_r[rs];
-          c.pos_r[rs] = -1;
-        }
-        n_cold_new = idx + 1;
-        requant = 1;
+  if (may_req && rq_pos == leaving && !leaving_evicted) {
+    const size_t rs = (size_t)s * c.Wst + rq_slot;
+    const int idx = n_cold_new;
+    if (idx >= c.cap || idx < 0) {
+      if (lane == 0) record_violation(c.err, kSiteEvictRequant, s, idx);
+    } else {
+      const size_t cb = (size_t)s * c.cap * D, cs = (size_t)s * c.cap + idx;
+      uint32_t pk;
+      const float ksc = row_quantize<D>(rq_k, &pk);
+      row_store_k8<D>(c.k8 + cb, idx, lane, pk);
+      const float vsc = row_quantize<D>(rq_v, &pk);
+      row_store_v8<D>(c.v8 + cb, idx, lane, pk);
+      if (lane == 0) {
+        c.ks[cs] = ksc;
+        c.vs[cs] = vsc;
+        c.pos_c[cs] = leaving;
+        c.sc_c[cs] = rq_sc;
+        c.pos_r[rs] = -1;
       }
+      n_cold_new = idx + 1;
+      requant = 1;
     }
   }
   if (lane == 0) c.n_cold[s] = n_cold_new;

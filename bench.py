@@ -94,6 +94,28 @@ def attn_traffic(w):
         return None
 
 
+def warm_library(w, dev):
+    """One small step through every entry point on a throwaway handle, so that
+    the first timed calls (the bulk first step among them) measure the work,
+    not the loading of the library's kernels."""
+    import torch
+    from confidence_gated_kv_logit_b200 import ConfKV, synth
+    from confidence_gated_kv_logit_b200.binding import ALL_LAYERS
+    h = ConfKV(2, w["Hkv"], w["Hq"], w["D"], max_batch=2, max_prefill=600, n_low=64, n_high=128,
+               protect_last=16, fp16_window=32)
+    g = synth.generator(7, dev)
+    k, v = synth.prefill_kv(2, w["Hkv"], 600, w["D"], g, dev)
+    for l in range(2):
+        h.prefill(k, v, [600, 500], layer=l)
+    q, kn, vn = synth.step_qkv((2, 2), w["Hq"], w["Hkv"], w["D"], g, dev)
+    out = torch.empty((2, 2, w["Hq"], w["D"]), device=dev)
+    h.decode_attn(q, kn, vn, out, ALL_LAYERS)
+    h.confidence(synth.bursty_logits(2, 4096, g, dev), torch.empty(2, device=dev))
+    h.evict_compact(ALL_LAYERS)
+    torch.cuda.synchronize()
+    h.close()
+
+
 def max_over_ranks(ms: float, device) -> float:
     """The slowest rank's time (every rank gets the same answer); the identity on one process."""
     import torch
@@ -287,6 +309,7 @@ def main():
     w = workload(args)
     L, Hq, Hkv, D, B, T, V = (w[k] for k in ("L", "Hq", "Hkv", "D", "B", "T", "V"))
     G = Hq // Hkv
+    warm_library(w, dev)
     h = ConfKV(L, Hkv, Hq, D, max_batch=B, max_prefill=T, n_low=w["n_low"], n_high=w["n_high"], tau=w["tau"],
                alpha=w["alpha"], ema_decay=w["beta"], protect_last=w["P"], fp16_window=w["W"])
     gen = synth.generator(1000 + rank, dev)
@@ -397,9 +420,11 @@ def main():
     for i in range(8):
         q, kn, vn, lg = pool[i]
         hpool.append(tuple(x.cpu().pin_memory() for x in (q, kn, vn, lg)))
-    # Two buffer sets: the copies of step i+1's inputs and of step i-1's
-    # results run on a copy stream while step i computes.
-    copy_s = torch.cuda.Stream(device=dev)
+    # Two buffer sets: step i+1's inputs upload on one copy stream and step
+    # i-1's results download on another (the two directions use separate
+    # copy engines) while step i computes.
+    up_s = torch.cuda.Stream(device=dev)
+    down_s = torch.cuda.Stream(device=dev)
     dbuf = [tuple(torch.empty_like(x) for x in pool[0]) for _ in range(2)]
     obuf = [torch.empty((L, B, Hq, D), device=dev) for _ in range(2)]
     cbuf = [torch.empty(B, device=dev) for _ in range(2)]
@@ -417,15 +442,16 @@ def main():
 
     def upload(i):
         j = i % 2
-        with torch.cuda.stream(copy_s):
+        with torch.cuda.stream(up_s):
             if i >= 2:
-                copy_s.wait_event(ev_comp[j])          # step i-2 is done with buffer set j
+                up_s.wait_event(ev_comp[j])            # step i-2 is done with buffer set j
             for dst, src in zip(dbuf[j], hpool[i % len(hpool)]):
                 dst.copy_(src, non_blocking=True)
-            ev_in[j].record(copy_s)
+            ev_in[j].record(up_s)
 
     e0.record(stream)
-    copy_s.wait_stream(stream)
+    up_s.wait_stream(stream)
+    down_s.wait_stream(stream)
     upload(0)
     for i in range(E):
         j = i % 2
@@ -439,12 +465,13 @@ def main():
         h.confidence(dl, cbuf[j])
         h.evict_compact(ALL_LAYERS)
         ev_comp[j].record(stream)
-        with torch.cuda.stream(copy_s):
-            copy_s.wait_event(ev_comp[j])
+        with torch.cuda.stream(down_s):
+            down_s.wait_event(ev_comp[j])
             host_out[j].copy_(obuf[j], non_blocking=True)
             host_c[j].copy_(cbuf[j], non_blocking=True)
-            ev_out[j].record(copy_s)
-    stream.wait_stream(copy_s)
+            ev_out[j].record(down_s)
+    stream.wait_stream(up_s)
+    stream.wait_stream(down_s)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
@@ -476,7 +503,7 @@ def main():
                          "ms_per_launch": attn_ms},
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "tok/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "pipelining": "two buffer sets; step i+1's inputs and step i-1's results copy on a second stream",
+                    "pipelining": "two buffer sets; step i+1's upload and step i-1's download on two copy streams",
                     "steps": E},
             "gpu_launches": sb["kernel_launches"] - sa["kernel_launches"],
             "clocks": clocks,

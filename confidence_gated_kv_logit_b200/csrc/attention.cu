@@ -1197,10 +1197,26 @@ cudaError_t run_attn(const Cache& c, const Policy& pol, const AttnLaunch& a, cud
     ++*launches;
   }
   if (pol.mode == 0) {
-    ProfScope ps(prof, kKEma, st);
-    e = run_ema(c, pol, a, st);
-    if (e != cudaSuccess) return e;
+    // The EMA pass only feeds eviction, so it can run beside whatever the
+    // caller issues next (the confidence reduction); eviction, the next
+    // append and prefill wait for ema_done.
+    cudaStream_t es = st;
+    if (a.ema_stream != nullptr) {
+      e = cudaEventRecord(a.attn_done, st);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(a.ema_stream, a.attn_done, 0);
+      if (e != cudaSuccess) return e;
+      es = a.ema_stream;
+    }
+    {
+      ProfScope ps(prof, kKEma, es);
+      e = run_ema(c, pol, a, es);
+      if (e != cudaSuccess) return e;
+    }
     ++*launches;
+    if (a.ema_stream != nullptr) {
+      e = cudaEventRecord(a.ema_done, es);
+      if (e != cudaSuccess) return e;
+    }
   }
   return cudaGetLastError();
 }

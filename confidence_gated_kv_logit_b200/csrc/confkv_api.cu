@@ -81,6 +81,8 @@ struct confkv_handle {
   confkv::EvictCand* cand;       // [S] eviction candidates from the EMA pass
   uint32_t* kscratch;            // evict scratch, per CTA of the largest evict grid
   int* sched;                    // attention unit counters (zero between launches)
+  cudaStream_t ema_stream;       // side stream of the EMA pass
+  cudaEvent_t attn_done, ema_done;
   int scratch_stride;
   int32_t* keep_list;
   int32_t* keep_count;
@@ -331,6 +333,20 @@ confkv_status confkv_create(int32_t layers, int32_t kv_heads, int32_t q_heads, i
     delete h;
     return cuda_status(e);
   }
+  h->ema_stream = nullptr;
+  h->attn_done = h->ema_done = nullptr;
+  if (cudaStreamCreateWithFlags(&h->ema_stream, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaEventCreateWithFlags(&h->attn_done, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&h->ema_done, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventRecord(h->ema_done, h->ema_stream) != cudaSuccess) {
+    if (h->ema_stream) cudaStreamDestroy(h->ema_stream);
+    if (h->attn_done) cudaEventDestroy(h->attn_done);
+    if (h->ema_done) cudaEventDestroy(h->ema_done);
+    B.release();
+    h->magic = kDead;
+    delete h;
+    return CONFKV_ERR_CUDA;
+  }
   {
     std::lock_guard<std::mutex> lk(g_live_mu);
     g_live.insert(h);
@@ -346,6 +362,9 @@ confkv_status confkv_destroy(confkv_handle* h) {
     if (g_live.erase(h) == 0) return CONFKV_ERR_STATE;
   }
   cudaDeviceSynchronize();
+  if (h->ema_stream) cudaStreamDestroy(h->ema_stream);
+  if (h->attn_done) cudaEventDestroy(h->attn_done);
+  if (h->ema_done) cudaEventDestroy(h->ema_done);
   h->buf.release();
   h->magic = kDead;
   delete h;
@@ -385,6 +404,7 @@ confkv_status confkv_prefill(confkv_handle* h, int32_t layer, int32_t batch, con
   layer_range(h, layer, &r);
   cudaError_t e = cudaMemcpyAsync(h->lens_dev, lens_host, (size_t)batch * 4, cudaMemcpyHostToDevice, st);
   if (e != cudaSuccess) return CONFKV_ERR_CUDA;
+  if (cudaStreamWaitEvent(st, h->ema_done, 0) != cudaSuccess) return CONFKV_ERR_CUDA;
   confkv::PrefillLaunch a;
   a.r = r;
   a.lens = h->lens_dev;
@@ -465,6 +485,11 @@ confkv_status confkv_decode_attn(confkv_handle* h, int32_t layer, const void* q,
   a.qf_stride = h->qf_stride;
   a.cand = h->cand;
   a.sched = h->sched;
+  a.ema_stream = h->ema_stream;
+  a.attn_done = h->attn_done;
+  a.ema_done = h->ema_done;
+  // the previous EMA pass must be done before this step rewrites scores and EMA values
+  if (cudaStreamWaitEvent(static_cast<cudaStream_t>(stream), h->ema_done, 0) != cudaSuccess) return CONFKV_ERR_CUDA;
   cudaError_t e =
       confkv::launch_decode_attn(h->c, h->pol, a, static_cast<cudaStream_t>(stream), &h->launches, h->prof_ptr());
   if (e != cudaSuccess) return cuda_status(e);
@@ -489,6 +514,8 @@ confkv_status confkv_evict_compact(confkv_handle* h, int32_t layer, void* stream
   a.kscratch = h->kscratch;
   a.scratch_stride = h->scratch_stride;
   a.scratch_keys = h->c.cap + h->c.Wst;
+  // the candidates and EMA values come from the EMA pass on the side stream
+  if (cudaStreamWaitEvent(static_cast<cudaStream_t>(stream), h->ema_done, 0) != cudaSuccess) return CONFKV_ERR_CUDA;
   cudaError_t e =
       confkv::launch_evict_compact(h->c, h->pol, a, static_cast<cudaStream_t>(stream), &h->launches, h->prof_ptr());
   if (e != cudaSuccess) return cuda_status(e);

@@ -342,17 +342,35 @@ __device__ __forceinline__ void move_pairs_warp(const Cache& c, int s, const int
         if (on && c0 + u < CH) store_part<D, CI8>(c, s, dst, c0 + u, v[u]);
     }
     if constexpr (CI8) {
-      // V codes: dimension-major, one byte per dimension, 16 dimensions in flight
+      // V codes: dimension-major, one byte per dimension. With the placement
+      // of layout.cuh, the byte of token i, dimension d sits at
+      //   blk(i) + ((32d + r) ^ X(d)),  r = i % 32, X(d) = ((d >> 2) & 7) << 4,
+      // which splits into a compile-time part (32d) ^ (X & 0x60) and one of
+      // two per-token bases (r or r ^ 16): every access below is a single
+      // load or store at an immediate offset.
       const unsigned char* vsrc = reinterpret_cast<const unsigned char*>(c.v8 + base);
       unsigned char* vdst = reinterpret_cast<unsigned char*>(c.v8 + base);
-#pragma unroll 1
+      const unsigned char* sb0 = vsrc + (size_t)(src >> 5) * 32 * D + (src & 31);
+      const unsigned char* sb1 = vsrc + (size_t)(src >> 5) * 32 * D + ((src & 31) ^ 16);
+      unsigned char* db0 = vdst + (size_t)(dst >> 5) * 32 * D + (dst & 31);
+      unsigned char* db1 = vdst + (size_t)(dst >> 5) * 32 * D + ((dst & 31) ^ 16);
+#pragma unroll
       for (int d0 = 0; d0 < D; d0 += 16) {
-        unsigned char b[16];
+        unsigned char bv[16];
 #pragma unroll
-        for (int u = 0; u < 16; ++u) b[u] = on ? vsrc[v8_off(src, d0 + u, D)] : 0;
+        for (int u = 0; u < 16; ++u) {
+          const int d = d0 + u;
+          const int X = ((d >> 2) & 7) << 4;
+          const int off = (32 * d) ^ (X & 0x60);
+          bv[u] = on ? ((X & 0x10) ? sb1 : sb0)[off] : 0;
+        }
 #pragma unroll
-        for (int u = 0; u < 16; ++u)
-          if (on) vdst[v8_off(dst, d0 + u, D)] = b[u];
+        for (int u = 0; u < 16; ++u) {
+          const int d = d0 + u;
+          const int X = ((d >> 2) & 7) << 4;
+          const int off = (32 * d) ^ (X & 0x60);
+          if (on) ((X & 0x10) ? db1 : db0)[off] = bv[u];
+        }
       }
     }
     if (on) {

@@ -65,6 +65,9 @@ struct AttnLaunch {
   int qf_stride;
   EvictCand* cand;        // [S] eviction candidates written by the EMA pass (confidence mode)
   int* sched;             // [2] unit counter and finished-CTA counter of the attention kernel (zero between launches)
+  cudaStream_t ema_stream;  // when set, the EMA pass runs there (forked after attention, joined on ema_done)
+  cudaEvent_t attn_done;    // recorded on the caller's stream after attention
+  cudaEvent_t ema_done;     // recorded on ema_stream after the EMA pass
 };
 cudaError_t launch_decode_attn(const Cache& c, const Policy& pol, const AttnLaunch& a, cudaStream_t st,
                                long long* launches, Prof* prof);

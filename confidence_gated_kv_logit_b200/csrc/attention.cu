@@ -1073,25 +1073,37 @@ __global__ void __launch_bounds__(256) ema_kernel(Cache c, AttnLaunch a, Policy 
     best.offer(rank_key(pol, ema, pos, t), idx);
     if (use_bound) best.update_bound(t1_over_oma);
   };
-  // cold region [0, n_cold): the region and the score rows are multiples of 64 long
+  // cold region [0, n_cold): the region and the score rows are multiples of 64
+  // long. A group of four whose smallest position is past the lane's bound
+  // offers nothing (one test for the group: the common case once the lane's
+  // list is full).
   for (int base = 0; base < n_cold; base += 256) {
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
       const int i0 = base + 128 * u + 4 * lane;
-      if (i0 < n_cold) {
+      if (i0 + 3 < n_cold) {
         const float4 e = ema_update4<G>(sb, a.score_stride, i0, *reinterpret_cast<const float4*>(scc + i0), lse, pol);
         const int4 p4 = *reinterpret_cast<const int4*>(pc + i0);
-        if (i0 + 3 < n_cold) {
-          *reinterpret_cast<float4*>(scc + i0) = e;
-        } else {
-          scc[i0] = e.x;
-          if (i0 + 1 < n_cold) scc[i0 + 1] = e.y;
-          if (i0 + 2 < n_cold) scc[i0 + 2] = e.z;
+        *reinterpret_cast<float4*>(scc + i0) = e;
+        if (min(min(p4.x, p4.y), min(p4.z, p4.w)) + 1 <= best.pos_bound) {
+          offer(p4.x, e.x, i0);
+          offer(p4.y, e.y, i0 + 1);
+          offer(p4.z, e.z, i0 + 2);
+          offer(p4.w, e.w, i0 + 3);
         }
+      } else if (i0 < n_cold) {   // the last, partial group
+        const float4 e = ema_update4<G>(sb, a.score_stride, i0, *reinterpret_cast<const float4*>(scc + i0), lse, pol);
+        const int4 p4 = *reinterpret_cast<const int4*>(pc + i0);
+        scc[i0] = e.x;
         offer(p4.x, e.x, i0);
-        if (i0 + 1 < n_cold) offer(p4.y, e.y, i0 + 1);
-        if (i0 + 2 < n_cold) offer(p4.z, e.z, i0 + 2);
-        if (i0 + 3 < n_cold) offer(p4.w, e.w, i0 + 3);
+        if (i0 + 1 < n_cold) {
+          scc[i0 + 1] = e.y;
+          offer(p4.y, e.y, i0 + 1);
+        }
+        if (i0 + 2 < n_cold) {
+          scc[i0 + 2] = e.z;
+          offer(p4.z, e.z, i0 + 2);
+        }
       }
     }
   }

@@ -335,7 +335,13 @@ confkv_status confkv_create(int32_t layers, int32_t kv_heads, int32_t q_heads, i
   }
   h->ema_stream = nullptr;
   h->attn_done = h->ema_done = nullptr;
-  if (cudaStreamCreateWithFlags(&h->ema_stream, cudaStreamNonBlocking) != cudaSuccess ||
+  // The EMA pass gets the device's highest stream priority: it and the
+  // caller's next kernel (the confidence reduction) become ready together
+  // when attention ends, and the EMA's long-segment warps should start first,
+  // with the other kernel filling the SM slots its short segments free.
+  int prio_least = 0, prio_greatest = 0;
+  if (cudaDeviceGetStreamPriorityRange(&prio_least, &prio_greatest) != cudaSuccess) prio_greatest = 0;
+  if (cudaStreamCreateWithPriority(&h->ema_stream, cudaStreamNonBlocking, prio_greatest) != cudaSuccess ||
       cudaEventCreateWithFlags(&h->attn_done, cudaEventDisableTiming) != cudaSuccess ||
       cudaEventCreateWithFlags(&h->ema_done, cudaEventDisableTiming) != cudaSuccess ||
       cudaEventRecord(h->ema_done, h->ema_stream) != cudaSuccess) {

@@ -155,19 +155,29 @@ __device__ bool evict_segment_warp(const Cache& c, const Policy& pol, const Evic
 
   // This step's EMA pass may have left the segment's smallest keys and its
   // window slot count (confidence mode): then nothing needs rescanning.
+  // The record is read whole and unconditionally (one round trip, next to the
+  // segment counters); whether it applies is decided afterwards.
   EvictCand* cd = a.cand != nullptr ? a.cand + s : nullptr;
+  int4 hdr = make_int4(0, 0, -1, -1);                 // n_ring, safe, stamp, n_cold
+  unsigned long long rec_key = kNoKey;
+  int rec_idx = -1;
+  if (cd != nullptr) {
+    hdr = *reinterpret_cast<const int4*>(&cd->n_ring);
+    if (lane < kCandMax) {
+      rec_key = cd->key[lane];
+      rec_idx = cd->idx[lane];
+    }
+  }
   bool have = false;
   int n_ring = 0, count = 0, safe = 0;
   unsigned long long my_key = kNoKey;
   int my_idx = -1;
-  if (cd != nullptr && pol.mode == 0 && !a.stable && cd->stamp == t + 1 && cd->n_cold == n_cold) {
+  if (cd != nullptr && pol.mode == 0 && !a.stable && hdr.z == t + 1 && hdr.w == n_cold) {
     have = true;
-    n_ring = cd->n_ring;
-    safe = cd->safe;
-    if (lane < kCandMax) {
-      my_key = cd->key[lane];
-      my_idx = cd->idx[lane];
-    }
+    n_ring = hdr.x;
+    safe = hdr.y;
+    my_key = rec_key;
+    my_idx = rec_idx;
     count = __popc(__ballot_sync(0xffffffffu, lane < kCandMax && my_key != kNoKey));
   }
   // Otherwise one pass over the segment counts the occupied window slots and

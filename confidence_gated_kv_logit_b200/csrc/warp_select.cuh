@@ -3,6 +3,8 @@
 // after updating the EMA values and hands the smallest ones to eviction).
 #pragma once
 
+#include <stddef.h>
+
 #include "common.cuh"
 
 namespace confkv {
@@ -12,13 +14,13 @@ constexpr int kWarpMaxVictims = kCandMax;
 constexpr int kLaneKeep = 4;              // smallest keys each lane keeps during the scan
 
 
+// Minimum over the warp of a 64-bit key: the smallest high half, then the
+// smallest low half among the lanes that hold it (two warp reductions).
 __device__ __forceinline__ unsigned long long warp_min_u64(unsigned long long v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const unsigned long long w = __shfl_xor_sync(0xffffffffu, v, o);
-    v = w < v ? w : v;
-  }
-  return v;
+  const unsigned hi = (unsigned)(v >> 32);
+  const unsigned mh = __reduce_min_sync(0xffffffffu, hi);
+  const unsigned ml = __reduce_min_sync(0xffffffffu, hi == mh ? (unsigned)v : 0xffffffffu);
+  return ((unsigned long long)mh << 32) | ml;
 }
 
 // Keeps the kLaneKeep smallest (key, index) pairs seen by this lane, ascending.
@@ -88,9 +90,10 @@ struct LaneBest {
 struct EvictCand {
   unsigned long long key[kCandMax];
   int idx[kCandMax];
-  int n_ring, safe, stamp, n_cold;
+  int n_ring, safe, stamp, n_cold;   // read as one 16-byte word
 };
 static_assert(sizeof(EvictCand) == 208, "candidate record layout");
+static_assert(offsetof(EvictCand, n_ring) % 16 == 0, "the record header is one aligned 16-byte word");
 
 // Merge every lane's list into the segment's smallest keys: lane j < count
 // receives the j-th smallest key and its index. Also returns (in every lane)

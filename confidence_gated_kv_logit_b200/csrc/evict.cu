@@ -339,17 +339,38 @@ __device__ __forceinline__ void move_pairs_warp(const Cache& c, int s, const int
     if (kChecked && on && !guard(dst >= 0 && dst < n_keep && src >= n_keep && src < n_cold, c.err, kSiteEvictPair,
                                  s, src))
       continue;
-    // K (or fp16 K and V) rows: 16-byte chunks, four in flight
+    // K (or fp16 K and V) rows as 16-byte chunks, with the row's metadata:
+    // every load of the round in flight before any store
     constexpr int CH = CI8 ? R::KP : R::NP;   // fp16 rows move K and V by chunks
+    constexpr int RND = CH < 4 ? CH : 4;
+    const size_t so = (size_t)s * c.cap + src, dO = (size_t)s * c.cap + dst;
+    int pv = 0;
+    float sv = 0.0f, kv = 0.0f, vv = 0.0f;
+    if (on) {
+      pv = c.pos_c[so];
+      sv = c.sc_c[so];
+      if (CI8) {
+        kv = c.ks[so];
+        vv = c.vs[so];
+      }
+    }
 #pragma unroll
-    for (int c0 = 0; c0 < CH; c0 += 4) {
-      uint4 v[4];
+    for (int c0 = 0; c0 < CH; c0 += RND) {
+      uint4 v[RND];
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
+      for (int u = 0; u < RND; ++u)
         if (on && c0 + u < CH) v[u] = load_part<D, CI8>(c, s, src, c0 + u);
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
+      for (int u = 0; u < RND; ++u)
         if (on && c0 + u < CH) store_part<D, CI8>(c, s, dst, c0 + u, v[u]);
+    }
+    if (on) {
+      c.pos_c[dO] = pv;
+      c.sc_c[dO] = sv;
+      if (CI8) {
+        c.ks[dO] = kv;
+        c.vs[dO] = vv;
+      }
     }
     if constexpr (CI8) {
       // V codes: dimension-major, one byte per dimension. With the placement
@@ -365,38 +386,22 @@ __device__ __forceinline__ void move_pairs_warp(const Cache& c, int s, const int
       unsigned char* db0 = vdst + (size_t)(dst >> 5) * 32 * D + (dst & 31);
       unsigned char* db1 = vdst + (size_t)(dst >> 5) * 32 * D + ((dst & 31) ^ 16);
 #pragma unroll
-      for (int d0 = 0; d0 < D; d0 += 16) {
-        unsigned char bv[16];
+      for (int d0 = 0; d0 < D; d0 += 32) {
+        unsigned char bv[32];
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
+        for (int u = 0; u < 32; ++u) {
           const int d = d0 + u;
           const int X = ((d >> 2) & 7) << 4;
           const int off = (32 * d) ^ (X & 0x60);
           bv[u] = on ? ((X & 0x10) ? sb1 : sb0)[off] : 0;
         }
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
+        for (int u = 0; u < 32; ++u) {
           const int d = d0 + u;
           const int X = ((d >> 2) & 7) << 4;
           const int off = (32 * d) ^ (X & 0x60);
           if (on) ((X & 0x10) ? db1 : db0)[off] = bv[u];
         }
-      }
-    }
-    if (on) {
-      const size_t so = (size_t)s * c.cap + src, dO = (size_t)s * c.cap + dst;
-      const int pv = c.pos_c[so];
-      const float sv = c.sc_c[so];
-      float kv = 0.0f, vv = 0.0f;
-      if (CI8) {
-        kv = c.ks[so];
-        vv = c.vs[so];
-      }
-      c.pos_c[dO] = pv;
-      c.sc_c[dO] = sv;
-      if (CI8) {
-        c.ks[dO] = kv;
-        c.vs[dO] = vv;
       }
     }
   }
@@ -509,14 +514,14 @@ __device__ void evict_segment_block(const Cache& c, const Policy& pol, const Evi
     }
     for (int slot = threadIdx.x; slot < W; slot += NT) khi[n_cold + slot] = hi_of(pos_r[slot], sc_r[slot]);
     __syncthreads();
-    const SelectResult sel = block_select_smallest_hi<NT>(khi, pos_of, span, e, sm);
-    const bool sel_lo = (sel.mask & 0xffffffffull) != 0;   // the low half (position) decides ties
-    auto is_victim = [&](int i) -> bool {
-      const uint32_t hv = khi[i];
-      if (hv == 0xFFFFFFFFu) return false;
-      const unsigned long long k64 = ((unsigned long long)hv << 32) | (sel_lo ? (uint32_t)pos_of(i) : 0u);
-      return is_selected(k64, sel);
+    // the e-th smallest key: the victims are the keys up to it
+    const unsigned long long thr =
+        block_select_threshold<NT>(khi, pos_of, span, e, sm, reinterpret_cast<unsigned long long*>(es.stage));
+    const uint32_t thr_hi = (uint32_t)(thr >> 32), thr_lo = (uint32_t)thr;
+    auto below_thr = [&](uint32_t hv, int i) -> bool {   // the position only matters on a tie of the high half
+      return hv != 0xFFFFFFFFu && (hv < thr_hi || (hv == thr_hi && (uint32_t)pos_of(i) <= thr_lo));
     };
+    auto is_victim = [&](int i) -> bool { return below_thr(khi[i], i); };
 
     // victim bitmask of the cold region: each thread builds whole 32-token
     // words from eight 16-byte loads of the key scratch
@@ -532,10 +537,7 @@ __device__ void evict_segment_block(const Cache& c, const Policy& pol, const Evi
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int i = 32 * w + 4 * u + j;
-          if (i < n_cold && hv[j] != 0xFFFFFFFFu) {
-            const unsigned long long k64 = ((unsigned long long)hv[j] << 32) | (sel_lo ? (uint32_t)pos_c[i] : 0u);
-            if (is_selected(k64, sel)) bits |= 1u << (4 * u + j);
-          }
+          if (i < n_cold && below_thr(hv[j], i)) bits |= 1u << (4 * u + j);
         }
       }
       vm[w] = bits;

@@ -324,4 +324,212 @@ __device__ __forceinline__ bool is_selected(unsigned long long key, const Select
   return key != kNoKey && (key & r.mask) <= r.prefix;
 }
 
+// Sort m (a power of two, at most 8*NT) keys of shared memory ascending with
+// a bitonic network; all NT threads call it; ends with a barrier. Each thread
+// loads two pairs of a stage before comparing either.
+template <int NT, typename K>
+__device__ __forceinline__ void block_bitonic_sort(K* buf, int m) {
+  for (int size = 2; size <= m; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i0 = (int)threadIdx.x; i0 < (m >> 1); i0 += 2 * NT) {
+        const int i1 = i0 + NT;
+        const int a0 = 2 * i0 - (i0 & (stride - 1)), a1 = 2 * i1 - (i1 & (stride - 1));
+        const bool two = i1 < (m >> 1);
+        const K x0 = buf[a0], y0 = buf[a0 + stride];
+        K x1 = x0, y1 = y0;
+        if (two) {
+          x1 = buf[a1];
+          y1 = buf[a1 + stride];
+        }
+        if ((x0 > y0) == ((a0 & size) == 0)) {
+          buf[a0] = y0;
+          buf[a0 + stride] = x0;
+        }
+        if (two && (x1 > y1) == ((a1 & size) == 0)) {
+          buf[a1] = y1;
+          buf[a1 + stride] = x1;
+        }
+      }
+      __syncthreads();
+    }
+  }
+}
+
+constexpr int kSelBuf = 2048;   // 64-bit entries of the shared buffer block_select_threshold uses
+constexpr int kSelBins = 2048;  // histogram bins (the first half of the buffer, as 32-bit counts)
+constexpr int kSelCand = (kSelBuf * 8 - kSelBins * 4) / 8;   // keys of one bin the rest of the buffer holds
+
+// The k-th smallest (1-based) of the n 64-bit keys (hi[i] << 32) | lo(i),
+// where hi[i] == 0xFFFFFFFF marks an entry that is never counted (k must not
+// exceed the counted entries): every counted key <= the result is one of the
+// k smallest. hi must be 16-byte aligned and readable up to n rounded up to
+// 4. Up to kSelBuf keys are sorted outright. Otherwise three passes over the
+// high halves: their range; a histogram of kSelBins bins, monotone in the
+// key, which locates the bin holding the k-th key; the keys of that bin,
+// which are sorted. When that bin is too full for the buffer, the radix
+// select above decides (its result, as a threshold, is prefix | ~mask).
+// buf: kSelBuf 64-bit entries of shared memory.
+template <int NT, typename LoFn>
+__device__ unsigned long long block_select_threshold(const uint32_t* __restrict__ hi, LoFn lo, int n, int k,
+                                                     SelectSmem<NT>& sm, unsigned long long* buf) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  if (n <= kSelBuf) {
+    int m = 1;
+    while (m < n) m <<= 1;
+    for (int i = threadIdx.x; i < m; i += NT) {
+      unsigned long long key = kNoKey;
+      if (i < n) {
+        const uint32_t hv = hi[i];
+        if (hv != 0xFFFFFFFFu) key = ((unsigned long long)hv << 32) | (uint32_t)lo(i);
+      }
+      buf[i] = key;
+    }
+    __syncthreads();
+    block_bitonic_sort<NT>(buf, m);
+    const unsigned long long r = buf[k - 1];
+    __syncthreads();
+    return r;
+  }
+  const uint4* hi4 = reinterpret_cast<const uint4*>(hi);
+  const int n4 = (n + 3) >> 2;
+  auto key_at = [&](const uint4& q, int j) { return j == 0 ? q.x : j == 1 ? q.y : j == 2 ? q.z : q.w; };
+  // pass 1: the range of the counted high halves
+  uint32_t mn = 0xFFFFFFFFu, mx = 0u;
+  for (int v0 = threadIdx.x; v0 < n4; v0 += 4 * NT) {
+    uint4 q[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) q[r] = v0 + r * NT < n4 ? hi4[v0 + r * NT] : make_uint4(~0u, ~0u, ~0u, ~0u);
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int i = 4 * (v0 + r * NT) + j;
+        const uint32_t hv = key_at(q[r], j);
+        if (i < n && hv != 0xFFFFFFFFu) {
+          mn = min(mn, hv);
+          mx = max(mx, hv);
+        }
+      }
+  }
+  mn = __reduce_min_sync(0xffffffffu, mn);
+  mx = __reduce_max_sync(0xffffffffu, mx);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(buf);
+  if (lane == 0) {
+    sm.hist[wid] = mn;
+    sm.hist[32 + wid] = mx;
+  }
+  for (int b = threadIdx.x; b < kSelBins; b += NT) hist[b] = 0u;
+  __syncthreads();
+  mn = sm.hist[0];
+  mx = sm.hist[32];
+#pragma unroll
+  for (int w = 1; w < NT / 32; ++w) {
+    mn = min(mn, sm.hist[w]);
+    mx = max(mx, sm.hist[32 + w]);
+  }
+  // bin(h) = floor((h - mn) * M / 2^32): monotone in h and below kSelBins
+  const unsigned long long range = (unsigned long long)(mx - mn) + 1ull;
+  const uint32_t M = range <= kSelBins ? 0u : (uint32_t)(((unsigned long long)kSelBins << 32) / range);
+  auto bin_of = [&](uint32_t hv) -> int {
+    const uint32_t d = hv - mn;
+    return range <= kSelBins ? (int)d : (int)__umulhi(d, M);
+  };
+  // pass 2: histogram
+  for (int v0 = threadIdx.x; v0 < n4; v0 += 4 * NT) {
+    uint4 q[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) q[r] = v0 + r * NT < n4 ? hi4[v0 + r * NT] : make_uint4(~0u, ~0u, ~0u, ~0u);
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int i = 4 * (v0 + r * NT) + j;
+        const uint32_t hv = key_at(q[r], j);
+        if (i < n && hv != 0xFFFFFFFFu) atomicAdd(&hist[bin_of(hv)], 1u);
+      }
+  }
+  __syncthreads();
+  // the bin holding the k-th key: each thread sums its kSelBins/NT bins, a
+  // block scan places them
+  constexpr int BPT = kSelBins / NT;
+  uint32_t cnt[BPT];
+  uint32_t tot = 0u;
+#pragma unroll
+  for (int j = 0; j < BPT; ++j) {
+    cnt[j] = hist[threadIdx.x * BPT + j];
+    tot += cnt[j];
+  }
+  int all;
+  const int excl = block_excl_scan_int<NT>((int)tot, sm, &all);
+  if (threadIdx.x == 0) sm.misc[2] = -1;
+  __syncthreads();
+  if (excl < k && k <= excl + (int)tot) {
+    int below = excl;
+#pragma unroll
+    for (int j = 0; j < BPT; ++j) {
+      if (below + (int)cnt[j] >= k) {
+        sm.misc[2] = threadIdx.x * BPT + j;   // the bin
+        sm.misc[3] = below;                   // counted keys in lower bins
+        sm.misc[0] = (int)cnt[j];
+        break;
+      }
+      below += (int)cnt[j];
+    }
+  }
+  __syncthreads();
+  const int bstar = sm.misc[2], nbelow = sm.misc[3], ncand = sm.misc[0];
+  if (bstar >= 0 && ncand <= kSelCand) {
+    // pass 3: the keys of that bin into the second half of the buffer
+    unsigned long long* cand = buf + kSelBins / 2;
+    __syncthreads();   // every thread has read the bin
+    if (threadIdx.x == 0) sm.misc[1] = 0;
+    __syncthreads();
+    for (int v0 = threadIdx.x; v0 < n4; v0 += 4 * NT) {
+      uint4 q[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) q[r] = v0 + r * NT < n4 ? hi4[v0 + r * NT] : make_uint4(~0u, ~0u, ~0u, ~0u);
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int i = 4 * (v0 + r * NT) + j;
+          const uint32_t hv = key_at(q[r], j);
+          if (i < n && hv != 0xFFFFFFFFu && bin_of(hv) == bstar) {
+            const int slot = atomicAdd(&sm.misc[1], 1);
+            cand[slot] = ((unsigned long long)hv << 32) | (uint32_t)i;   // index for now
+          }
+        }
+    }
+    __syncthreads();
+    // the low halves, all loads of a thread in flight together
+    for (int j0 = (int)threadIdx.x; j0 < ncand; j0 += 4 * NT) {
+      int idx[4];
+      uint32_t lov[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int j = j0 + r * NT;
+        idx[r] = j < ncand ? (int)(uint32_t)cand[j] : -1;
+      }
+#pragma unroll
+      for (int r = 0; r < 4; ++r) lov[r] = idx[r] >= 0 ? (uint32_t)lo(idx[r]) : 0u;
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int j = j0 + r * NT;
+        if (j < ncand) cand[j] = (cand[j] & 0xFFFFFFFF00000000ull) | lov[r];
+      }
+    }
+    int m = 1;
+    while (m < ncand) m <<= 1;
+    for (int i = ncand + threadIdx.x; i < m; i += NT) cand[i] = kNoKey;
+    __syncthreads();
+    block_bitonic_sort<NT>(cand, m);
+    const unsigned long long r = cand[k - nbelow - 1];
+    __syncthreads();
+    return r;
+  }
+  __syncthreads();
+  const SelectResult r = block_select_smallest_hi<NT>(hi, lo, n, k, sm);
+  return r.prefix | ~r.mask;
+}
+
 }  // namespace confkv

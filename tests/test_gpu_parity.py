@@ -36,6 +36,27 @@ def test_shapes_and_policies_synced(case):
     run_synced(pair, case["lens"], 12, 2048)
 
 
+class ZeroQueryPair(Pair):
+    """All-zero queries: every score is 0, attention is uniform, and every
+    token of a segment gets the same EMA value."""
+
+    def step_inputs(self, V):
+        q, kn, vn, pn, logits = super().step_inputs(V)
+        return torch.zeros_like(q), kn, vn, pn, logits
+
+
+@pytest.mark.parametrize("alpha,zero_q", [(0.5, False), (1.0, True)], ids=["histogram", "all_keys_tied"])
+def test_bulk_select_long_prompts_synced(alpha, zero_q):
+    # Prompts longer than the 2048 keys the whole-CTA select sorts outright, so
+    # the first step's bulk eviction finds its threshold from the key histogram;
+    # with uniform attention and alpha 1 every key ties in its score, one bin
+    # holds them all and the radix select decides (ties go by position).
+    p = Params(n_low=300, n_high=600, alpha=alpha, protect_last=32, fp16_window=64, n_sink=2)
+    cls = ZeroQueryPair if zero_q else Pair
+    pair = cls(1, 2, 8, 128, 2, p, max_prefill=5000, seed=11)
+    run_synced(pair, [5000, 3100], 4, 2048)
+
+
 @pytest.mark.parametrize("int8", [False, True])
 def test_fixed_budget_mode_synced(int8):
     p = Params(mode="fixed", n_sink=4, protect_last=24, fixed_budget=96, int8=int8, fp16_window=40)

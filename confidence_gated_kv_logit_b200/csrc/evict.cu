@@ -1,5 +1,6 @@
 // Eviction, compaction and conversion of the token leaving the FP16 window,
-// one CTA per segment (CONF-KV post, decode-loop pseudo-code: evict only when
+// one warp per segment in the common step, the whole CTA for large evictions
+// (CONF-KV post, decode-loop pseudo-code: evict only when
 // the layer holds more than its budget, rank by alpha*EMA + (1-alpha)*recency,
 // never evict the last P tokens, then convert tokens older than the window to
 // INT8; the post's implementation note names contiguous compaction as the hard
@@ -10,8 +11,10 @@
 //   1. n = cold tokens + occupied window slots; budget_eff = max(budget, P + s)
 //      (fixed mode: B); e = n - budget_eff victims if positive.
 //   2. keys (ordered score bits << 32 | position) of unprotected tokens; the e
-//      smallest are the victims: argmin when e = 1 (the steady state: one new
-//      token per step), MSD radix select otherwise (budget drops, step 1).
+//      smallest are the victims. Up to 16 victims (the steady state: one new
+//      token per step) by one warp, from this step's candidate record or a
+//      warp scan; more (budget drops, step 1) by the whole CTA, from the e-th
+//      smallest key found by a histogram of the keys (select.cuh).
 //   3. victims in the window ring free their slot; victims in the cold region
 //      are recorded in a bitmask and the region is compacted: hole-fill moves
 //      the survivors above the new end into the holes below it (bytes

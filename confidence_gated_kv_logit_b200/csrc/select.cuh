@@ -1,6 +1,7 @@
 // Block-wide building blocks for the segmented top-k select (one CTA per
-// segment): flag scans, ordered collection, argmin and MSD radix select on
-// 64-bit keys (score bits, position) that are unique within a segment.
+// segment): flag scans, ordered collection, argmin, MSD radix select and a
+// histogram threshold select on 64-bit keys (score bits, position) that are
+// unique within a segment.
 #pragma once
 
 #include "common.cuh"

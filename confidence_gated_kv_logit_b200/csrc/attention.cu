@@ -188,20 +188,26 @@ __global__ void __launch_bounds__(256) append_kernel(Cache c, AttnLaunch a, int 
   if (warp >= r.items(c.Hkv)) return;
   int l, b, h;
   const int s = seg_of(c, r, warp, &l, &b, &h);
-  prepare_query<D, GP>(c, a, s, l, b, h, lane, qscale);   // independent of the cache state: first
+  // Every load that depends on nothing but the segment is issued first (the
+  // query work below stores, and the compiler keeps loads after stores):
+  // the counters and the new K/V row travel with the query's loads.
   const int t = c.next_pos[s];
-  if (!guard(t >= 0 && c.n_cold[s] >= 0 && c.n_cold[s] <= c.cap, c.err, kSiteAppendSeg, s, t)) return;
+  const int n_cold0 = c.n_cold[s];
   const size_t in_row = ((size_t)((l - r.l0) * r.B + b) * c.Hkv + h);
   const __half* kn = a.k_new + in_row * D;
   const __half* vn = a.v_new + in_row * D;
   const float sc_new = fixed_mode ? a.prio_new[in_row] : 0.0f;
-  uint32_t w[D / 64];
+  uint32_t kw[D / 64], vw[D / 64];
+  row_load_plain<D>(kn, lane, kw);
+  row_load_plain<D>(vn, lane, vw);
+  prepare_query<D, GP>(c, a, s, l, b, h, lane, qscale);   // independent of the cache state
+  if (!guard(t >= 0 && n_cold0 >= 0 && n_cold0 <= c.cap, c.err, kSiteAppendSeg, s, t)) return;
   if (c.W > 0) {
     const int slot = t % c.W;
     const size_t rs = (size_t)s * c.Wst + slot;
     const int old = c.pos_r[rs];
     if (old >= 0) {
-      const int idx = c.n_cold[s];
+      const int idx = n_cold0;
       if (idx >= c.cap) {
         if (lane == 0) set_error(c.err, kErrDevice);
         return;
@@ -216,25 +222,21 @@ __global__ void __launch_bounds__(256) append_kernel(Cache c, AttnLaunch a, int 
       }
       __syncwarp();
     }
-    row_load_plain<D>(kn, lane, w);
-    row_store_h<D>(c.kr + (size_t)s * c.Wst * D, slot, lane, w);
-    row_load_plain<D>(vn, lane, w);
-    row_store_h<D>(c.vr + (size_t)s * c.Wst * D, slot, lane, w);
+    row_store_h<D>(c.kr + (size_t)s * c.Wst * D, slot, lane, kw);
+    row_store_h<D>(c.vr + (size_t)s * c.Wst * D, slot, lane, vw);
     if (lane == 0) {
       c.pos_r[rs] = t;
       c.sc_r[rs] = sc_new;
     }
   } else {
-    const int idx = c.n_cold[s];
+    const int idx = n_cold0;
     if (idx >= c.cap) {
       if (lane == 0) set_error(c.err, kErrDevice);
       return;
     }
     const size_t cs = (size_t)s * c.cap + idx;
-    row_load_plain<D>(kn, lane, w);
-    row_store_h<D>(c.kc + (size_t)s * c.cap * D, idx, lane, w);
-    row_load_plain<D>(vn, lane, w);
-    row_store_h<D>(c.vc + (size_t)s * c.cap * D, idx, lane, w);
+    row_store_h<D>(c.kc + (size_t)s * c.cap * D, idx, lane, kw);
+    row_store_h<D>(c.vc + (size_t)s * c.cap * D, idx, lane, vw);
     if (lane == 0) {
       c.pos_c[cs] = t;
       c.sc_c[cs] = sc_new;

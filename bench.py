@@ -45,6 +45,10 @@ def args_parse():
     ap.add_argument("--prefill", type=int, default=None, help="smaller case for profiling captures")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--calls", default="all-layers", choices=["all-layers", "per-layer"],
+                    help="per-layer: one attention call per layer, as a model's layers run (eviction stays one call)")
+    ap.add_argument("--compact", default="hole-fill", choices=["hole-fill", "stable"],
+                    help="stable: order-preserving compaction instead of hole-fill")
     return ap.parse_args()
 
 
@@ -54,6 +58,8 @@ def workload(args):
         w["L"] = args.layers
     if args.prefill:
         w["T"] = args.prefill
+    w["calls"] = getattr(args, "calls", "all-layers")
+    w["compact"] = getattr(args, "compact", "hole-fill")
     return w
 
 
@@ -61,6 +67,10 @@ def workload_name(w):
     name = (f"llama3-8b-shape decode: {w['L']} layers, {w['Hq']}q/{w['Hkv']}kv heads, D{w['D']}, batch {w['B']}, "
             f"prefill {w['T']}, vocab {w['V']}, N {w['n_low']}/{w['n_high']}, P{w['P']}, W{w['W']}, "
             f"steady-state steps after the bulk first step")
+    if w.get("calls", "all-layers") != "all-layers":
+        name += ", one attention call per layer"
+    if w.get("compact", "hole-fill") != "hole-fill":
+        name += ", stable compaction"
     return name if (w["L"], w["T"]) == (FULL["L"], FULL["T"]) else "reduced case (profiling): " + name
 
 
@@ -311,7 +321,8 @@ def main():
     G = Hq // Hkv
     warm_library(w, dev)
     h = ConfKV(L, Hkv, Hq, D, max_batch=B, max_prefill=T, n_low=w["n_low"], n_high=w["n_high"], tau=w["tau"],
-               alpha=w["alpha"], ema_decay=w["beta"], protect_last=w["P"], fp16_window=w["W"])
+               alpha=w["alpha"], ema_decay=w["beta"], protect_last=w["P"], fp16_window=w["W"],
+               compact=1 if w["compact"] == "stable" else 0)
     gen = synth.generator(1000 + rank, dev)
     for l in range(L):
         k, v = synth.prefill_kv(B, Hkv, T, D, gen, dev)
@@ -326,9 +337,16 @@ def main():
     c_out = torch.empty(B, device=dev)
     stream = torch.cuda.current_stream()
 
+    def attn_call(q, kn, vn, o):
+        if w["calls"] == "per-layer":
+            for l in range(L):
+                h.decode_attn(q[l], kn[l], vn[l], o[l], l)
+        else:
+            h.decode_attn(q, kn, vn, o, ALL_LAYERS)
+
     def step(i):
         q, kn, vn, lg = pool[i % POOL]
-        h.decode_attn(q, kn, vn, out, ALL_LAYERS)
+        attn_call(q, kn, vn, out)
         h.confidence(lg, c_out)
         h.evict_compact(ALL_LAYERS)
 
@@ -382,8 +400,8 @@ def main():
     n8 = sb["attn_tokens_int8"] - sa["attn_tokens_int8"]
     n16 = sb["attn_tokens_fp16"] - sa["attn_tokens_fp16"]
     launches = max(1, prof["attention"]["launches"])
-    qo = L * B * Hq * (2 * D + 4 * D + 4)                       # q read, out + lse written
-    attn_bytes = (n8 * (2 * D + 8 + 4 * G) + n16 * (4 * D + 4 * G)) / launches + qo
+    qo = L * B * Hq * (2 * D + 4 * D + 4)                       # q read, out + lse written, per step
+    attn_bytes = (n8 * (2 * D + 8 + 4 * G) + n16 * (4 * D + 4 * G) + qo * K) / launches
     attn_ms = prof["attention"]["ms"] / launches
     peak, peak_kind = peaks()
     achieved = attn_bytes / (attn_ms * 1e-3) / 1e9
@@ -461,7 +479,7 @@ def main():
         if i >= 2:
             stream.wait_event(ev_out[j])               # step i-2's results have left buffer set j
         dq, dk, dv, dl = dbuf[j]
-        h.decode_attn(dq, dk, dv, obuf[j], ALL_LAYERS)
+        attn_call(dq, dk, dv, obuf[j])
         h.confidence(dl, cbuf[j])
         h.evict_compact(ALL_LAYERS)
         ev_comp[j].record(stream)

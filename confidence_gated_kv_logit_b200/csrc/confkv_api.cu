@@ -82,7 +82,16 @@ struct confkv_handle {
   uint32_t* kscratch;            // evict scratch, per CTA of the largest evict grid
   int* sched;                    // attention unit counters (zero between launches)
   cudaStream_t ema_stream;       // side stream of the EMA pass
-  cudaEvent_t attn_done, ema_done;
+  cudaEvent_t attn_done;
+  // Completion of the EMA passes, per layer: layer_ev[l] indexes the ring
+  // event recorded after the last EMA pass over layer l (-1: none yet). A
+  // call waits only for the passes of its own layers, so per-layer calls do
+  // not queue behind the previous layer's pass. Ring slots are reused oldest
+  // first; a reused slot completes after the pass it replaced (one side
+  // stream), so waiting on it is never too early.
+  std::vector<cudaEvent_t> ema_ev;
+  std::vector<int> layer_ev;
+  int ev_next = 0;
   int scratch_stride;
   int32_t* keep_list;
   int32_t* keep_count;
@@ -334,20 +343,24 @@ confkv_status confkv_create(int32_t layers, int32_t kv_heads, int32_t q_heads, i
     return cuda_status(e);
   }
   h->ema_stream = nullptr;
-  h->attn_done = h->ema_done = nullptr;
+  h->attn_done = nullptr;
   // The EMA pass gets the device's highest stream priority: it and the
   // caller's next kernel (the confidence reduction) become ready together
   // when attention ends, and the EMA's long-segment warps should start first,
   // with the other kernel filling the SM slots its short segments free.
   int prio_least = 0, prio_greatest = 0;
   if (cudaDeviceGetStreamPriorityRange(&prio_least, &prio_greatest) != cudaSuccess) prio_greatest = 0;
-  if (cudaStreamCreateWithPriority(&h->ema_stream, cudaStreamNonBlocking, prio_greatest) != cudaSuccess ||
-      cudaEventCreateWithFlags(&h->attn_done, cudaEventDisableTiming) != cudaSuccess ||
-      cudaEventCreateWithFlags(&h->ema_done, cudaEventDisableTiming) != cudaSuccess ||
-      cudaEventRecord(h->ema_done, h->ema_stream) != cudaSuccess) {
+  h->layer_ev.assign(layers, -1);
+  h->ema_ev.assign(2 * (size_t)layers + 2, nullptr);
+  bool ev_ok = cudaStreamCreateWithPriority(&h->ema_stream, cudaStreamNonBlocking, prio_greatest) == cudaSuccess &&
+               cudaEventCreateWithFlags(&h->attn_done, cudaEventDisableTiming) == cudaSuccess;
+  for (cudaEvent_t& ev : h->ema_ev)
+    ev_ok = ev_ok && cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) == cudaSuccess;
+  if (!ev_ok) {
     if (h->ema_stream) cudaStreamDestroy(h->ema_stream);
     if (h->attn_done) cudaEventDestroy(h->attn_done);
-    if (h->ema_done) cudaEventDestroy(h->ema_done);
+    for (cudaEvent_t ev : h->ema_ev)
+      if (ev) cudaEventDestroy(ev);
     B.release();
     h->magic = kDead;
     delete h;
@@ -361,6 +374,19 @@ confkv_status confkv_create(int32_t layers, int32_t kv_heads, int32_t q_heads, i
   return CONFKV_OK;
 }
 
+// Make `st` wait for the last EMA pass over every layer of r.
+static cudaError_t wait_ema(confkv_handle* h, const confkv::Range& r, cudaStream_t st) {
+  int last = -1;
+  for (int l = r.l0; l < r.l0 + r.nl; ++l) {
+    const int k = h->layer_ev[l];
+    if (k < 0 || k == last) continue;   // consecutive layers of one call share their event
+    const cudaError_t e = cudaStreamWaitEvent(st, h->ema_ev[k], 0);
+    if (e != cudaSuccess) return e;
+    last = k;
+  }
+  return cudaSuccess;
+}
+
 confkv_status confkv_destroy(confkv_handle* h) {
   if (!h) return CONFKV_OK;
   {
@@ -370,7 +396,8 @@ confkv_status confkv_destroy(confkv_handle* h) {
   cudaDeviceSynchronize();
   if (h->ema_stream) cudaStreamDestroy(h->ema_stream);
   if (h->attn_done) cudaEventDestroy(h->attn_done);
-  if (h->ema_done) cudaEventDestroy(h->ema_done);
+  for (cudaEvent_t ev : h->ema_ev)
+    if (ev) cudaEventDestroy(ev);
   h->buf.release();
   h->magic = kDead;
   delete h;
@@ -410,7 +437,7 @@ confkv_status confkv_prefill(confkv_handle* h, int32_t layer, int32_t batch, con
   layer_range(h, layer, &r);
   cudaError_t e = cudaMemcpyAsync(h->lens_dev, lens_host, (size_t)batch * 4, cudaMemcpyHostToDevice, st);
   if (e != cudaSuccess) return CONFKV_ERR_CUDA;
-  if (cudaStreamWaitEvent(st, h->ema_done, 0) != cudaSuccess) return CONFKV_ERR_CUDA;
+  if (wait_ema(h, r, st) != cudaSuccess) return CONFKV_ERR_CUDA;
   confkv::PrefillLaunch a;
   a.r = r;
   a.lens = h->lens_dev;
@@ -493,12 +520,18 @@ confkv_status confkv_decode_attn(confkv_handle* h, int32_t layer, const void* q,
   a.sched = h->sched;
   a.ema_stream = h->ema_stream;
   a.attn_done = h->attn_done;
-  a.ema_done = h->ema_done;
-  // the previous EMA pass must be done before this step rewrites scores and EMA values
-  if (cudaStreamWaitEvent(static_cast<cudaStream_t>(stream), h->ema_done, 0) != cudaSuccess) return CONFKV_ERR_CUDA;
+  const int ev = h->ev_next;
+  a.ema_done = h->ema_ev[ev];
+  // the previous EMA pass over these layers must be done before this step
+  // rewrites their scores and EMA values
+  if (wait_ema(h, r, static_cast<cudaStream_t>(stream)) != cudaSuccess) return CONFKV_ERR_CUDA;
   cudaError_t e =
       confkv::launch_decode_attn(h->c, h->pol, a, static_cast<cudaStream_t>(stream), &h->launches, h->prof_ptr());
   if (e != cudaSuccess) return cuda_status(e);
+  if (h->pol.mode == 0) {   // an EMA pass ran (and recorded ema_ev[ev]) for these layers
+    for (int l = r.l0; l < r.l0 + r.nl; ++l) h->layer_ev[l] = ev;
+    h->ev_next = (ev + 1) % (int)h->ema_ev.size();
+  }
   for (int l = r.l0; l < r.l0 + r.nl; ++l) h->ub_len[l] += 1;
   return CONFKV_OK;
 }
@@ -520,8 +553,8 @@ confkv_status confkv_evict_compact(confkv_handle* h, int32_t layer, void* stream
   a.kscratch = h->kscratch;
   a.scratch_stride = h->scratch_stride;
   a.scratch_keys = h->c.cap + h->c.Wst;
-  // the candidates and EMA values come from the EMA pass on the side stream
-  if (cudaStreamWaitEvent(static_cast<cudaStream_t>(stream), h->ema_done, 0) != cudaSuccess) return CONFKV_ERR_CUDA;
+  // the candidates and EMA values come from the EMA passes on the side stream
+  if (wait_ema(h, r, static_cast<cudaStream_t>(stream)) != cudaSuccess) return CONFKV_ERR_CUDA;
   cudaError_t e =
       confkv::launch_evict_compact(h->c, h->pol, a, static_cast<cudaStream_t>(stream), &h->launches, h->prof_ptr());
   if (e != cudaSuccess) return cuda_status(e);

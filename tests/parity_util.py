@@ -74,10 +74,17 @@ class Pair:
         logits = synth.bursty_logits(self.B, V, self.gen, self.dev) if self.p.mode != "fixed" else None
         return q, kn, vn, pn, logits
 
+    def gpu_decode_attn(self, q, kn, vn, out, pn, lse):
+        """The library's attention for every layer of the step (one call)."""
+        self.gpu.decode_attn(q, kn, vn, out, ALL_LAYERS, prio_new=pn, lse_out=lse)
+
+    def gpu_evict(self):
+        self.gpu.evict_compact()
+
     def attn(self, q, kn, vn, pn):
         out = torch.empty((self.L, self.B, self.Hq, self.D), device=self.dev)
         lse = torch.empty((self.L, self.B, self.Hq), device=self.dev)
-        self.gpu.decode_attn(q, kn, vn, out, ALL_LAYERS, prio_new=pn, lse_out=lse)
+        self.gpu_decode_attn(q, kn, vn, out, pn, lse)
         qh, kh, vh = q.cpu().numpy(), kn.cpu().numpy(), vn.cpu().numpy()
         ph = None if pn is None else pn.cpu().numpy()
         o_out = np.zeros((self.L, self.B, self.Hq, self.D))
@@ -162,7 +169,7 @@ def run_synced(pair: Pair, lens, steps, V, T=None, check_every=1):
             assert np.abs(c_g - c_o).max() <= ATOL_C, (c_g, c_o)
             assert np.array_equal(bud_g, bud_o), (step, bud_g, bud_o, override)
         pair.sync_scores_from_gpu()
-        pair.gpu.evict_compact()
+        pair.gpu_evict()
         for l in range(pair.L):
             pair.orc.evict_compact(l)
         if check:

@@ -57,6 +57,30 @@ def test_bulk_select_long_prompts_synced(alpha, zero_q):
     run_synced(pair, [5000, 3100], 4, 2048)
 
 
+class PerLayerPair(Pair):
+    """Real-model call pattern: one attention call per layer (as a model's
+    layers run one after another), then one eviction call per layer."""
+
+    def gpu_decode_attn(self, q, kn, vn, out, pn, lse):
+        for l in range(self.L):
+            self.gpu.decode_attn(q[l], kn[l], vn[l], out[l], l, prio_new=None if pn is None else pn[l],
+                                 lse_out=lse[l])
+
+    def gpu_evict(self):
+        for l in range(self.L):
+            self.gpu.evict_compact(l)
+
+
+@pytest.mark.parametrize("mode", ["confidence", "fixed"])
+def test_per_layer_calls_synced(mode):
+    if mode == "fixed":
+        p = Params(mode="fixed", n_sink=4, protect_last=24, fixed_budget=96, fp16_window=40)
+    else:
+        p = Params(n_low=64, n_high=160, protect_last=16, fp16_window=32, n_sink=2, pyramidal=True)
+    pair = PerLayerPair(3, 2, 8, 128, 2, p, max_prefill=400, seed=12)
+    run_synced(pair, [400, 150], 8, 0 if mode == "fixed" else 2048)
+
+
 @pytest.mark.parametrize("int8", [False, True])
 def test_fixed_budget_mode_synced(int8):
     p = Params(mode="fixed", n_sink=4, protect_last=24, fixed_budget=96, int8=int8, fp16_window=40)

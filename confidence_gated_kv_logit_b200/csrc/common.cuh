@@ -144,6 +144,14 @@ __device__ __forceinline__ void i8x4_to_f2x2(uint32_t w, float2& lo, float2& hi)
   hi = __fadd2_rn(b, bias);
 }
 
+// 2^x with the SFU's approximation (relative error about 2^-22; results below
+// 2^-126 flush to zero): the softmax weights and the EMA terms.
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ float2 h2_to_f2(uint32_t w) {
   return __half22float2(*reinterpret_cast<const __half2*>(&w));
 }

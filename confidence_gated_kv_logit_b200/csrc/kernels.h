@@ -73,6 +73,9 @@ cudaError_t launch_decode_attn(const Cache& c, const Policy& pol, const AttnLaun
                                long long* launches, Prof* prof);
 // Bytes of the prepared query operands of one segment (qfrag stride).
 int qfrag_bytes(int D, int G);
+// The EMA pass of a decode call (after attention and, with splits, the
+// combine), on stream st.
+cudaError_t run_ema(const Cache& c, const Policy& pol, const AttnLaunch& a, cudaStream_t st);
 
 // K4 + K5 + K6: select, compaction, conversion of the token leaving the window.
 struct EvictLaunch {

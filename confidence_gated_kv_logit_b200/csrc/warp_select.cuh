@@ -100,8 +100,12 @@ static_assert(offsetof(EvictCand, n_ring) % 16 == 0, "the record header is one a
 // how many of them are certainly the segment's smallest: a lane whose list
 // was full dropped only keys above its largest kept key k3, so the merged
 // keys up to the smallest such k3 are exact.
+// If `complete_below` is given it receives a key B such that every key <= B
+// that this warp saw is in the merged list (the smallest full-list k3, or the
+// last merged key when the list was cut at `want`).
 __device__ __forceinline__ void warp_merge_smallest(LaneBest& best, int lane, int want, unsigned long long* my_key,
-                                                    int* my_idx, int* count, int* safe) {
+                                                    int* my_idx, int* count, int* safe,
+                                                    unsigned long long* complete_below = nullptr) {
   const unsigned long long k3 = best.k[kLaneKeep - 1];
   const unsigned long long lim = warp_min_u64(k3);   // kNoKey when no list is full
   unsigned long long mk = kNoKey;
@@ -123,6 +127,10 @@ __device__ __forceinline__ void warp_merge_smallest(LaneBest& best, int lane, in
   *my_idx = mi;
   *count = n;
   *safe = __popc(__ballot_sync(0xffffffffu, lane < n && mk <= lim));
+  if (complete_below != nullptr) {
+    const unsigned long long last = n == want && n > 0 ? __shfl_sync(0xffffffffu, mk, n - 1) : kNoKey;
+    *complete_below = last < lim ? last : lim;
+  }
 }
 
 }  // namespace confkv

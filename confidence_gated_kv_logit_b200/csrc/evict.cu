@@ -495,7 +495,15 @@ __device__ void evict_segment_block(const Cache& c, const Policy& pol, const Evi
       return none ? 0xFFFFFFFFu : (uint32_t)(rank_key(pol, sc, pos, t) >> 32);
     };
     // cold region: 8 tokens per thread per step in two 16-byte loads each of
-    // positions and EMA values (the region is a multiple of 64 tokens long)
+    // positions and EMA values (the region is a multiple of 64 tokens long);
+    // each thread also keeps the range of its counted keys for the select
+    uint32_t kmn = 0xFFFFFFFFu, kmx = 0u;
+    auto track = [&](uint32_t hv) {
+      if (hv != 0xFFFFFFFFu) {
+        kmn = min(kmn, hv);
+        kmx = max(kmx, hv);
+      }
+    };
     for (int i0 = 8 * threadIdx.x; i0 < n_cold; i0 += 8 * NT) {
       const int4 p0 = reinterpret_cast<const int4*>(pos_c + i0)[0];
       const int4 p1 = reinterpret_cast<const int4*>(pos_c + i0)[1];
@@ -505,7 +513,10 @@ __device__ void evict_segment_block(const Cache& c, const Policy& pol, const Evi
       const float ff[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
       uint32_t hv[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) hv[j] = i0 + j < n_cold ? hi_of(pp[j], ff[j]) : 0xFFFFFFFFu;
+      for (int j = 0; j < 8; ++j) {
+        hv[j] = i0 + j < n_cold ? hi_of(pp[j], ff[j]) : 0xFFFFFFFFu;
+        track(hv[j]);
+      }
       if (i0 + 8 <= n_cold) {
         reinterpret_cast<uint4*>(khi + i0)[0] = make_uint4(hv[0], hv[1], hv[2], hv[3]);
         reinterpret_cast<uint4*>(khi + i0)[1] = make_uint4(hv[4], hv[5], hv[6], hv[7]);
@@ -515,11 +526,15 @@ __device__ void evict_segment_block(const Cache& c, const Policy& pol, const Evi
           if (i0 + j < n_cold) khi[i0 + j] = hv[j];
       }
     }
-    for (int slot = threadIdx.x; slot < W; slot += NT) khi[n_cold + slot] = hi_of(pos_r[slot], sc_r[slot]);
+    for (int slot = threadIdx.x; slot < W; slot += NT) {
+      const uint32_t hv = hi_of(pos_r[slot], sc_r[slot]);
+      khi[n_cold + slot] = hv;
+      track(hv);
+    }
     __syncthreads();
     // the e-th smallest key: the victims are the keys up to it
-    const unsigned long long thr =
-        block_select_threshold<NT>(khi, pos_of, span, e, sm, reinterpret_cast<unsigned long long*>(es.stage));
+    const unsigned long long thr = block_select_threshold<NT>(
+        khi, pos_of, span, e, sm, reinterpret_cast<unsigned long long*>(es.stage), true, kmn, kmx);
     const uint32_t thr_hi = (uint32_t)(thr >> 32), thr_lo = (uint32_t)thr;
     auto below_thr = [&](uint32_t hv, int i) -> bool {   // the position only matters on a tie of the high half
       return hv != 0xFFFFFFFFu && (hv < thr_hi || (hv == thr_hi && (uint32_t)pos_of(i) <= thr_lo));

@@ -370,9 +370,14 @@ constexpr int kSelCand = (kSelBuf * 8 - kSelBins * 4) / 8;   // keys of one bin 
 // which are sorted. When that bin is too full for the buffer, the radix
 // select above decides (its result, as a threshold, is prefix | ~mask).
 // buf: kSelBuf 64-bit entries of shared memory.
+// A caller that has just written the high halves may pass its threads' own
+// minimum and maximum of the counted ones (range_given): the range pass is
+// then skipped.
 template <int NT, typename LoFn>
 __device__ unsigned long long block_select_threshold(const uint32_t* __restrict__ hi, LoFn lo, int n, int k,
-                                                     SelectSmem<NT>& sm, unsigned long long* buf) {
+                                                     SelectSmem<NT>& sm, unsigned long long* buf,
+                                                     bool range_given = false, uint32_t my_mn = 0xFFFFFFFFu,
+                                                     uint32_t my_mx = 0u) {
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   if (n <= kSelBuf) {
     int m = 1;
@@ -395,8 +400,8 @@ __device__ unsigned long long block_select_threshold(const uint32_t* __restrict_
   const int n4 = (n + 3) >> 2;
   auto key_at = [&](const uint4& q, int j) { return j == 0 ? q.x : j == 1 ? q.y : j == 2 ? q.z : q.w; };
   // pass 1: the range of the counted high halves
-  uint32_t mn = 0xFFFFFFFFu, mx = 0u;
-  for (int v0 = threadIdx.x; v0 < n4; v0 += 4 * NT) {
+  uint32_t mn = my_mn, mx = my_mx;
+  for (int v0 = threadIdx.x; !range_given && v0 < n4; v0 += 4 * NT) {
     uint4 q[4];
 #pragma unroll
     for (int r = 0; r < 4; ++r) q[r] = v0 + r * NT < n4 ? hi4[v0 + r * NT] : make_uint4(~0u, ~0u, ~0u, ~0u);

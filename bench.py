@@ -49,6 +49,8 @@ def args_parse():
                     help="per-layer: one attention call per layer, as a model's layers run (eviction stays one call)")
     ap.add_argument("--compact", default="hole-fill", choices=["hole-fill", "stable"],
                     help="stable: order-preserving compaction instead of hole-fill")
+    ap.add_argument("--score", default="ema", choices=["ema", "accum", "random"],
+                    help="ranking source: attention-mass EMA, accumulated attention, or a static random draw")
     return ap.parse_args()
 
 
@@ -60,6 +62,7 @@ def workload(args):
         w["T"] = args.prefill
     w["calls"] = getattr(args, "calls", "all-layers")
     w["compact"] = getattr(args, "compact", "hole-fill")
+    w["score"] = getattr(args, "score", "ema")
     return w
 
 
@@ -71,6 +74,8 @@ def workload_name(w):
         name += ", one attention call per layer"
     if w.get("compact", "hole-fill") != "hole-fill":
         name += ", stable compaction"
+    if w.get("score", "ema") != "ema":
+        name += {"accum": ", accumulated-attention ranking", "random": ", random ranking"}[w["score"]]
     return name if (w["L"], w["T"]) == (FULL["L"], FULL["T"]) else "reduced case (profiling): " + name
 
 
@@ -322,7 +327,8 @@ def main():
     warm_library(w, dev)
     h = ConfKV(L, Hkv, Hq, D, max_batch=B, max_prefill=T, n_low=w["n_low"], n_high=w["n_high"], tau=w["tau"],
                alpha=w["alpha"], ema_decay=w["beta"], protect_last=w["P"], fp16_window=w["W"],
-               compact=1 if w["compact"] == "stable" else 0)
+               compact=1 if w["compact"] == "stable" else 0,
+               score_source={"ema": 0, "accum": 1, "random": 2}[w["score"]], seed=7)
     gen = synth.generator(1000 + rank, dev)
     for l in range(L):
         k, v = synth.prefill_kv(B, Hkv, T, D, gen, dev)

@@ -22,6 +22,7 @@ ALL_LAYERS = -1
 MODE_CONF, MODE_FIXED = 0, 1
 GATE_PROSE, GATE_LITERAL = 0, 1
 COMPACT_HOLEFILL, COMPACT_STABLE = 0, 1
+SCORE_EMA, SCORE_ACCUM, SCORE_RANDOM = 0, 1, 2
 
 STATUS = {0: "OK", 1: "ERR_ARG", 2: "ERR_CAPACITY", 3: "ERR_STATE", 4: "ERR_NONFINITE",
           5: "ERR_CUDA", 6: "ERR_OOM", 7: "ERR_DEVICE"}
@@ -47,7 +48,8 @@ class Params(ctypes.Structure):
                 ("n_sink", ctypes.c_int32), ("fixed_budget", ctypes.c_int32),
                 ("pyramidal", ctypes.c_int32), ("gate", ctypes.c_int32),
                 ("int8_enable", ctypes.c_int32), ("compact", ctypes.c_int32),
-                ("max_batch", ctypes.c_int32), ("max_prefill", ctypes.c_int32)]
+                ("max_batch", ctypes.c_int32), ("max_prefill", ctypes.c_int32),
+                ("score_source", ctypes.c_int32), ("seed", ctypes.c_uint32)]
 
 
 class Stats(ctypes.Structure):

@@ -172,7 +172,8 @@ __device__ __forceinline__ void prepare_query(const Cache& c, const AttnLaunch& 
 // operands are prepared.
 // ---------------------------------------------------------------------------
 template <int D, int GP>
-__global__ void __launch_bounds__(256) append_kernel(Cache c, AttnLaunch a, int fixed_mode, float qscale) {
+__global__ void __launch_bounds__(256) append_kernel(Cache c, AttnLaunch a, Policy pol, float qscale) {
+  const bool fixed_mode = pol.mode == 1;
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const Range r = a.r;
@@ -187,7 +188,7 @@ __global__ void __launch_bounds__(256) append_kernel(Cache c, AttnLaunch a, int 
   const size_t in_row = ((size_t)((l - r.l0) * r.B + b) * c.Hkv + h);
   const __half* kn = a.k_new + in_row * D;
   const __half* vn = a.v_new + in_row * D;
-  const float sc_new = fixed_mode ? a.prio_new[in_row] : 0.0f;
+  const float sc_new = fixed_mode ? a.prio_new[in_row] : initial_score(pol, l, b, h, t);
   uint32_t kw[D / 64], vw[D / 64];
   row_load_plain<D>(kn, lane, kw);
   row_load_plain<D>(vn, lane, vw);
@@ -1017,7 +1018,7 @@ cudaError_t run_attn(const Cache& c, const Policy& pol, const AttnLaunch& a, cud
   const float qscale = rsqrtf((float)D);
   {
     ProfScope ps(prof, kKAppend, st);
-    append_kernel<D, GP><<<(items * 32 + 255) / 256, 256, 0, st>>>(c, a, pol.mode == 1, qscale);
+    append_kernel<D, GP><<<(items * 32 + 255) / 256, 256, 0, st>>>(c, a, pol, qscale);
   }
   ++*launches;
   cudaError_t e = cudaGetLastError();

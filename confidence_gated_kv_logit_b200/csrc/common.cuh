@@ -70,7 +70,32 @@ struct Policy {
   int fixed_budget;
   int gate;           // 0 prose, 1 literal
   int pyramidal;
+  int score_source;   // confkv.h CONFKV_SCORE_*
+  uint32_t seed;      // static draws (CONFKV_SCORE_RANDOM)
 };
+
+constexpr int kScoreEma = 0, kScoreAccum = 1, kScoreRandom = 2;   // confkv.h CONFKV_SCORE_*
+
+// The static draw of the random ranker for token `pos` of segment (l, b, h):
+// SplitMix64 (Steele, Lea and Flood, 2014) at counter pos | h << 32 | b << 40 |
+// l << 52, i.e. its output for state seed + (counter + 1) * 0x9E3779B97F4A7C15,
+// top 24 bits as a fraction in [0, 1) (exact in fp32).
+__host__ __device__ __forceinline__ float random_priority(uint32_t seed, int l, int b, int h, int pos) {
+  const unsigned long long ctr = (unsigned long long)(uint32_t)pos | ((unsigned long long)(h & 0xff) << 32) |
+                                 ((unsigned long long)(b & 0xfff) << 40) | ((unsigned long long)(l & 0xfff) << 52);
+  unsigned long long z = (unsigned long long)seed + (ctr + 1ull) * 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  z ^= z >> 31;
+  return (float)(z >> 40) * 0x1p-24f;
+}
+
+// The initial score source of a token entering the cache (prefill or append)
+// in confidence mode: 0 for the EMA and the accumulated mass, the draw for the
+// random ranker.
+__device__ __forceinline__ float initial_score(const Policy& pol, int l, int b, int h, int pos) {
+  return pol.score_source == kScoreRandom ? random_priority(pol.seed, l, b, h, pos) : 0.0f;
+}
 
 // A call covers layers [l0, l0 + nl) and sequences [0, B) of every KV head.
 struct Range {

@@ -135,7 +135,7 @@ static bool layer_range(const confkv_handle* h, int32_t layer, confkv::Range* r)
 
 extern "C" {
 
-int32_t confkv_version(void) { return 100; }
+int32_t confkv_version(void) { return 101; }
 
 const char* confkv_status_string(confkv_status s) {
   switch (s) {
@@ -170,6 +170,8 @@ confkv_status confkv_default_params(confkv_params* p) {
   p->compact = CONFKV_COMPACT_HOLEFILL;
   p->max_batch = 1;
   p->max_prefill = 4096;
+  p->score_source = CONFKV_SCORE_EMA;
+  p->seed = 0u;
   return CONFKV_OK;
 }
 
@@ -185,6 +187,9 @@ confkv_status confkv_create(int32_t layers, int32_t kv_heads, int32_t q_heads, i
   if (p.mode != CONFKV_MODE_CONF && p.mode != CONFKV_MODE_FIXED) return CONFKV_ERR_ARG;
   if (p.gate != CONFKV_GATE_PROSE && p.gate != CONFKV_GATE_LITERAL) return CONFKV_ERR_ARG;
   if (p.compact != CONFKV_COMPACT_HOLEFILL && p.compact != CONFKV_COMPACT_STABLE) return CONFKV_ERR_ARG;
+  if (p.score_source != CONFKV_SCORE_EMA && p.score_source != CONFKV_SCORE_ACCUM &&
+      p.score_source != CONFKV_SCORE_RANDOM)
+    return CONFKV_ERR_ARG;
   if (p.max_batch < 1 || p.max_prefill < 0 || p.protect_last < 0 || p.n_sink < 0) return CONFKV_ERR_ARG;
   if (!(p.alpha >= 0.0f && p.alpha <= 1.0f) || !(p.ema_decay >= 0.0f && p.ema_decay <= 1.0f)) return CONFKV_ERR_ARG;
   if (!std::isfinite(p.tau)) return CONFKV_ERR_ARG;
@@ -254,8 +259,15 @@ confkv_status confkv_create(int32_t layers, int32_t kv_heads, int32_t q_heads, i
   pol.tau = p.tau;
   pol.alpha = p.alpha;
   pol.one_minus_alpha = 1.0f - p.alpha;
-  pol.beta = p.ema_decay;
-  pol.one_minus_beta = 1.0f - p.ema_decay;
+  // The EMA pass computes fl(beta*x + w*m) with m the step's mean attention:
+  // EMA w = 1 - beta; accumulated attention beta = w = 1 (x + m); a static
+  // draw beta = 1, w = 0 (x unchanged).
+  pol.score_source = p.mode == CONFKV_MODE_CONF ? p.score_source : CONFKV_SCORE_EMA;
+  pol.seed = p.seed;
+  pol.beta = pol.score_source == CONFKV_SCORE_EMA ? p.ema_decay : 1.0f;
+  pol.one_minus_beta = pol.score_source == CONFKV_SCORE_EMA    ? 1.0f - p.ema_decay
+                       : pol.score_source == CONFKV_SCORE_ACCUM ? 1.0f
+                                                                : 0.0f;
   pol.P = p.protect_last;
   pol.n_sink = p.n_sink;
   pol.fixed_budget = p.fixed_budget;

@@ -81,7 +81,7 @@ __global__ void __launch_bounds__(NT) prefill_select_kernel(Cache c, Policy pol,
 
 // One warp per (segment, token): copy or quantise the K and V rows.
 template <int D>
-__global__ void __launch_bounds__(NT) prefill_ingest_kernel(Cache c, PrefillLaunch a, int fixed_mode,
+__global__ void __launch_bounds__(NT) prefill_ingest_kernel(Cache c, Policy pol, PrefillLaunch a, int fixed_mode,
                                                             int per_item) {
   const long long gw = ((long long)blockIdx.x * NT + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
@@ -102,7 +102,7 @@ __global__ void __launch_bounds__(NT) prefill_ingest_kernel(Cache c, PrefillLaun
   const size_t in_row = (((size_t)((l - a.r.l0) * a.r.B + b) * c.Hkv + h) * a.t_stride + p);
   const __half* ksrc = a.k + in_row * D;
   const __half* vsrc = a.v + in_row * D;
-  const float sc = fixed_mode ? a.prio[in_row] : 0.0f;
+  const float sc = fixed_mode ? a.prio[in_row] : initial_score(pol, l, b, h, p);
   uint32_t w[D / 64];
   if (c.W > 0 && p > len - c.W) {
     const int slot = p % c.W;
@@ -163,8 +163,8 @@ cudaError_t launch_prefill(const Cache& c, const Policy& pol, const PrefillLaunc
   const long long warps = (long long)items * per_item;
   if (warps == 0) return cudaSuccess;
   const long long blocks = (warps * 32 + NT - 1) / NT;
-  if (c.D == 128) prefill_ingest_kernel<128><<<(unsigned)blocks, NT, 0, st>>>(c, a, fixed ? 1 : 0, per_item);
-  else prefill_ingest_kernel<64><<<(unsigned)blocks, NT, 0, st>>>(c, a, fixed ? 1 : 0, per_item);
+  if (c.D == 128) prefill_ingest_kernel<128><<<(unsigned)blocks, NT, 0, st>>>(c, pol, a, fixed ? 1 : 0, per_item);
+  else prefill_ingest_kernel<64><<<(unsigned)blocks, NT, 0, st>>>(c, pol, a, fixed ? 1 : 0, per_item);
   ++*launches;
   return cudaGetLastError();
 }

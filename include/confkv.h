@@ -70,6 +70,18 @@ enum { CONFKV_MODE_CONF = 0, CONFKV_MODE_FIXED = 1 };
 enum { CONFKV_GATE_PROSE = 0, CONFKV_GATE_LITERAL = 1 };
 /* Compaction variant; both give the same logical cache content. */
 enum { CONFKV_COMPACT_HOLEFILL = 0, CONFKV_COMPACT_STABLE = 1 };
+/* Score source of the confidence mode's ranking (score = alpha*source +
+ * (1-alpha)*recency):
+ *   EMA    ema <- beta*ema + (1-beta)*a (the CONF-KV post's EMA; the default);
+ *   ACCUM  acc <- acc + a, the attention mass accumulated over the steps (the
+ *          heavy-hitter score the CONF-KV post's related work, H2O, uses);
+ *   RANDOM a static per-token draw u in [0, 1), from SplitMix64 (Steele, Lea
+ *          and Flood, 2014) at counter pos | h << 32 | b << 40 | l << 52
+ *          (position, KV head, sequence, layer): state seed + (counter + 1) *
+ *          0x9E3779B97F4A7C15, mixed, u = (mix >> 40) * 2^-24.
+ * a is the token's attention probability this step, averaged over the G query
+ * heads. These are the ranker variants of the matched-rate ablation. */
+enum { CONFKV_SCORE_EMA = 0, CONFKV_SCORE_ACCUM = 1, CONFKV_SCORE_RANDOM = 2 };
 
 #define CONFKV_ALL_LAYERS (-1)
 
@@ -90,6 +102,8 @@ typedef struct {
   int32_t compact;       /* CONFKV_COMPACT_HOLEFILL or CONFKV_COMPACT_STABLE */
   int32_t max_batch;     /* sequences the cache is sized for */
   int32_t max_prefill;   /* longest prompt confkv_prefill accepts (tokens) */
+  int32_t score_source;  /* CONFKV_SCORE_EMA, CONFKV_SCORE_ACCUM or CONFKV_SCORE_RANDOM (confidence mode) */
+  uint32_t seed;         /* CONFKV_SCORE_RANDOM: seed of the per-token draws */
 } confkv_params;
 
 typedef struct {

@@ -29,6 +29,14 @@ Readings where the pages are silent:
 * Order: the higher (score, position) pair is kept, so equal scores go to the
   newer token. Protected tokens (age t - pos < P, or pos < n_sink) never
   compete.
+* Ranker variants (the matched-rate ablation of the hot-path plan): the EMA
+  above; the attention mass accumulated over the steps, acc <- acc + a (the
+  heavy-hitter score of H2O, which the CONF-KV post lists as related work);
+  and a static uniform draw per token. The draw is SplitMix64 (Steele, Lea and
+  Flood, 2014, "Fast splittable pseudorandom number generators") used as a
+  counter-based generator: the output for state seed + (c + 1) * gamma with
+  c = pos | h << 32 | b << 40 | l << 52 (position, KV head, sequence, layer),
+  gamma = 0x9E3779B97F4A7C15, and the value (output >> 40) * 2^-24.
 
 Pins (tests/test_oracle_policy.py): constant attention for n steps from zero
 gives a (1 - beta^n); exhaustive subset enumeration for n <= 12 equals the
@@ -54,6 +62,33 @@ def ema_update(ema, w, beta):
     a = np.asarray(w, dtype=np.float64).mean(axis=0)
     new = beta * np.asarray(ema, dtype=np.float32).astype(np.float64) + (1.0 - beta) * a
     return new.astype(np.float32)
+
+
+def accum_update(acc, w):
+    """Accumulated attention after one step: fp32(acc + a), a the mean over the
+    G heads of w [G, n] (fp64), acc fp32 [n]."""
+    a = np.asarray(w, dtype=np.float64).mean(axis=0)
+    return (np.asarray(acc, dtype=np.float32).astype(np.float64) + a).astype(np.float32)
+
+
+_M64 = (1 << 64) - 1
+_GAMMA = 0x9E3779B97F4A7C15
+
+
+def splitmix64_output(state):
+    """The SplitMix64 output for a generator state (after its increment)."""
+    z = state & _M64
+    z = ((z ^ (z >> 30)) * 0xBF58476D1CE4E5B9) & _M64
+    z = ((z ^ (z >> 27)) * 0x94D049BB133111EB) & _M64
+    return z ^ (z >> 31)
+
+
+def random_priority(seed, layer, seq, kv_head, pos):
+    """Static draw in [0, 1) for token pos of segment (layer, seq, kv_head)."""
+    ctr = (int(pos) & 0xFFFFFFFF) | ((int(kv_head) & 0xFF) << 32) | ((int(seq) & 0xFFF) << 40) \
+        | ((int(layer) & 0xFFF) << 52)
+    out = splitmix64_output(int(seed) + (ctr + 1) * _GAMMA)
+    return np.float32((out >> 40) / float(1 << 24))
 
 
 def recency(pos, t):

@@ -39,7 +39,7 @@ import numpy as np
 
 from .attention import attend
 from .confidence import confidence, choose_budget, layer_budgets
-from .policy import composite_score, ema_update, recency, select_victims
+from .policy import accum_update, composite_score, ema_update, random_priority, recency, select_victims
 from .quant import dequantize_rows, quantize_row, quantize_rows
 
 
@@ -59,6 +59,8 @@ class Params:
     pyramidal: bool = False
     gate: str = "prose"           # "prose" or "literal"
     int8: bool = True
+    score_source: str = "ema"     # conf mode ranking source: "ema", "accum" or "random"
+    seed: int = 0                 # "random": seed of the static draws
 
     def budgets_for(self, budget: int, layers: int) -> list[int]:
         return layer_budgets(budget, layers, self.pyramidal)
@@ -84,6 +86,7 @@ class Segment:
     vs: np.ndarray = None
     score_src: np.ndarray = None  # float32 [n]: EMA (conf mode) or priority (fixed)
     next_pos: int = 0
+    ident: tuple = (0, 0, 0)      # (layer, seq, kv_head), for the random ranker's draws
 
     def __post_init__(self):
         D = self.head_dim
@@ -104,7 +107,7 @@ class Segment:
     def take(self, idx) -> "Segment":
         return Segment(self.head_dim, self.pos[idx], self.is_fp16[idx], self.k16[idx],
                        self.v16[idx], self.k8[idx], self.v8[idx], self.ks[idx], self.vs[idx],
-                       self.score_src[idx], self.next_pos)
+                       self.score_src[idx], self.next_pos, self.ident)
 
     def rows_hat(self):
         """(k_hat, v_hat) as fp32 [n, D]: fp16 rows widened, INT8 rows dequantised."""
@@ -139,7 +142,15 @@ class Segment:
         self.is_fp16[i] = False
 
 
-def prefill_segment(k16, v16, prio, params: Params) -> Segment:
+def initial_score(params: Params, ident, pos) -> np.float32:
+    """Score source of a token entering the cache in confidence mode: 0, or its
+    static draw for the random ranker."""
+    if params.score_source == "random":
+        return random_priority(params.seed, *ident, pos)
+    return np.float32(0)
+
+
+def prefill_segment(k16, v16, prio, params: Params, ident=(0, 0, 0)) -> Segment:
     """Ingest T prompt tokens (positions 0..T-1) of one segment.
 
     Confidence mode evicts nothing at prefill. Fixed mode keeps the sinks, the
@@ -150,6 +161,7 @@ def prefill_segment(k16, v16, prio, params: Params) -> Segment:
     v16 = np.asarray(v16, np.float16)
     T, D = k16.shape
     seg = Segment(D)
+    seg.ident = tuple(ident)
     seg.pos = np.arange(T, dtype=np.int64)
     seg.is_fp16 = np.ones(T, bool)
     seg.k16 = k16.copy()
@@ -161,7 +173,7 @@ def prefill_segment(k16, v16, prio, params: Params) -> Segment:
     if params.mode == "fixed":
         seg.score_src = np.asarray(prio, np.float32).copy()
     else:
-        seg.score_src = np.zeros(T, np.float32)
+        seg.score_src = np.array([initial_score(params, seg.ident, p) for p in range(T)], np.float32)
     seg.next_pos = T
     if params.mode == "fixed" and T > 0:
         evict = select_victims(seg.pos, seg.score_src, T - 1, params.fixed_budget,
@@ -186,7 +198,7 @@ def decode_attn_segment(seg: Segment, q, k_new, v_new, prio_new, params: Params)
     leaving the window, and this only acts when a step skipped eviction.
     Returns (out [G, D], lse [G], w [G, n]) in fp64.
     """
-    seg.append(k_new, v_new, prio_new if params.mode == "fixed" else None)
+    seg.append(k_new, v_new, prio_new if params.mode == "fixed" else initial_score(params, seg.ident, seg.next_pos))
     if params.int8:
         t = seg.next_pos - 1
         for i in np.flatnonzero(seg.is_fp16 & (t - seg.pos >= params.fp16_window)):
@@ -194,7 +206,12 @@ def decode_attn_segment(seg: Segment, q, k_new, v_new, prio_new, params: Params)
     k_hat, v_hat = seg.rows_hat()
     out, lse, w = attend(q, k_hat, v_hat)
     if params.mode != "fixed":
-        seg.score_src = ema_update(seg.score_src, w, params.ema_decay)
+        if params.score_source == "ema":
+            seg.score_src = ema_update(seg.score_src, w, params.ema_decay)
+        elif params.score_source == "accum":
+            seg.score_src = accum_update(seg.score_src, w)
+        elif params.score_source != "random":   # random: the static draws stand
+            raise ValueError(f"unknown score source {params.score_source!r}")
     return out, lse, w
 
 
@@ -264,7 +281,8 @@ class OracleCache:
                 if not self.tracked(layer, b, h):
                     continue
                 pr = None if prio is None else np.asarray(prio)[b, h, :T]
-                self.segs[(layer, b, h)] = prefill_segment(k[b, h, :T], np.asarray(v)[b, h, :T], pr, self.p)
+                self.segs[(layer, b, h)] = prefill_segment(k[b, h, :T], np.asarray(v)[b, h, :T], pr, self.p,
+                                                           (layer, b, h))
 
     def decode_attn(self, layer, q, k_new, v_new, prio_new=None):
         q = np.asarray(q)

@@ -24,7 +24,8 @@ def c_params(p: Params, max_batch: int, max_prefill: int, stable: bool = False) 
                 fp16_window=p.fp16_window, n_sink=p.n_sink, fixed_budget=p.fixed_budget,
                 pyramidal=int(p.pyramidal), gate=0 if p.gate == "prose" else 1,
                 int8_enable=int(p.int8), compact=1 if stable else 0, max_batch=max_batch,
-                max_prefill=max_prefill)
+                max_prefill=max_prefill, score_source={"ema": 0, "accum": 1, "random": 2}[p.score_source],
+                seed=p.seed)
 
 
 class Pair:
@@ -163,7 +164,7 @@ def run_synced(pair: Pair, lens, steps, V, T=None, check_every=1):
             assert np.abs(lse_g[l, b, sl] - lse_o[l, b, sl]).max() <= ATOL_LSE
             if check:
                 assert_segment_equal(pair.gpu_segment(l, b, h), pair.orc.segment(l, b, h), (step, l, b, h),
-                                     exact_scores=pair.p.mode == "fixed")
+                                     exact_scores=pair.p.mode == "fixed" or pair.p.score_source == "random")
         if logits is not None:
             c_g, bud_g, c_o, bud_o, override = pair.confidence(logits)
             assert np.abs(c_g - c_o).max() <= ATOL_C, (c_g, c_o)

@@ -81,6 +81,16 @@ def test_per_layer_calls_synced(mode):
     run_synced(pair, [400, 150], 8, 0 if mode == "fixed" else 2048)
 
 
+@pytest.mark.parametrize("source,alpha", [("accum", 0.5), ("random", 0.5), ("random", 1.0)],
+                         ids=["accumulated_attention", "random_blend", "random_only"])
+def test_ranker_variants_synced(source, alpha):
+    # the ranker variants of the matched-rate ablation, at the same budgets
+    p = Params(n_low=80, n_high=160, alpha=alpha, protect_last=16, fp16_window=32, n_sink=2,
+               score_source=source, seed=123)
+    pair = Pair(2, 2, 8, 128, 2, p, max_prefill=600, seed=13)
+    run_synced(pair, [600, 250], 10, 2048)
+
+
 @pytest.mark.parametrize("int8", [False, True])
 def test_fixed_budget_mode_synced(int8):
     p = Params(mode="fixed", n_sink=4, protect_last=24, fixed_budget=96, int8=int8, fp16_window=40)

@@ -234,3 +234,66 @@ def test_ema_and_score_pins_catch_planted_mistakes():
             except AssertionError:
                 caught += 1
         assert caught >= 1, bad.__name__
+
+
+# ---------------------------------------------------------------------------
+# ranker variants: accumulated attention and the static random draw
+# ---------------------------------------------------------------------------
+import os  # noqa: E402
+
+from oracle.policy import accum_update, random_priority, splitmix64_output  # noqa: E402
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def test_accum_constant_attention_closed_form():
+    # constant attention a = 1/4 on every head for n steps from zero accumulates
+    # to n/4 exactly (dyadic values: every fp32 sum is exact)
+    acc = np.zeros(5, np.float32)
+    w = np.full((4, 5), 0.25)
+    for n in range(1, 41):
+        acc = accum_update(acc, w)
+        assert np.all(acc == np.float32(n / 4))
+
+
+def test_accum_is_the_running_sum_of_head_means():
+    rng = np.random.default_rng(3)
+    steps = [rng.random((3, 7)) for _ in range(6)]
+    acc = np.zeros(7, np.float32)
+    total = np.zeros(7)
+    for w in steps:
+        acc = accum_update(acc, w)
+        total += w.mean(axis=0)
+    np.testing.assert_allclose(acc, total, rtol=3e-7 * 6)
+
+
+def test_splitmix64_reference_outputs():
+    lines = open(os.path.join(GOLDEN, "splitmix64_seed0.txt")).read().splitlines()
+    want = [int(x, 16) for x in lines if x.strip() and not x.startswith("#")]
+    gamma = 0x9E3779B97F4A7C15
+    got = [splitmix64_output((k * gamma) & ((1 << 64) - 1)) for k in range(1, 6)]
+    assert got == want
+
+
+def test_random_priority_range_determinism_and_uniformity():
+    u = np.array([random_priority(9, 3, 1, 2, p) for p in range(20000)], np.float64)
+    assert np.all((u >= 0.0) & (u < 1.0))
+    assert np.all(np.float32(u) == u)   # 24-bit fractions: exact in fp32
+    assert random_priority(9, 3, 1, 2, 17) == random_priority(9, 3, 1, 2, 17)
+    # chi-square over 32 equal bins (31 degrees of freedom; 70 is far in the tail)
+    counts = np.bincount(np.minimum((u * 32).astype(int), 31), minlength=32)
+    chi2 = float(((counts - len(u) / 32) ** 2 / (len(u) / 32)).sum())
+    assert chi2 < 70.0, chi2
+    # different segments and seeds give unrelated draws
+    v = np.array([random_priority(9, 3, 1, 3, p) for p in range(20000)])
+    s2 = np.array([random_priority(10, 3, 1, 2, p) for p in range(20000)])
+    assert abs(np.corrcoef(u, v)[0, 1]) < 0.03 and abs(np.corrcoef(u, s2)[0, 1]) < 0.03
+
+
+def test_random_ranker_segment_uses_its_draws():
+    # a prefilled segment under the random ranker carries the draws of its own
+    # (layer, seq, kv_head) as its score source
+    p = Params(score_source="random", seed=5, fp16_window=4)
+    k = np.zeros((12, 8), np.float16)
+    seg = prefill_segment(k, k, None, p, (2, 1, 3))
+    assert np.array_equal(seg.score_src, np.array([random_priority(5, 2, 1, 3, i) for i in range(12)], np.float32))

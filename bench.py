@@ -49,6 +49,8 @@ def args_parse():
                     help="per-layer: one attention call per layer, as a model's layers run (eviction stays one call)")
     ap.add_argument("--compact", default="hole-fill", choices=["hole-fill", "stable"],
                     help="stable: order-preserving compaction instead of hole-fill")
+    ap.add_argument("--paged-study", action="store_true",
+                    help="after the run, the dead space a position-ordered paged layout would hold")
     ap.add_argument("--score", default="ema", choices=["ema", "accum", "random"],
                     help="ranking source: attention-mass EMA, accumulated attention, or a static random draw")
     return ap.parse_args()
@@ -107,6 +109,39 @@ def attn_traffic(w):
         return per_seg * w["L"] * w["B"] * w["Hkv"]
     except Exception:
         return None
+
+
+def paged_study(h, w, block_sizes=(16, 32, 64, 128)):
+    """Design study of a paged layout (the PagedAttention "partially dead
+    blocks" issue), from the kept positions of sampled segments after the run:
+    with tokens stored in position order in blocks of `bs` positions (as a
+    paged cache appends them) and eviction freeing only blocks left empty,
+    how many slots the retained blocks hold per live token, and how many of
+    those blocks are partially dead. The library's own layout is compacted
+    (one slot per live token)."""
+    import numpy as np
+    L, B, Hkv = w["L"], w["B"], w["Hkv"]
+    layers = sorted({0, L // 2, L - 1})
+    pos_sets = []
+    for l in layers:
+        for hh in range(Hkv):
+            ex = h.export_segment(l, 0, hh)
+            live = ex["pos_r"] >= 0
+            pos_sets.append(np.concatenate([ex["pos_c"].astype(np.int64), ex["pos_r"][live].astype(np.int64)]))
+    out = {"segments": f"layers {layers} x sequence 0 x {Hkv} KV heads", "live_tokens_mean":
+           float(np.mean([len(p) for p in pos_sets]))}
+    for bs in block_sizes:
+        slots = live = partial = blocks = 0
+        for p in pos_sets:
+            blk, cnt = np.unique(p // bs, return_counts=True)
+            newest = blk.max() if blk.size else -1
+            blocks += blk.size
+            slots += blk.size * bs
+            live += p.size
+            partial += int(((cnt < bs) & (blk != newest)).sum())   # the newest block is still filling
+        out[f"block_{bs}"] = {"slots_per_live_token": slots / max(1, live),
+                              "partially_dead_block_fraction": partial / max(1, blocks)}
+    return out
 
 
 def warm_library(w, dev):
@@ -504,6 +539,7 @@ def main():
     e2e_value = whole_job_rate(world, B, E, e2e_ms)
 
     stats = h.query()
+    study = paged_study(h, w) if args.paged_study else None
     full_cache = L * B * Hkv * (T + 1 + args.warmup + K + E) * 4 * D
     sw512 = L * B * Hkv * 512 * 4 * D
     _report_device_error(h, "the run")
@@ -543,6 +579,8 @@ def main():
             "kv_resident_bytes": {"conf_kv": stats["bytes_payload"], "full_fp16": full_cache, "sliding_window_512": sw512,
                                   "tokens_int8": stats["tokens_int8"], "tokens_fp16": stats["tokens_fp16"]},
         }
+        if study is not None:
+            line["paged_study"] = study
         print(json.dumps(line), flush=True)
     h.close()
     if world > 1:

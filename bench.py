@@ -49,6 +49,8 @@ def args_parse():
                     help="per-layer: one attention call per layer, as a model's layers run (eviction stays one call)")
     ap.add_argument("--compact", default="hole-fill", choices=["hole-fill", "stable"],
                     help="stable: order-preserving compaction instead of hole-fill")
+    ap.add_argument("--graph", action="store_true",
+                    help="also time the step replayed from a CUDA graph (the handle then runs single-stream)")
     ap.add_argument("--paged-study", action="store_true",
                     help="after the run, the dead space a position-ordered paged layout would hold")
     ap.add_argument("--score", default="ema", choices=["ema", "accum", "random"],
@@ -65,6 +67,7 @@ def workload(args):
     w["calls"] = getattr(args, "calls", "all-layers")
     w["compact"] = getattr(args, "compact", "hole-fill")
     w["score"] = getattr(args, "score", "ema")
+    w["graph"] = bool(getattr(args, "graph", False))
     return w
 
 
@@ -76,6 +79,8 @@ def workload_name(w):
         name += ", one attention call per layer"
     if w.get("compact", "hole-fill") != "hole-fill":
         name += ", stable compaction"
+    if w.get("graph"):
+        name += ", single-stream handle (graph-capturable)"
     if w.get("score", "ema") != "ema":
         name += {"accum": ", accumulated-attention ranking", "random": ", random ranking"}[w["score"]]
     return name if (w["L"], w["T"]) == (FULL["L"], FULL["T"]) else "reduced case (profiling): " + name
@@ -363,7 +368,8 @@ def main():
     h = ConfKV(L, Hkv, Hq, D, max_batch=B, max_prefill=T, n_low=w["n_low"], n_high=w["n_high"], tau=w["tau"],
                alpha=w["alpha"], ema_decay=w["beta"], protect_last=w["P"], fp16_window=w["W"],
                compact=1 if w["compact"] == "stable" else 0,
-               score_source={"ema": 0, "accum": 1, "random": 2}[w["score"]], seed=7)
+               score_source={"ema": 0, "accum": 1, "random": 2}[w["score"]], seed=7,
+               single_stream=1 if args.graph else 0)
     gen = synth.generator(1000 + rank, dev)
     for l in range(L):
         k, v = synth.prefill_kv(B, Hkv, T, D, gen, dev)
@@ -538,6 +544,42 @@ def main():
     e2e_ms = max_over_ranks(e2e_ms, dev)
     e2e_value = whole_job_rate(world, B, E, e2e_ms)
 
+    # ---- optional: the same step replayed from a CUDA graph ----
+    graph_line = None
+    if args.graph:
+        sq, skn, svn, slg = (x.clone() for x in pool[0])
+        gout = torch.empty_like(out)
+        gc = torch.empty_like(c_out)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            attn_call(sq, skn, svn, gout)
+            h.confidence(slg, gc)
+            h.evict_compact(ALL_LAYERS)
+
+        def replay(i):
+            q, kn, vn, lg = pool[i % POOL]
+            sq.copy_(q)
+            skn.copy_(kn)
+            svn.copy_(vn)
+            slg.copy_(lg)
+            graph.replay()
+
+        for i in range(3):
+            replay(i)
+        torch.cuda.synchronize()
+        Kg = min(K, 1000)
+        e0.record(stream)
+        for i in range(Kg):
+            replay(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        _report_device_error(h, "graph replays")
+        g_ms = max_over_ranks(e0.elapsed_time(e1), dev)
+        graph_line = {"ms_per_step": g_ms / Kg, "value": whole_job_rate(world, B, Kg, g_ms), "steps": Kg,
+                      "note": "one captured step (inputs copied into its static buffers each step, inside the timing)"}
+        del graph
+
     stats = h.query()
     study = paged_study(h, w) if args.paged_study else None
     full_cache = L * B * Hkv * (T + 1 + args.warmup + K + E) * 4 * D
@@ -581,6 +623,8 @@ def main():
         }
         if study is not None:
             line["paged_study"] = study
+        if graph_line is not None:
+            line["graph"] = graph_line
         print(json.dumps(line), flush=True)
     h.close()
     if world > 1:

@@ -49,7 +49,7 @@ class Params(ctypes.Structure):
                 ("pyramidal", ctypes.c_int32), ("gate", ctypes.c_int32),
                 ("int8_enable", ctypes.c_int32), ("compact", ctypes.c_int32),
                 ("max_batch", ctypes.c_int32), ("max_prefill", ctypes.c_int32),
-                ("score_source", ctypes.c_int32), ("seed", ctypes.c_uint32)]
+                ("score_source", ctypes.c_int32), ("seed", ctypes.c_uint32), ("single_stream", ctypes.c_int32)]
 
 
 class Stats(ctypes.Structure):

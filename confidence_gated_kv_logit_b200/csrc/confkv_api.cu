@@ -363,11 +363,14 @@ confkv_status confkv_create(int32_t layers, int32_t kv_heads, int32_t q_heads, i
   int prio_least = 0, prio_greatest = 0;
   if (cudaDeviceGetStreamPriorityRange(&prio_least, &prio_greatest) != cudaSuccess) prio_greatest = 0;
   h->layer_ev.assign(layers, -1);
-  h->ema_ev.assign(2 * (size_t)layers + 2, nullptr);
-  bool ev_ok = cudaStreamCreateWithPriority(&h->ema_stream, cudaStreamNonBlocking, prio_greatest) == cudaSuccess &&
-               cudaEventCreateWithFlags(&h->attn_done, cudaEventDisableTiming) == cudaSuccess;
-  for (cudaEvent_t& ev : h->ema_ev)
-    ev_ok = ev_ok && cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) == cudaSuccess;
+  bool ev_ok = true;
+  if (!p.single_stream) {   // single stream: no side stream and no events (capturable calls)
+    h->ema_ev.assign(2 * (size_t)layers + 2, nullptr);
+    ev_ok = cudaStreamCreateWithPriority(&h->ema_stream, cudaStreamNonBlocking, prio_greatest) == cudaSuccess &&
+            cudaEventCreateWithFlags(&h->attn_done, cudaEventDisableTiming) == cudaSuccess;
+    for (cudaEvent_t& ev : h->ema_ev)
+      ev_ok = ev_ok && cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) == cudaSuccess;
+  }
   if (!ev_ok) {
     if (h->ema_stream) cudaStreamDestroy(h->ema_stream);
     if (h->attn_done) cudaEventDestroy(h->attn_done);
@@ -388,6 +391,7 @@ confkv_status confkv_create(int32_t layers, int32_t kv_heads, int32_t q_heads, i
 
 // Make `st` wait for the last EMA pass over every layer of r.
 static cudaError_t wait_ema(confkv_handle* h, const confkv::Range& r, cudaStream_t st) {
+  if (h->ema_stream == nullptr) return cudaSuccess;   // single stream: stream order suffices
   int last = -1;
   for (int l = r.l0; l < r.l0 + r.nl; ++l) {
     const int k = h->layer_ev[l];
@@ -533,14 +537,14 @@ confkv_status confkv_decode_attn(confkv_handle* h, int32_t layer, const void* q,
   a.ema_stream = h->ema_stream;
   a.attn_done = h->attn_done;
   const int ev = h->ev_next;
-  a.ema_done = h->ema_ev[ev];
+  a.ema_done = h->ema_stream != nullptr ? h->ema_ev[ev] : nullptr;
   // the previous EMA pass over these layers must be done before this step
   // rewrites their scores and EMA values
   if (wait_ema(h, r, static_cast<cudaStream_t>(stream)) != cudaSuccess) return CONFKV_ERR_CUDA;
   cudaError_t e =
       confkv::launch_decode_attn(h->c, h->pol, a, static_cast<cudaStream_t>(stream), &h->launches, h->prof_ptr());
   if (e != cudaSuccess) return cuda_status(e);
-  if (h->pol.mode == 0) {   // an EMA pass ran (and recorded ema_ev[ev]) for these layers
+  if (h->pol.mode == 0 && h->ema_stream != nullptr) {   // an EMA pass ran on the side stream and recorded ema_ev[ev]
     for (int l = r.l0; l < r.l0 + r.nl; ++l) h->layer_ev[l] = ev;
     h->ev_next = (ev + 1) % (int)h->ema_ev.size();
   }

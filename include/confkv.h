@@ -104,6 +104,11 @@ typedef struct {
   int32_t max_prefill;   /* longest prompt confkv_prefill accepts (tokens) */
   int32_t score_source;  /* CONFKV_SCORE_EMA, CONFKV_SCORE_ACCUM or CONFKV_SCORE_RANDOM (confidence mode) */
   uint32_t seed;         /* CONFKV_SCORE_RANDOM: seed of the per-token draws */
+  int32_t single_stream; /* nonzero: every kernel of a call runs on the caller's stream (the EMA pass
+                            too, instead of on the handle's side stream joined by events), so that a
+                            caller can capture a whole decode step in a CUDA graph. Launch
+                            configurations are then fixed at capture time, and the handle's host-side
+                            length bounds are not advanced by replays */
 } confkv_params;
 
 typedef struct {

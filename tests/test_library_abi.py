@@ -50,6 +50,15 @@ def test_default_params(lib):
     assert (p.n_low, p.n_high, p.protect_last, p.fp16_window) == (256, 512, 64, 128)
     assert abs(p.tau - 0.6) < 1e-7 and abs(p.alpha - 0.5) < 1e-7 and abs(p.ema_decay - 0.9) < 1e-7
     assert lib.confkv_default_params(None) == 1
+    assert (p.score_source, p.seed, p.single_stream) == (binding.SCORE_EMA, 0, 0)
+
+
+def test_param_struct_matches_the_header():
+    # every field of confkv_params in include/confkv.h, in order, is in the ctypes mirror
+    text = open(os.path.join(ROOT, "include", "confkv.h")).read()
+    body = text[text.index("typedef struct {", text.index("CONFKV_ALL_LAYERS")):text.index("} confkv_params;")]
+    fields = re.findall(r"^\s*(?:int32_t|uint32_t|float)\s+(\w+);", body, re.M)
+    assert fields == [name for name, _ in binding.Params._fields_]
 
 
 @pytest.mark.parametrize("shape,kw", [
@@ -61,6 +70,7 @@ def test_default_params(lib):
     ((1, 4, 4, 64), {"fp16_window": 0}),
     ((1, 4, 4, 64), {"mode": 1, "fixed_budget": 10, "n_sink": 8, "protect_last": 8}),
     ((1, 4, 4, 64), {"gate": 7}),
+    ((1, 4, 4, 64), {"score_source": 3}),
 ])
 def test_create_rejects_bad_arguments_before_touching_the_device(lib, shape, kw):
     p = binding.default_params()

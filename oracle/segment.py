@@ -30,6 +30,13 @@ Readings where the pages are silent (each restated where it is used):
   than B = s + w + k tokens between steps, so prefill applies the selection
   (sinks, the last w, the top k by priority) as it ingests. INT8 is off by
   default in this mode since the KVpop summary says nothing of quantisation.
+
+Pins: tests/test_oracle_segment.py (decode-loop invariants on seeded runs)
+and tests/test_oracle_readings.py, whose expected kept sets are written out
+by hand for a budget below P + s (sinks and the last P stay), for eviction
+before the first confidence call and after a new batch (the larger budget,
+per layer under the pyramid), and for a skipped eviction (the next append
+converts position t + 1 - W); planted mistakes in copies of each fail them.
 """
 from __future__ import annotations
 

@@ -3,6 +3,7 @@ host-side argument validation works without a GPU (CPU only)."""
 import ctypes
 import os
 import re
+import subprocess
 
 import pytest
 
@@ -101,3 +102,39 @@ def _load_missing(tmp_path):
         binding.load_library(str(tmp_path / "missing.so"))
     finally:
         binding._LIB = saved
+
+
+def test_plain_c_caller_sees_the_binding_layout(lib, tmp_path):
+    """Compile tests/abi_check.c against include/confkv.h with gcc, link it to
+    the library, run it, and compare the struct layout it prints (offsetof,
+    sizeof) with the ctypes mirrors; it also calls the entry points that need
+    no device and checks their results itself."""
+    exe = tmp_path / "abi_check"
+    libdir = os.path.dirname(binding.LIB_PATH)
+    cc = subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                         os.path.join(ROOT, "tests", "abi_check.c"), "-o", str(exe), binding.LIB_PATH,
+                         f"-Wl,-rpath,{libdir}"], capture_output=True, text=True)
+    assert cc.returncode == 0, cc.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert run.returncode == 0, (run.returncode, run.stdout, run.stderr)
+    lines = run.stdout.splitlines()
+    assert lines[-1] == "ok"
+    layout = {}
+    for ln in lines:
+        parts = ln.split()
+        if ln.startswith("sizeof "):
+            layout[parts[1]] = int(parts[2])
+        elif "." in parts[0] and parts[0].startswith("confkv_"):
+            layout[parts[0]] = (int(parts[1]), int(parts[2]))
+    for struct, mirror in (("confkv_params", binding.Params), ("confkv_stats", binding.Stats),
+                           ("confkv_profile", binding.Profile)):
+        assert layout[struct] == ctypes.sizeof(mirror), struct
+        for name, _ in mirror._fields_:
+            f = getattr(mirror, name)
+            assert layout[f"{struct}.{name}"] == (f.offset, f.size), (struct, name)
+    d = next(ln for ln in lines if ln.startswith("default "))
+    assert d.split()[1:6] == ["256", "512", "64", "128", "4096"]
+    statuses = [ln for ln in lines if ln.startswith("status ")]
+    assert len(statuses) == 8
+    for code, ln in enumerate(statuses):
+        assert ln.split(" ", 2)[2] == lib.confkv_status_string(code).decode()

@@ -263,8 +263,11 @@ CONFKV_API confkv_status confkv_profile_read(confkv_handle* h, confkv_profile* o
  *  - batch may be at most 256 and vocab at most 262144; larger sizes return
  *    CONFKV_ERR_CAPACITY before anything runs;
  *  - the first call on a device looks up the array's device address (a
- *    host-side step, no allocation); make that first call before any stream
- *    capture;
+ *    host-side step, no allocation) and keeps it for the life of the process;
+ *    make that first call before any stream capture. A device reset
+ *    (cudaDeviceReset, or a reset of the primary context) reloads the library
+ *    on that device and leaves the kept address stale: do not call this entry
+ *    point on a device after resetting it;
  *  - every call shares the one array: calls that overlap on the GPU (on two
  *    streams, or from two threads) race and give wrong results. Serialise them.
  * It calls no cudaMalloc, cudaFree or allocating routine. A row with a NaN or

@@ -309,13 +309,15 @@ class OracleCache:
                 lse[b, g0:g0 + self.G] = s
         return out, lse
 
-    def confidence(self, logits, override=None):
+    def confidence(self, logits, override=None, rows=None):
         """Per-sequence confidence and budgets. ``override`` maps a sequence to a
-        budget to use instead of the gate's (near-tie steps)."""
+        budget to use instead of the gate's (near-tie steps). ``rows`` limits
+        the work to those sequences (the others keep their budgets and get
+        c = NaN), for runs that simulate only a few sequences."""
         logits = np.asarray(logits)
         B = logits.shape[0]
-        c = np.empty(B)
-        for b in range(B):
+        c = np.full(B, np.nan)
+        for b in (range(B) if rows is None else rows):
             c[b] = confidence(logits[b])["c"]
             N = choose_budget(c[b], self.p.tau, self.p.n_low, self.p.n_high, self.p.gate)
             if override is not None and b in override:

@@ -32,9 +32,12 @@ class Pair:
     """The library and the oracle, fed identical inputs."""
 
     def __init__(self, L, Hkv, Hq, D, B, params: Params, max_prefill: int, track=None, stable=False,
-                 seed=0):
+                 seed=0, gen_chunk=None):
         _build.build()
         self.L, self.Hkv, self.Hq, self.D, self.B, self.p = L, Hkv, Hq, D, B, params
+        # prompt K/V are drawn this many sequences at a time (bounds the fp32
+        # temporaries of the generator at the largest shapes)
+        self.gen_chunk = gen_chunk or B
         self.gpu = ConfKV(L, Hkv, Hq, D, **c_params(params, B, max_prefill, stable))
         self.orc = OracleCache(L, Hkv, Hq, D, params, track)
         self.track = track
@@ -52,7 +55,14 @@ class Pair:
         T = T or max(max(lens), 1)
         fixed = self.p.mode == "fixed"
         for l in range(self.L):
-            k, v = synth.prefill_kv(self.B, self.Hkv, T, self.D, self.gen, self.dev)
+            if self.gen_chunk >= self.B:
+                k, v = synth.prefill_kv(self.B, self.Hkv, T, self.D, self.gen, self.dev)
+            else:
+                k = torch.empty((self.B, self.Hkv, T, self.D), dtype=torch.float16, device=self.dev)
+                v = torch.empty_like(k)
+                for b0 in range(0, self.B, self.gen_chunk):
+                    b1 = min(self.B, b0 + self.gen_chunk)
+                    k[b0:b1], v[b0:b1] = synth.prefill_kv(b1 - b0, self.Hkv, T, self.D, self.gen, self.dev)
             pr = synth.priorities((self.B, self.Hkv, T), self.gen, self.dev) if fixed else None
             self.gpu.prefill(k, v, lens, layer=l, priority=pr)
             keys = [key for key in self.segments() if key[0] == l]
@@ -82,43 +92,69 @@ class Pair:
     def gpu_evict(self):
         self.gpu.evict_compact()
 
+    def tracked_layers(self):
+        return sorted({l for (l, _, _) in self.segments()})
+
     def attn(self, q, kn, vn, pn):
+        """One attention step on both sides. Only the tracked layers are copied
+        to the host and simulated: returns (GPU out, GPU lse, oracle out, oracle
+        lse), each a dict from a tracked layer to its [B, Hq, ...] array."""
         out = torch.empty((self.L, self.B, self.Hq, self.D), device=self.dev)
         lse = torch.empty((self.L, self.B, self.Hq), device=self.dev)
         self.gpu_decode_attn(q, kn, vn, out, pn, lse)
-        qh, kh, vh = q.cpu().numpy(), kn.cpu().numpy(), vn.cpu().numpy()
-        ph = None if pn is None else pn.cpu().numpy()
-        o_out = np.zeros((self.L, self.B, self.Hq, self.D))
-        o_lse = np.zeros((self.L, self.B, self.Hq))
-        for l in range(self.L):
-            o, s = self.orc.decode_attn(l, qh[l], kh[l], vh[l], None if ph is None else ph[l])
-            o_out[l], o_lse[l] = o, s
+        ls = self.tracked_layers()
+        idx = torch.tensor(ls, device=self.dev)
+        qh, kh, vh = (x.index_select(0, idx).cpu().numpy() for x in (q, kn, vn))
+        ph = None if pn is None else pn.index_select(0, idx).cpu().numpy()
+        o_out, o_lse = {}, {}
+        for i, l in enumerate(ls):
+            o_out[l], o_lse[l] = self.orc.decode_attn(l, qh[i], kh[i], vh[i], None if ph is None else ph[i])
         torch.cuda.synchronize()
-        return out.cpu().numpy(), lse.cpu().numpy(), o_out, o_lse
+        go = out.index_select(0, idx).cpu().numpy()
+        gl = lse.index_select(0, idx).cpu().numpy()
+        g_out = {l: go[i] for i, l in enumerate(ls)}
+        g_lse = {l: gl[i] for i, l in enumerate(ls)}
+        return g_out, g_lse, o_out, o_lse
 
-    def confidence(self, logits):
+    def tracked_seqs(self):
+        return sorted({b for (_, b, _) in self.segments()})
+
+    def confidence(self, logits, all_rows=True):
+        """Confidence on both sides. With all_rows False the oracle evaluates
+        only the tracked sequences (the other rows of c_o are NaN and their
+        budgets are not compared)."""
         c = torch.empty(self.B, device=self.dev)
         bud = torch.empty((self.B, self.L), device=self.dev, dtype=torch.int32)
         self.gpu.confidence(logits, c, bud)
         torch.cuda.synchronize()
         c_g, bud_g = c.cpu().numpy(), bud.cpu().numpy()
         from oracle import confidence as oconf
-        lh = logits.cpu().numpy()
+        rows = list(range(self.B)) if all_rows else self.tracked_seqs()
+        lh = logits.index_select(0, torch.tensor(rows, device=self.dev)).cpu().numpy()
+        full = np.zeros((self.B, lh.shape[1]), np.float32)
+        full[rows] = lh
         override = {}
-        for b in range(self.B):
-            co = oconf(lh[b])["c"]
+        for i, b in enumerate(rows):
+            co = oconf(lh[i])["c"]
             if abs(co - self.p.tau) < NEAR_TIE:
                 # the GPU's chosen N, read back from its layer-0 budget (2N under the pyramid)
                 override[b] = int(bud_g[b, 0]) // (2 if (self.p.pyramidal and self.L > 1) else 1)
-        c_o, bud_o = self.orc.confidence(lh, override=override)
-        return c_g, bud_g, c_o, bud_o, override
+        c_o, bud_o = self.orc.confidence(full, override=override, rows=rows)
+        return c_g[rows], bud_g[rows], c_o[rows], bud_o[rows], override
 
     def gpu_segment(self, l, b, h):
         return logical_segment(self.gpu.export_segment(l, b, h))
 
+    def exact_scores(self):
+        """Whether both sides hold the same score sources bit for bit without
+        synchronisation (static priorities or static draws)."""
+        return self.p.mode == "fixed" or self.p.score_source == "random"
+
     def sync_scores_from_gpu(self):
         """Step-synchronised mode: give the oracle the GPU's EMA values (matched by
         position) so that selection can be compared bit for bit."""
+        if self.exact_scores():
+            return
         for key in self.segments():
             g = self.gpu_segment(*key)
             o = self.orc.segment(*key)
@@ -144,37 +180,50 @@ def assert_segment_equal(g: dict, o, key, exact_scores=True):
         np.testing.assert_allclose(g["score_src"], o.score_src, rtol=RTOL_EMA, atol=ATOL_EMA, err_msg=str(key))
 
 
-def run_synced(pair: Pair, lens, steps, V, T=None, check_every=1):
+def run_synced(pair: Pair, lens, steps, V, T=None, check_every=1, schedule=None, all_rows_every=None):
     """Step-synchronised parity run: per step, attention (tolerance), EMA
     (tolerance), confidence and budgets, then -- with the oracle given the
-    GPU's EMA -- the kept set, compaction and INT8 codes bit for bit."""
+    GPU's EMA -- the kept set, compaction and INT8 codes bit for bit.
+
+    ``schedule`` lists, per step, which calls run: "a" attention, "c"
+    confidence, "e" eviction (default "ace" every step; fixed mode has no
+    confidence). Segments are compared every ``check_every`` steps and at the
+    last step. The oracle's confidence covers every row every
+    ``all_rows_every`` steps (default: every step), otherwise only the tracked
+    sequences."""
+    if schedule is None:
+        schedule = ["ace"] * steps
+    steps = len(schedule)
+    all_rows_every = all_rows_every or 1
     pair.prefill(lens, T)
     for key in pair.segments():
         assert_segment_equal(pair.gpu_segment(*key), pair.orc.segment(*key), key)
     worst = 0.0
-    for step in range(steps):
+    for step, calls in enumerate(schedule):
         check = (step % check_every == 0) or step == steps - 1
         q, kn, vn, pn, logits = pair.step_inputs(V)
-        out_g, lse_g, out_o, lse_o = pair.attn(q, kn, vn, pn)
-        for (l, b, h) in pair.segments():
-            sl = slice(h * pair.orc.G, (h + 1) * pair.orc.G)
-            err = float(np.abs(out_g[l, b, sl] - out_o[l, b, sl]).max())
-            worst = max(worst, err)
-            assert err <= ATOL_OUT, (step, l, b, h, err)
-            assert np.abs(lse_g[l, b, sl] - lse_o[l, b, sl]).max() <= ATOL_LSE
-            if check:
-                assert_segment_equal(pair.gpu_segment(l, b, h), pair.orc.segment(l, b, h), (step, l, b, h),
-                                     exact_scores=pair.p.mode == "fixed" or pair.p.score_source == "random")
-        if logits is not None:
-            c_g, bud_g, c_o, bud_o, override = pair.confidence(logits)
+        if "a" in calls:
+            out_g, lse_g, out_o, lse_o = pair.attn(q, kn, vn, pn)
+            for (l, b, h) in pair.segments():
+                sl = slice(h * pair.orc.G, (h + 1) * pair.orc.G)
+                err = float(np.abs(out_g[l][b, sl] - out_o[l][b, sl]).max())
+                worst = max(worst, err)
+                assert err <= ATOL_OUT, (step, l, b, h, err)
+                assert np.abs(lse_g[l][b, sl] - lse_o[l][b, sl]).max() <= ATOL_LSE
+                if check:
+                    assert_segment_equal(pair.gpu_segment(l, b, h), pair.orc.segment(l, b, h), (step, l, b, h),
+                                         exact_scores=pair.exact_scores())
+        if "c" in calls and logits is not None:
+            c_g, bud_g, c_o, bud_o, override = pair.confidence(logits, all_rows=step % all_rows_every == 0)
             assert np.abs(c_g - c_o).max() <= ATOL_C, (c_g, c_o)
             assert np.array_equal(bud_g, bud_o), (step, bud_g, bud_o, override)
-        pair.sync_scores_from_gpu()
-        pair.gpu_evict()
-        for l in range(pair.L):
-            pair.orc.evict_compact(l)
-        if check:
-            for key in pair.segments():
-                assert_segment_equal(pair.gpu_segment(*key), pair.orc.segment(*key), (step,) + key)
+        if "e" in calls:
+            pair.sync_scores_from_gpu()
+            pair.gpu_evict()
+            for l in range(pair.L):
+                pair.orc.evict_compact(l)
+            if check:
+                for key in pair.segments():
+                    assert_segment_equal(pair.gpu_segment(*key), pair.orc.segment(*key), (step,) + key)
     assert pair.gpu.last_error() == 0
     return worst

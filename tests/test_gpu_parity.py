@@ -168,3 +168,50 @@ def test_confidence_parity_vocab_sizes(V, B):
         if trial == 2:
             assert abs(c[0].item() - (0.15 + 0.3 / V)) <= 1e-6
     h.close()
+
+
+# ---- the three decode-loop readings pinned by tests/test_oracle_readings.py ----
+
+def test_budget_below_protected_count_synced():
+    # budget n_low = 10 below P + s = 20: the effective budget is P + s, so a
+    # segment keeps exactly its sinks and its last P tokens; with n_high = 40
+    # the gate moves between the clamp and a real budget
+    p = Params(n_low=10, n_high=40, protect_last=16, n_sink=4, fp16_window=8)
+    pair = Pair(2, 2, 8, 128, 2, p, max_prefill=300, seed=21)
+    run_synced(pair, [300, 90], 12, 2048)
+    p = Params(n_low=10, n_high=10, protect_last=16, n_sink=4, fp16_window=8, alpha=0.5)
+    pair = Pair(1, 2, 8, 128, 2, p, max_prefill=300, seed=22)
+    run_synced(pair, [300, 21], 5, 2048)
+    for b, T in ((0, 300), (1, 21)):
+        t = T + 4
+        for h in range(2):
+            got = pair.gpu_segment(0, b, h)["pos"].tolist()
+            assert got == list(range(4)) + list(range(t - 15, t + 1)), (b, h, got)
+
+
+def test_budget_before_first_confidence_call_synced():
+    # eviction before any confidence call uses the larger budget, per layer
+    # under the pyramid: floor(160 (8 - 3l) / 4) = 320, 200, 80 over 3 layers;
+    # recency-only ranking keeps the most recent tokens
+    p = Params(n_low=64, n_high=160, protect_last=16, fp16_window=32, pyramidal=True, alpha=0.0)
+    pair = Pair(3, 2, 8, 128, 2, p, max_prefill=400, seed=23)
+    run_synced(pair, [400, 400], 3, 2048, schedule=["ae", "ace", "ace"])
+    p2 = Params(n_low=64, n_high=160, protect_last=16, fp16_window=32, pyramidal=True, alpha=0.0)
+    pair = Pair(3, 2, 8, 128, 2, p2, max_prefill=400, seed=24)
+    run_synced(pair, [400, 400], 1, 2048, schedule=["ae"])
+    for l, eff in enumerate((320, 200, 80)):
+        for b in range(2):
+            for h in range(2):
+                assert pair.gpu_segment(l, b, h)["pos"].tolist() == list(range(401 - eff, 401)), (l, b, h)
+
+
+@pytest.mark.parametrize("stable", [False, True], ids=["hole_fill", "stable"])
+def test_skipped_eviction_converts_on_append_synced(stable):
+    # a caller that skips eviction: the next append converts the token that
+    # has left the FP16 window (the oracle converts t + 1 - W on append too)
+    p = Params(n_low=100, n_high=200, protect_last=16, fp16_window=32, n_sink=2)
+    pair = Pair(2, 2, 8, 128, 2, p, max_prefill=400, seed=25, stable=stable)
+    schedule = ["a", "a", "ace", "ac", "a", "ace", "ace", "a", "ace"]
+    run_synced(pair, [400, 130], 0, 2048, schedule=schedule)
+    st = pair.gpu.query()
+    assert st["requant_rows"] > 0

@@ -19,7 +19,8 @@ pytestmark = pytest.mark.gpu
 ATOL_C = 1e-5   # the confidence tolerance used by every parity test
 
 
-@pytest.mark.parametrize("B,V,L,pyramidal,gate", [(16, 128256, 32, 0, 0), (3, 50257, 12, 1, 1), (256, 1024, 4, 1, 0)])
+@pytest.mark.parametrize("B,V,L,pyramidal,gate", [(16, 128256, 32, 0, 0), (3, 50257, 12, 1, 1), (256, 1024, 4, 1, 0),
+                                                   (2, 262144, 8, 0, 0)])   # the largest vocabulary it accepts
 def test_noalloc_matches_handle_on_two_calls(B, V, L, pyramidal, gate):
     _build.build()
     dev = torch.device("cuda")
@@ -52,4 +53,10 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     b = torch.empty((257, 1), dtype=torch.int32, device=dev)
     with pytest.raises(binding.ConfKVError) as e:
         binding.confidence_noalloc(torch.zeros((257, 16), device=dev), 1, c, b)
+    assert e.value.status == 2
+    # one token past the largest vocabulary whose per-row partials fit the array
+    c1 = torch.empty(1, device=dev)
+    b1 = torch.empty((1, 1), dtype=torch.int32, device=dev)
+    with pytest.raises(binding.ConfKVError) as e:
+        binding.confidence_noalloc(torch.zeros((1, 262145), device=dev), 1, c1, b1)
     assert e.value.status == 2

@@ -1,17 +1,34 @@
 #!/usr/bin/env python
 """Decode-step benchmark of the CONF-KV B200 library.
 
-Workload (one "step" = one decode step of the whole hot path for every layer,
-sequence and KV head): Llama-3-8B shape, 32 layers, 32 query / 8 KV heads,
-head_dim 128, batch 16, every sequence prefilled to 32768 tokens (fp16
-N(0,1), 1% of keys x4), vocab 128256 with bursty logits, N_low 1024 /
-N_high 2048, P 128, W 256, tau 0.6, alpha 0.5, EMA decay 0.9. A step is
-  decode_attn(all layers) -> confidence(logits) -> evict_compact(all layers).
-The first step after prefill evicts ~31K tokens per segment and is timed on
-its own ("step1_ms"); the timed region covers steady-state steps after it.
+One "step" is one decode step of the whole hot path for every layer, sequence
+and KV head of the workload:
+  decode_attn(all layers) -> confidence(logits) -> evict_compact(all layers)
+(fixed-budget mode has no confidence call). Five workloads, one per
+configuration of the method's evaluation shapes (`--config`, default 3):
+
+  1  tiny: 1 layer, 4 MHA heads, D64, batch 1, 600-token prompt, 32 steps,
+     vocab 1024, N 256/512, P64, W128
+  2  GPT-2-small shape: 12 layers, 12 MHA heads, D64, batch 1, 128-token
+     prompt, 4096 steps, vocab 50257, N 256/512, P64, W128; the fixed
+     512-token sliding window (alpha 0, P 512, INT8 off) is timed beside it
+  3  Llama-3-8B shape (the headline): 32 layers, 32q/8kv, D128, batch 16,
+     32768-token prompts, vocab 128256, N 1024/2048, P128, W256. The first
+     step after prefill evicts ~31K tokens per segment and is timed on its
+     own; the timed region covers steady-state steps after it
+  4  Qwen-32B shape with pyramidal budgets: 64 layers, 40q/8kv, D128,
+     batch 32, 512-token prompt, 4096 steps, vocab 152064, N 512/1024,
+     P128, W256
+  5  fixed sink + window + top-k budget at a Qwen3-8B-like shape: 36
+     layers, 32q/8kv, D128, B = 2048 = 4 sinks + 512 window + 1532 top-k by
+     static priority, INT8 off; batch {1, 8, 64} x context {4K, 32K, 128K},
+     each point's prefill (select + gather) and decode step timed apart
+
+tau 0.6, alpha 0.5, EMA decay 0.9 throughout. Inputs are synthetic and seeded
+(fp16 N(0,1) q/k/v with 1% of keys x4, bursty logits, U(0,1) priorities).
 
 Prints one JSON line. `--impl reference` times the CPU oracle on the same
-metric instead (rank 0 only).
+workload and metric instead (rank 0 only).
 """
 from __future__ import annotations
 
@@ -29,17 +46,37 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "decode tok/s at Llama-8B shape (attn+evict)"
-FULL = dict(L=32, Hq=32, Hkv=8, D=128, B=16, T=32768, V=128256, n_low=1024, n_high=2048, P=128, W=256,
-            tau=0.6, alpha=0.5, beta=0.9)
-POOL = 48   # distinct pre-generated step inputs, reused cyclically (1.4 GB/step working set >> L2)
+POLICY = dict(tau=0.6, alpha=0.5, beta=0.9)
+CONFIGS = {
+    1: dict(config=1, shape="tiny", L=1, Hq=4, Hkv=4, D=64, B=1, T=600, V=1024, n_low=256, n_high=512, P=64,
+            W=128, run_steps=32, **POLICY),
+    2: dict(config=2, shape="gpt2-small-shape", L=12, Hq=12, Hkv=12, D=64, B=1, T=128, V=50257, n_low=256,
+            n_high=512, P=64, W=128, run_steps=4096, **POLICY),
+    3: dict(config=3, shape="llama3-8b-shape", L=32, Hq=32, Hkv=8, D=128, B=16, T=32768, V=128256, n_low=1024,
+            n_high=2048, P=128, W=256, run_steps=256, **POLICY),
+    4: dict(config=4, shape="qwen-32b-shape pyramid", L=64, Hq=40, Hkv=8, D=128, B=32, T=512, V=152064,
+            n_low=512, n_high=1024, P=128, W=256, run_steps=4096, pyramidal=True, **POLICY),
+    5: dict(config=5, shape="qwen3-8b-like fixed sink+window+top-k", L=36, Hq=32, Hkv=8, D=128, B=8, T=32768,
+            V=0, fixed=2048, sinks=4, P=512, W=0, run_steps=256, mode="fixed", **POLICY),
+}
+FULL = CONFIGS[3]
+SWEEP5 = [(b, c) for b in (1, 8, 64) for c in (4096, 32768, 131072)]
+POOL = 48   # distinct pre-generated step inputs, reused cyclically
 
 
-def args_parse():
+def args_parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: 3000 steady steps for config 3, else the rest of the "
+                         "configuration's stated run after the warm-up)")
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--config", type=int, default=3, choices=sorted(CONFIGS))
+    ap.add_argument("--batch", type=int, default=None, help="config 5: one sweep point's batch (with --ctx)")
+    ap.add_argument("--ctx", type=int, default=None, help="config 5: one sweep point's context (with --batch)")
+    ap.add_argument("--gate", default="prose", choices=["prose", "literal"],
+                    help="budget gate polarity: prose (confident -> N_low) or literal (confident -> N_high)")
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--layers", type=int, default=None, help="smaller case for profiling captures")
     ap.add_argument("--prefill", type=int, default=None, help="smaller case for profiling captures")
@@ -52,29 +89,47 @@ def args_parse():
     ap.add_argument("--graph", action="store_true",
                     help="also time the step replayed from a CUDA graph (the handle then runs single-stream)")
     ap.add_argument("--paged-study", action="store_true",
-                    help="after the run, the dead space a position-ordered paged layout would hold")
+                    help="after the run, the dead space and block-compaction traffic of a paged layout")
     ap.add_argument("--score", default="ema", choices=["ema", "accum", "random"],
                     help="ranking source: attention-mass EMA, accumulated attention, or a static random draw")
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
-def workload(args):
-    w = dict(FULL)
-    if args.layers:
+def workload(args, batch=None, ctx=None):
+    """The workload dict of a configuration with the command line's variants."""
+    w = dict(CONFIGS[getattr(args, "config", 3) or 3])
+    w.setdefault("mode", "conf")
+    w.setdefault("pyramidal", False)
+    if w["mode"] == "fixed":
+        w["B"] = batch or getattr(args, "batch", None) or w["B"]
+        w["T"] = ctx or getattr(args, "ctx", None) or w["T"]
+    if getattr(args, "layers", None):
         w["L"] = args.layers
-    if args.prefill:
+    if getattr(args, "prefill", None):
         w["T"] = args.prefill
     w["calls"] = getattr(args, "calls", "all-layers")
     w["compact"] = getattr(args, "compact", "hole-fill")
     w["score"] = getattr(args, "score", "ema")
     w["graph"] = bool(getattr(args, "graph", False))
+    w["gate"] = getattr(args, "gate", "prose") or "prose"
+    w["reduced"] = bool(getattr(args, "layers", None) or getattr(args, "prefill", None))
     return w
 
 
 def workload_name(w):
-    name = (f"llama3-8b-shape decode: {w['L']} layers, {w['Hq']}q/{w['Hkv']}kv heads, D{w['D']}, batch {w['B']}, "
-            f"prefill {w['T']}, vocab {w['V']}, N {w['n_low']}/{w['n_high']}, P{w['P']}, W{w['W']}, "
-            f"steady-state steps after the bulk first step")
+    if w.get("mode", "conf") == "fixed":
+        name = (f"{w['shape']}: {w['L']} layers, {w['Hq']}q/{w['Hkv']}kv heads, D{w['D']}, batch {w['B']}, "
+                f"context {w['T']}, B={w['fixed']} = {w['sinks']} sinks + {w['P']} window + "
+                f"{w['fixed'] - w['sinks'] - w['P']} top-k, INT8 off, decode steps after the prefill select")
+    else:
+        name = (f"{w['shape']} decode: {w['L']} layers, {w['Hq']}q/{w['Hkv']}kv heads, D{w['D']}, batch {w['B']}, "
+                f"prefill {w['T']}, vocab {w['V']}, N {w['n_low']}/{w['n_high']}, P{w['P']}, W{w['W']}")
+        name += (", steady-state steps after the bulk first step" if w["config"] == 3
+                 else f", the {w['run_steps']}-step run after the prompt")
+        if w.get("pyramidal"):
+            name += ", pyramidal budgets"
+        name += ", gate " + ("confident -> N_high (pseudo-code line)" if w.get("gate") == "literal"
+                             else "confident -> N_low (prose)")
     if w.get("calls", "all-layers") != "all-layers":
         name += ", one attention call per layer"
     if w.get("compact", "hole-fill") != "hole-fill":
@@ -83,7 +138,7 @@ def workload_name(w):
         name += ", single-stream handle (graph-capturable)"
     if w.get("score", "ema") != "ema":
         name += {"accum": ", accumulated-attention ranking", "random": ", random ranking"}[w["score"]]
-    return name if (w["L"], w["T"]) == (FULL["L"], FULL["T"]) else "reduced case (profiling): " + name
+    return "reduced case (profiling): " + name if w.get("reduced") else name
 
 
 def peaks():
@@ -95,11 +150,15 @@ def peaks():
         return 6650.0, "fallback"
 
 
-def attn_traffic(w):
-    """dram bytes per attention launch from the committed ncu summary, if the
-    kernel source has not changed since it was taken (else None)."""
+def attn_traffic(w, tokens_per_launch):
+    """DRAM bytes of one attention launch, from the committed ncu summary of a
+    reduced case of the same configuration, scaled by the attention tokens
+    (INT8 + FP16 token-rows) the launch processes; None when the kernel source
+    has changed since the capture or there is no capture for this shape."""
     src = os.path.join(ROOT, "confidence_gated_kv_logit_b200", "csrc", "attention.cu")
     path = os.path.join(ROOT, "profiles", "attention_llama8b_traffic.txt")
+    if w["config"] != 3:
+        return None
     try:
         sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
         kv = {}
@@ -109,23 +168,31 @@ def attn_traffic(w):
                 kv[k.strip()] = v.strip()
         if kv.get("attention_cu_sha256") != sha:
             return None
-        # scaled from the captured case by segments processed per launch
-        per_seg = float(kv["dram_bytes_per_segment"])
-        return per_seg * w["L"] * w["B"] * w["Hkv"]
+        per_tok = float(kv["dram_bytes"]) / float(kv["attn_tokens"])
+        return per_tok * tokens_per_launch
     except Exception:
         return None
 
 
-def paged_study(h, w, block_sizes=(16, 32, 64, 128)):
+def paged_study(h, w, block_sizes=(16, 32, 64, 128), history=None, thresholds=(0.25, 0.5)):
     """Design study of a paged layout (the PagedAttention "partially dead
-    blocks" issue), from the kept positions of sampled segments after the run:
-    with tokens stored in position order in blocks of `bs` positions (as a
-    paged cache appends them) and eviction freeing only blocks left empty,
-    how many slots the retained blocks hold per live token, and how many of
-    those blocks are partially dead. The library's own layout is compacted
-    (one slot per live token)."""
+    blocks" issue), from the kept positions of sampled segments.
+
+    Dead space: with tokens stored in position order in blocks of `bs`
+    positions (as a paged cache appends them) and eviction freeing only blocks
+    left empty, how many slots the retained blocks hold per live token, and
+    how many of them are partially dead. The library's own layout is
+    compacted (one slot per live token).
+
+    Block-granular compaction (with `history`, the kept positions of the same
+    segments over consecutive steps): a paged cache that rewrites a block
+    once its live count falls below `theta * bs` -- moving its live tokens to
+    the tail block -- holds fewer slots but moves rows. Replayed over the
+    history per block size and threshold: rows moved per segment-step, the
+    bytes that costs at the layout's row size, and the slots held per live
+    token at the end."""
     import numpy as np
-    L, B, Hkv = w["L"], w["B"], w["Hkv"]
+    L, Hkv = w["L"], w["Hkv"]
     layers = sorted({0, L // 2, L - 1})
     pos_sets = []
     for l in layers:
@@ -146,7 +213,69 @@ def paged_study(h, w, block_sizes=(16, 32, 64, 128)):
             partial += int(((cnt < bs) & (blk != newest)).sum())   # the newest block is still filling
         out[f"block_{bs}"] = {"slots_per_live_token": slots / max(1, live),
                               "partially_dead_block_fraction": partial / max(1, blocks)}
+    if history:
+        row_bytes = 2 * w["D"] + 16 if w.get("W", 0) else 4 * w["D"] + 8
+        out["block_compaction"] = block_compaction_study(history, block_sizes, thresholds, row_bytes)
     return out
+
+
+def block_compaction_study(history, block_sizes, thresholds, row_bytes):
+    """Replay of a block-granular compaction policy over kept-position
+    histories (one list of per-step position arrays per segment).
+
+    Model: a paged cache holds tokens in blocks of `bs` slots, filled in
+    arrival order; the newest block receives appended tokens. After each
+    step's eviction, every non-tail block whose live count is below
+    theta * bs is compacted: its live tokens are appended to the tail (moving
+    one row each, read and write), and the block is freed. Blocks left empty
+    are freed at no cost. Reported per (bs, theta): rows moved per
+    segment-step, bytes moved per segment-step (2 x row bytes per row), and
+    the slots held per live token averaged over the replay."""
+    import numpy as np
+    res = {}
+    for bs in block_sizes:
+        for theta in thresholds:
+            moved = steps = 0
+            slot_ratio = []
+            for seq in history:
+                block_of = {}                       # position -> block id
+                fill = {}                           # block id -> slots used (ever)
+                tail = -1
+                next_id = 0
+                prev = set()
+                for pos in seq:
+                    cur = set(int(x) for x in pos)
+                    for p in sorted(cur - prev):    # arrivals (the prompt, then one per step)
+                        if tail < 0 or fill[tail] >= bs:
+                            tail, next_id = next_id, next_id + 1
+                            fill[tail] = 0
+                        block_of[p] = tail
+                        fill[tail] += 1
+                    for p in prev - cur:            # evictions
+                        del block_of[p]
+                    live = {}
+                    for p, bl in block_of.items():
+                        live[bl] = live.get(bl, 0) + 1
+                    for bl in [b for b in list(fill) if b != tail and live.get(b, 0) == 0]:
+                        del fill[bl]                # empty blocks are freed
+                    for bl in sorted(b for b in fill if b != tail and 0 < live.get(b, 0) < theta * bs):
+                        for p in [p for p, b in block_of.items() if b == bl]:
+                            if fill[tail] >= bs:
+                                tail, next_id = next_id, next_id + 1
+                                fill[tail] = 0
+                            block_of[p] = tail
+                            fill[tail] += 1
+                            moved += 1
+                        del fill[bl]
+                    if prev:
+                        steps += 1
+                    slot_ratio.append(len(fill) * bs / max(1, len(block_of)))
+                    prev = cur
+            res[f"block_{bs}_theta_{theta}"] = {
+                "rows_moved_per_segment_step": moved / max(1, steps),
+                "bytes_moved_per_segment_step": 2 * row_bytes * moved / max(1, steps),
+                "slots_per_live_token": float(np.mean(slot_ratio)) if slot_ratio else None}
+    return res
 
 
 def warm_library(w, dev):
@@ -156,16 +285,21 @@ def warm_library(w, dev):
     import torch
     from confidence_gated_kv_logit_b200 import ConfKV, synth
     from confidence_gated_kv_logit_b200.binding import ALL_LAYERS
-    h = ConfKV(2, w["Hkv"], w["Hq"], w["D"], max_batch=2, max_prefill=600, n_low=64, n_high=128,
-               protect_last=16, fp16_window=32)
+    fixed = w["mode"] == "fixed"
+    kw = dict(mode=1, fixed_budget=96, n_sink=4, protect_last=24, int8_enable=0) if fixed else \
+        dict(n_low=64, n_high=128, protect_last=16, fp16_window=32)
+    h = ConfKV(2, w["Hkv"], w["Hq"], w["D"], max_batch=2, max_prefill=600, **kw)
     g = synth.generator(7, dev)
     k, v = synth.prefill_kv(2, w["Hkv"], 600, w["D"], g, dev)
+    pr = synth.priorities((2, w["Hkv"], 600), g, dev) if fixed else None
     for l in range(2):
-        h.prefill(k, v, [600, 500], layer=l)
+        h.prefill(k, v, [600, 500], layer=l, priority=pr)
     q, kn, vn = synth.step_qkv((2, 2), w["Hq"], w["Hkv"], w["D"], g, dev)
     out = torch.empty((2, 2, w["Hq"], w["D"]), device=dev)
-    h.decode_attn(q, kn, vn, out, ALL_LAYERS)
-    h.confidence(synth.bursty_logits(2, 4096, g, dev), torch.empty(2, device=dev))
+    h.decode_attn(q, kn, vn, out, ALL_LAYERS,
+                  prio_new=synth.priorities((2, 2, w["Hkv"]), g, dev) if fixed else None)
+    if not fixed:
+        h.confidence(synth.bursty_logits(2, 4096, g, dev), torch.empty(2, device=dev))
     h.evict_compact(ALL_LAYERS)
     torch.cuda.synchronize()
     h.close()
@@ -185,6 +319,13 @@ def max_over_ranks(ms: float, device) -> float:
 def whole_job_rate(world: int, batch: int, steps: int, ms: float) -> float:
     """Tokens per second of the whole job: every rank decodes `batch` sequences for `steps` steps."""
     return world * batch * steps / (ms / 1e3)
+
+
+def amortised_rate(batch: int, run_steps: int, step1_ms: float, steady_ms: float) -> dict:
+    """A run of `run_steps` steps whose first step costs step1_ms and the rest
+    steady_ms each: its mean step time and tokens per second."""
+    ms = (step1_ms + (run_steps - 1) * steady_ms) / run_steps
+    return {"steps": run_steps, "ms_per_step": ms, "value": batch / (ms * 1e-3), "unit": "tok/s"}
 
 
 def roofline_table(bytes_per_kernel, ms_per_kernel, peak):
@@ -207,7 +348,6 @@ class ClockSampler:
     def __init__(self, index: int):
         self.index = index
         self.proc = None
-        self.lines = []
 
     def start(self):
         try:
@@ -226,6 +366,10 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
             out = ""
+        return self.summarise(out)
+
+    @staticmethod
+    def summarise(out):
         rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 8]
         if not rows:
             return None
@@ -253,80 +397,133 @@ def physical_gpu_index(local_rank: int) -> int:
     return local_rank
 
 
+def default_steps(w, args):
+    """Timed steps: config 3 times 3000 steady steps; the others time the rest
+    of their stated run after the warm-up (at least one step)."""
+    if args.steps is not None:
+        return args.steps
+    if w["config"] == 3:
+        return 3000
+    return max(1, w["run_steps"] - args.warmup)
+
+
 # ---------------------------------------------------------------------------
 # CPU oracle legs (cpu_baseline and --impl reference)
 # ---------------------------------------------------------------------------
 
-def oracle_sample(w, seconds: float, steps_hint: int = 1):
-    """Time the oracle on a bounded sample of the workload; returns tok/s for
-    the whole workload extrapolated from per-segment-step and per-row times."""
-    import numpy as np
+def _oracle_worker(job):
+    """One oracle process: one segment of the workload, prefilled, then decode
+    steps (append, attention, EMA, eviction, conversion) for `seconds`, plus
+    confidence rows in confidence mode. Single-threaded. Returns the timed
+    segment-steps and rows and their seconds."""
+    os.environ["OMP_NUM_THREADS"] = "1"
+    os.environ["OPENBLAS_NUM_THREADS"] = "1"
+    os.environ["MKL_NUM_THREADS"] = "1"
     import torch
-    from threadpoolctl import threadpool_info
-
+    torch.set_num_threads(1)
     from confidence_gated_kv_logit_b200 import synth
     from oracle.confidence import confidence
     from oracle.segment import (Params, decode_attn_segment, evict_compact_segment, prefill_segment)
 
-    p = Params(n_low=w["n_low"], n_high=w["n_high"], tau=w["tau"], alpha=w["alpha"], ema_decay=w["beta"],
-               protect_last=w["P"], fp16_window=w["W"])
+    w, seconds, seed, layer = job
+    fixed = w["mode"] == "fixed"
+    if fixed:
+        p = Params(mode="fixed", n_sink=w["sinks"], protect_last=w["P"], fixed_budget=w["fixed"], int8=False,
+                   fp16_window=1)
+    else:
+        p = Params(n_low=w["n_low"], n_high=w["n_high"], tau=w["tau"], alpha=w["alpha"], ema_decay=w["beta"],
+                   protect_last=w["P"], fp16_window=w["W"], pyramidal=w["pyramidal"])
+    budget = p.budgets_for(w["n_low"], w["L"])[layer] if not fixed else w["fixed"]
     G = w["Hq"] // w["Hkv"]
-    g = synth.generator(1234)
-    nseg = 2
-    segs = []
-    for h in range(nseg):
-        k, v = synth.prefill_kv(1, 1, w["T"], w["D"], g)
-        segs.append(prefill_segment(k[0, 0].numpy(), v[0, 0].numpy(), None, p))
-    # bulk first step (not timed)
-    for i in range(nseg):
+    g = synth.generator(seed)
+    k, v = synth.prefill_kv(1, 1, w["T"], w["D"], g)
+    pr = synth.priorities((w["T"],), g).numpy() if fixed else None
+    seg = prefill_segment(k[0, 0].numpy(), v[0, 0].numpy(), pr, p, (layer, 0, 0))
+
+    def one_step(timed):
+        nonlocal seg
         q, kn, vn = synth.step_qkv((1,), G, 1, w["D"], g)
-        decode_attn_segment(segs[i], q[0].numpy(), kn[0, 0].numpy(), vn[0, 0].numpy(), None, p)
-        segs[i] = evict_compact_segment(segs[i], w["n_low"], p)
-    # steady segment-steps, timed
-    t_seg, n_seg = 0.0, 0
-    t_row, n_row = 0.0, 0
+        pn = float(synth.priorities((1,), g)[0]) if fixed else None
+        qn, knn, vnn = q[0].numpy(), kn[0, 0].numpy(), vn[0, 0].numpy()
+        t0 = time.perf_counter()
+        decode_attn_segment(seg, qn, knn, vnn, pn, p)
+        seg = evict_compact_segment(seg, budget, p)
+        return time.perf_counter() - t0
+
+    if w["config"] == 3:
+        one_step(False)   # the bulk first step: not part of the steady-state sample
+    t_seg = t_row = 0.0
+    n_seg = n_row = 0
     deadline = time.perf_counter() + seconds
-    while (time.perf_counter() < deadline or n_seg < 2 * steps_hint) and n_seg < 10000:
-        for i in range(nseg):
-            q, kn, vn = synth.step_qkv((1,), G, 1, w["D"], g)
-            qn, knn, vnn = q[0].numpy(), kn[0, 0].numpy(), vn[0, 0].numpy()
-            t0 = time.perf_counter()
-            decode_attn_segment(segs[i], qn, knn, vnn, None, p)
-            segs[i] = evict_compact_segment(segs[i], w["n_low"], p)
-            t_seg += time.perf_counter() - t0
-            n_seg += 1
-        if n_row < max(2, n_seg // 8):
+    while (time.perf_counter() < deadline or n_seg < 2) and n_seg < w["run_steps"] * 4 + 8:
+        t_seg += one_step(True)
+        n_seg += 1
+        if not fixed and n_row < max(1, n_seg // 16):
             logits = synth.bursty_logits(1, w["V"], g).numpy()[0]
             t0 = time.perf_counter()
             confidence(logits)
             t_row += time.perf_counter() - t0
             n_row += 1
-    per_seg = t_seg / n_seg
-    per_row = t_row / max(1, n_row)
+    return {"n_seg": n_seg, "t_seg": t_seg, "n_row": n_row, "t_row": t_row, "len": len(seg)}
+
+
+def oracle_workers() -> int:
+    try:
+        n = len(os.sched_getaffinity(0))
+    except Exception:
+        n = os.cpu_count() or 1
+    return max(1, min(n, 32))
+
+
+def oracle_sample(w, seconds: float, workers: int | None = None):
+    """Time the oracle on a bounded sample of the workload, one segment per
+    single-threaded process, all processes at once. The whole step's time is
+    extrapolated: S segments at the pool's aggregate segment-step rate plus B
+    confidence rows at its row rate."""
+    import multiprocessing as mp
+    # no more processes than the step has independent segments
+    n = min(workers or oracle_workers(), w["L"] * w["B"] * w["Hkv"])
+    layers = [0, w["L"] // 2, w["L"] - 1]
+    jobs = [(w, seconds, 4321 + i, layers[i % len(layers)]) for i in range(n)]
+    t0 = time.perf_counter()
+    if n == 1:
+        res = [_oracle_worker(jobs[0])]
+    else:
+        with mp.get_context("spawn").Pool(n) as pool:
+            res = pool.map(_oracle_worker, jobs)
+    wall = time.perf_counter() - t0
+    seg_rate = sum(r["n_seg"] / r["t_seg"] for r in res if r["t_seg"] > 0)
+    fixed = w["mode"] == "fixed"
+    row_rate = sum(r["n_row"] / r["t_row"] for r in res if r["t_row"] > 0) if not fixed else None
     S = w["L"] * w["B"] * w["Hkv"]
-    step_s = per_seg * S + per_row * w["B"]
-    threads = max([x.get("num_threads", 1) for x in threadpool_info()] + [1])
-    return {
-        "value": w["B"] / step_s, "unit": "tok/s", "cores": threads, "kind": "oracle",
-        "sample": (f"{n_seg} steady segment-steps over {nseg} of {S} segments (layer 0, seq 0) after a "
-                   f"{w['T']}-token prefill and the bulk first step (budget N_low each step), plus {n_row} "
-                   f"confidence rows of vocab {w['V']}; step time = per-segment-step x {S} + per-row x {w['B']}"),
-        "ms_per_step": step_s * 1e3,
-    }
+    step_s = S / seg_rate + (w["B"] / row_rate if row_rate else 0.0)
+    n_seg = sum(r["n_seg"] for r in res)
+    n_row = sum(r["n_row"] for r in res)
+    what = "the bulk first step, then steady" if w["config"] == 3 else "the first"
+    sample = (f"{n} single-threaded oracle processes at once, each one segment (layers {layers} in turn) "
+              f"after a {w['T']}-token prompt, timing {what} decode steps (append, fp64 attention, EMA, "
+              f"full-sort eviction, conversion): {n_seg} segment-steps"
+              + (f" and {n_row} confidence rows of vocab {w['V']}" if not fixed else "")
+              + f"; step time extrapolated = {S} segments / aggregate segment-step rate"
+              + (f" + {w['B']} rows / aggregate row rate" if not fixed else "")
+              + f" ({wall:.1f} s wall)")
+    return {"value": w["B"] / step_s, "unit": "tok/s", "cores": n, "kind": "oracle", "sample": sample,
+            "ms_per_step": step_s * 1e3, "wall_s": wall}
 
 
 def run_reference(args):
     if int(os.environ.get("RANK", "0")) != 0:
         return
     w = workload(args)
-    budget = max(1.0, 150.0 / max(1, args.steps + args.warmup))
-    r = oracle_sample(w, seconds=min(args.cpu_seconds * 3, budget * (args.steps + args.warmup)),
-                      steps_hint=args.steps)
-    line = {"metric": METRIC, "value": r["value"], "unit": "tok/s", "n_gpus": args.gpus, "steps": args.steps,
+    steps = args.steps if args.steps is not None else 20
+    r = oracle_sample(w, seconds=min(args.cpu_seconds * 3, 60.0))
+    line = {"metric": METRIC, "value": r["value"], "unit": "tok/s", "n_gpus": args.gpus, "steps": steps,
             "warmup": args.warmup, "ms_per_step": r["ms_per_step"], "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": {"workload": workload_name(w), "global_batch": w["B"], "seq_len": w["T"],
-                       "parallelism": "cpu oracle, rank 0"},
+                       "parallelism": "cpu oracle, rank 0", "gate": w["gate"]},
+            "extrapolated": (f"ms_per_step is extrapolated from the sample ({r['wall_s']:.1f} s of wall time), "
+                             f"not {steps} steps actually run; steps x ms_per_step exceeds the run's duration"),
             "cpu_baseline": {k: r[k] for k in ("value", "unit", "cores", "kind", "sample")},
             "e2e": {"value": r["value"], "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -336,87 +533,168 @@ def run_reference(args):
 # GPU leg
 # ---------------------------------------------------------------------------
 
-def main():
-    args = args_parse()
-    if args.impl == "reference":
-        run_reference(args)
-        return
+def make_handle(w, L=None, args=None, sliding_window=False):
+    from confidence_gated_kv_logit_b200 import ConfKV
+    L = L or w["L"]
+    if w["mode"] == "fixed":
+        return ConfKV(L, w["Hkv"], w["Hq"], w["D"], mode=1, max_batch=w["B"], max_prefill=w["T"],
+                      fixed_budget=w["fixed"], n_sink=w["sinks"], protect_last=w["P"], int8_enable=0,
+                      compact=1 if w["compact"] == "stable" else 0,
+                      single_stream=1 if w["graph"] else 0)
+    if sliding_window:
+        return ConfKV(L, w["Hkv"], w["Hq"], w["D"], max_batch=w["B"], max_prefill=w["T"], n_low=512,
+                      n_high=512, tau=w["tau"], alpha=0.0, ema_decay=w["beta"], protect_last=512,
+                      int8_enable=0, fp16_window=1)
+    return ConfKV(L, w["Hkv"], w["Hq"], w["D"], max_batch=w["B"], max_prefill=w["T"], n_low=w["n_low"],
+                  n_high=w["n_high"], tau=w["tau"], alpha=w["alpha"], ema_decay=w["beta"], protect_last=w["P"],
+                  fp16_window=w["W"], pyramidal=1 if w["pyramidal"] else 0,
+                  gate=1 if w["gate"] == "literal" else 0,
+                  compact=1 if w["compact"] == "stable" else 0,
+                  score_source={"ema": 0, "accum": 1, "random": 2}[w["score"]], seed=7,
+                  single_stream=1 if w["graph"] else 0)
+
+
+def step_bytes_model(w, d, K, launches_attn):
+    """Algorithmic bytes per kernel kind for K steps whose library counters
+    moved by `d` (SURVEY-style per-unit figures: INT8 token 2D+8 read + 4G
+    score write; FP16 token 4D + 4G; EMA 4G+12 per token + 208 per segment;
+    eviction 8 per scanned token + 2 x row bytes per moved row + 6D+8 per
+    converted token; confidence 4 per logit; append q + K/V + prepared query
+    operands; the fused EMA + eviction kernel both passes' bytes less the
+    candidate records). Returns (per-kernel bytes per step, attention bytes
+    per launch)."""
+    L, B, Hq, Hkv, D = w["L"], w["B"], w["Hq"], w["Hkv"], w["D"]
+    G = Hq // Hkv
+    fixed = w["mode"] == "fixed"
+    S = L * B * Hkv
+    qo = L * B * Hq * (2 * D + 4 * D + 4)
+    n8, n16 = d["attn_tokens_int8"], d["attn_tokens_fp16"]
+    attn_total = n8 * (2 * D + 8 + 4 * G) + n16 * (4 * D + 4 * G) + qo * K
+    cand = 0 if fixed else S * 208
+    ema = 0 if fixed else (n8 + n16) * (4 * G + 12) / K + cand
+    row = (2 * D + 16) if w.get("W", 0) and not fixed else (4 * D + 8)
+    evict = d["evict_tokens"] * 8 / K + cand + d["moved_rows"] * 2 * row / K + d["requant_rows"] * (6 * D + 8) / K
+    conf = 0 if fixed else B * w["V"] * 4
+    GP = 4 if G <= 4 else 8
+    qf = 2 * D * G + (4 * GP + 16) * D + 4 * GP
+    append = S * (4 * D + 4 * D + qf)
+    # the eviction kernel with the EMA pass fused in: both passes' bytes, without
+    # the candidate record the separate passes hand over (written and read once)
+    fused = ema + evict - 2 * cand
+    return ({"attention": attn_total / K, "ema": ema, "evict": evict, "ema_evict": fused, "confidence": conf,
+             "append": append}, attn_total / max(1, launches_attn))
+
+
+def counters_delta(a, b):
+    return {k: b[k] - a[k] for k in ("attn_tokens_int8", "attn_tokens_fp16", "evict_tokens", "moved_rows",
+                                     "requant_rows", "kernel_launches", "evict_block_segments")}
+
+
+def measure(w, args, dev, world, rank, local, with_e2e=True, with_graph=False, study=False):
+    """Run one workload: prefill, (config 3: the bulk first step on its own),
+    warm-up, the timed steps, then the same steps end to end with host
+    buffers. Returns a dict of measurements."""
     import torch
     import torch.distributed as dist
+    from confidence_gated_kv_logit_b200 import ALL_LAYERS, synth
 
-    from __graft_entry__ import build
-    from confidence_gated_kv_logit_b200 import ALL_LAYERS, ConfKV, synth
-
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
-    if rank == 0:
-        build()
-    if world > 1:
-        dist.barrier()
-    from confidence_gated_kv_logit_b200 import binding
-    binding.load_library()
-
-    w = workload(args)
     L, Hq, Hkv, D, B, T, V = (w[k] for k in ("L", "Hq", "Hkv", "D", "B", "T", "V"))
-    G = Hq // Hkv
-    warm_library(w, dev)
-    h = ConfKV(L, Hkv, Hq, D, max_batch=B, max_prefill=T, n_low=w["n_low"], n_high=w["n_high"], tau=w["tau"],
-               alpha=w["alpha"], ema_decay=w["beta"], protect_last=w["P"], fp16_window=w["W"],
-               compact=1 if w["compact"] == "stable" else 0,
-               score_source={"ema": 0, "accum": 1, "random": 2}[w["score"]], seed=7,
-               single_stream=1 if args.graph else 0)
+    fixed = w["mode"] == "fixed"
+    K = default_steps(w, args)
+    h = make_handle(w)
     gen = synth.generator(1000 + rank, dev)
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    # ---- prefill (fixed mode: select + gather, timed per layer) ----
+    pf_ms = 0.0
+    chunk = max(1, (1 << 30) // max(1, Hkv * T * D))
+    h.profile(True)
+    h.profile_read(reset=True)
+    s_pf0 = h.query()
     for l in range(L):
-        k, v = synth.prefill_kv(B, Hkv, T, D, gen, dev)
-        h.prefill(k, v, [T] * B, layer=l)
-        del k, v
+        if chunk >= B:
+            k, v = synth.prefill_kv(B, Hkv, T, D, gen, dev)
+        else:
+            k = torch.empty((B, Hkv, T, D), dtype=torch.float16, device=dev)
+            v = torch.empty_like(k)
+            for b0 in range(0, B, chunk):
+                b1 = min(B, b0 + chunk)
+                k[b0:b1], v[b0:b1] = synth.prefill_kv(b1 - b0, Hkv, T, D, gen, dev)
+        pr = synth.priorities((B, Hkv, T), gen, dev) if fixed else None
+        torch.cuda.synchronize()
+        e0.record(stream)
+        h.prefill(k, v, [T] * B, layer=l, priority=pr)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        pf_ms += e0.elapsed_time(e1)
+        del k, v, pr
+    prof_pf = h.profile_read(reset=True)
+    h.profile(False)
     torch.cuda.synchronize()
+
     pool = []
     for _ in range(POOL):
         q, kn, vn = synth.step_qkv((L, B), Hq, Hkv, D, gen, dev)
-        pool.append((q, kn, vn, synth.bursty_logits(B, V, gen, dev)))
+        extra = synth.priorities((L, B, Hkv), gen, dev) if fixed else synth.bursty_logits(B, V, gen, dev)
+        pool.append((q, kn, vn, extra))
     out = torch.empty((L, B, Hq, D), device=dev)
     c_out = torch.empty(B, device=dev)
-    stream = torch.cuda.current_stream()
 
-    def attn_call(q, kn, vn, o):
+    def attn_call(hh, q, kn, vn, o, pn):
         if w["calls"] == "per-layer":
             for l in range(L):
-                h.decode_attn(q[l], kn[l], vn[l], o[l], l)
+                hh.decode_attn(q[l], kn[l], vn[l], o[l], l, prio_new=None if pn is None else pn[l])
         else:
-            h.decode_attn(q, kn, vn, o, ALL_LAYERS)
+            hh.decode_attn(q, kn, vn, o, ALL_LAYERS, prio_new=pn)
 
-    def step(i):
-        q, kn, vn, lg = pool[i % POOL]
-        attn_call(q, kn, vn, out)
-        h.confidence(lg, c_out)
-        h.evict_compact(ALL_LAYERS)
+    def step_on(hh, i, o=out, c=c_out):
+        q, kn, vn, extra = pool[i % POOL]
+        attn_call(hh, q, kn, vn, o, extra if fixed else None)
+        if not fixed:
+            hh.confidence(extra, c)
+        hh.evict_compact(ALL_LAYERS)
 
-    # bulk first step, on its own (per-kernel times from the library's event brackets)
+    res = {"prefill_ms": pf_ms}
+    # ---- config 3: the bulk first step on its own ----
+    first = 0
     s0 = h.query()
-    h.profile(True)
-    h.profile_read(reset=True)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    step(0)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    step1_ms = e0.elapsed_time(e1)
-    prof1 = h.profile_read(reset=True)
-    h.profile(False)
-    s1 = h.query()
-    _report_device_error(h, "first step")
-    for i in range(1, 1 + args.warmup):
-        step(i)
+    if w["config"] == 3:
+        h.profile(True)
+        h.profile_read(reset=True)
+        e0.record(stream)
+        step_on(h, 0)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        res["step1_ms"] = e0.elapsed_time(e1)
+        prof1 = h.profile_read(reset=True)
+        h.profile(False)
+        s1 = h.query()
+        _report_device_error(h, "first step")
+        d1 = counters_delta(s0, s1)
+        b1, _ = step_bytes_model(w, d1, 1, max(1, prof1["attention"]["launches"]))
+        peak, _ = peaks()
+        res["step1_kernels"] = roofline_table(b1, {k: v["ms"] for k, v in prof1.items() if v["launches"]}, peak)
+        res["step1_counts"] = {k: d1[k] for k in ("attn_tokens_int8", "attn_tokens_fp16", "evict_tokens",
+                                                   "moved_rows", "requant_rows")}
+        first = 1
+    else:
+        # prefill's own traffic model (fixed mode: priorities read, kept rows gathered)
+        if fixed:
+            S = L * B * Hkv
+            kept = min(T, w["fixed"])
+            pf_bytes = S * (4 * T + kept * (4 * D + 8) * 2)
+            peak, _ = peaks()
+            res["prefill"] = {"ms": pf_ms, "bytes": pf_bytes, "gbs": pf_bytes / (pf_ms * 1e-3) / 1e9,
+                              "frac": pf_bytes / (pf_ms * 1e-3) / 1e9 / peak,
+                              "kernels_ms": {k: round(v["ms"], 4) for k, v in prof_pf.items() if v["launches"]}}
+    for i in range(first, first + args.warmup):
+        step_on(h, i)
     torch.cuda.synchronize()
     _report_device_error(h, "warm-up")
 
     # ---- timed region ----
+    history = [] if study else None
     h.profile(True)
     h.profile_read(reset=True)
     sa = h.query()
@@ -427,8 +705,9 @@ def main():
         dist.barrier()
     torch.cuda.synchronize()
     e0.record(stream)
-    for i in range(args.steps):
-        step(1 + args.warmup + i)
+    base = first + args.warmup
+    for i in range(K):
+        step_on(h, base + i)
     e1.record(stream)
     torch.cuda.synchronize()
     if world > 1:
@@ -440,54 +719,66 @@ def main():
     h.profile(False)
     sb = h.query()
     elapsed_ms = max_over_ranks(elapsed_ms, dev)
-    K = args.steps
-    value = whole_job_rate(world, B, K, elapsed_ms)
-
-    # ---- roofline of the dominant kernel (attention) ----
-    n8 = sb["attn_tokens_int8"] - sa["attn_tokens_int8"]
-    n16 = sb["attn_tokens_fp16"] - sa["attn_tokens_fp16"]
+    d = counters_delta(sa, sb)
     launches = max(1, prof["attention"]["launches"])
-    qo = L * B * Hq * (2 * D + 4 * D + 4)                       # q read, out + lse written, per step
-    attn_bytes = (n8 * (2 * D + 8 + 4 * G) + n16 * (4 * D + 4 * G) + qo * K) / launches
-    attn_ms = prof["attention"]["ms"] / launches
+    per_kernel, attn_bytes = step_bytes_model(w, d, K, launches)
     peak, peak_kind = peaks()
-    achieved = attn_bytes / (attn_ms * 1e-3) / 1e9
-    traffic = attn_traffic(w)
-    # whole-step algorithmic bytes: attention + EMA pass + confidence + eviction scan/moves
-    cand_bytes = L * B * Hkv * 208                                # eviction candidates, written and read once
-    ema_bytes = (n8 + n16) * (4 * G + 12) / K + cand_bytes          # scores, EMA r/w, positions
-    evict_bytes = (sb["evict_tokens"] - sa["evict_tokens"]) * 8 / K + cand_bytes
-    move_bytes = (sb["moved_rows"] - sa["moved_rows"]) * 2 * (2 * D + 16) / K
-    req_bytes = (sb["requant_rows"] - sa["requant_rows"]) * (6 * D + 8) / K
-    conf_bytes = B * V * 4
-    step_bytes = attn_bytes + ema_bytes + evict_bytes + move_bytes + req_bytes + conf_bytes
-    ms_step = elapsed_ms / K
-    kernel_ms = {k: round(v["ms"] / K, 4) for k, v in prof.items() if v["launches"]}
-    GP = 4 if G <= 4 else 8
-    qf_bytes = 2 * D * G + (4 * GP + 16) * D + 4 * GP               # q read + prepared operands written
-    append_bytes = L * B * Hkv * (4 * D + 4 * D + qf_bytes)
-    per_kernel_bytes = {"attention": attn_bytes * launches / K, "ema": ema_bytes,
-                        "evict": evict_bytes + move_bytes + req_bytes, "confidence": conf_bytes,
-                        "append": append_bytes}
-    kernels = roofline_table(per_kernel_bytes, kernel_ms, peak)
-    # step 1: the bulk eviction from the prompt down to the budget
-    d1 = {k: s1[k] - s0[k] for k in ("attn_tokens_int8", "attn_tokens_fp16", "evict_tokens", "moved_rows",
-                                     "requant_rows")}
-    step1_bytes = {
-        "attention": d1["attn_tokens_int8"] * (2 * D + 8 + 4 * G) + d1["attn_tokens_fp16"] * (4 * D + 4 * G) + qo,
-        "ema": (d1["attn_tokens_int8"] + d1["attn_tokens_fp16"]) * (4 * G + 12) + cand_bytes,
-        "evict": d1["evict_tokens"] * 8 + d1["moved_rows"] * 2 * (2 * D + 16) + d1["requant_rows"] * (6 * D + 8),
-        "confidence": conf_bytes, "append": append_bytes}
-    step1_kernels = roofline_table(step1_bytes, {k: v["ms"] for k, v in prof1.items() if v["launches"]}, peak)
+    attn_ms = prof["attention"]["ms"] / launches
+    res.update(K=K, elapsed_ms=elapsed_ms, ms_step=elapsed_ms / K, clocks=clocks, counters=d,
+               value=whole_job_rate(world, B, K, elapsed_ms), peak=peak, peak_kind=peak_kind,
+               attn_bytes=attn_bytes, attn_ms=attn_ms,
+               attn_tokens_per_launch=(d["attn_tokens_int8"] + d["attn_tokens_fp16"]) / launches,
+               kernel_ms={k: round(v["ms"] / K, 4) for k, v in prof.items() if v["launches"]},
+               gpu_launches=d["kernel_launches"])
+    res["kernels"] = roofline_table(per_kernel, res["kernel_ms"], peak)
+    res["step_hbm_gbs"] = sum(per_kernel.values()) / (res["ms_step"] * 1e-3) / 1e9
+    if w["config"] == 3:
+        res["amortised"] = amortised_rate(B, w["run_steps"], res["step1_ms"], res["ms_step"])
+
+    # ---- paged-layout study history: kept positions over a few more steps ----
+    if study:
+        import numpy as np
+        layers = sorted({0, L // 2, L - 1})
+        keys = [(l, hh) for l in layers for hh in range(Hkv)]
+        hist = {key: [] for key in keys}
+        for i in range(24):
+            step_on(h, base + K + i)
+            for (l, hh) in keys:
+                ex = h.export_segment(l, 0, hh)
+                live = ex["pos_r"] >= 0
+                hist[(l, hh)].append(np.concatenate([ex["pos_c"], ex["pos_r"][live]]).astype(np.int64))
+        history = list(hist.values())
+        res["paged_study"] = paged_study(h, w, history=history)
+        base += 24
 
     # ---- end to end through the public API with pinned host buffers ----
-    hpool = []
-    for i in range(8):
-        q, kn, vn, lg = pool[i]
-        hpool.append(tuple(x.cpu().pin_memory() for x in (q, kn, vn, lg)))
-    # Two buffer sets: step i+1's inputs upload on one copy stream and step
-    # i-1's results download on another (the two directions use separate
-    # copy engines) while step i computes.
+    if with_e2e:
+        res["e2e"] = e2e_leg(h, w, pool, args, dev, world, attn_call, base + K)
+    if with_graph:
+        res["graph"] = graph_leg(h, w, pool, K, dev, world, attn_call)
+    stats = h.query()
+    res["stats"] = stats
+    res["full_cache"] = L * B * Hkv * (T + first + args.warmup + K) * 4 * D
+    res["sw512"] = L * B * Hkv * 512 * 4 * D
+    _report_device_error(h, "the run")
+    h.close()
+    return res
+
+
+def e2e_leg(h, w, pool, args, dev, world, attn_call, start):
+    """The same steps through the public API with host buffers: each step's
+    inputs copied host->device from pinned memory and its outputs (attention
+    output, and c in confidence mode) device->host inside the timed region.
+    Two buffer sets: step i+1's upload and step i-1's download run on two copy
+    streams (separate copy engines) while step i computes."""
+    import torch
+    import torch.distributed as dist
+    from confidence_gated_kv_logit_b200 import ALL_LAYERS
+    fixed = w["mode"] == "fixed"
+    L, B, Hq, D = w["L"], w["B"], w["Hq"], w["D"]
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    hpool = [tuple(x.cpu().pin_memory() for x in pool[i]) for i in range(8)]
     up_s = torch.cuda.Stream(device=dev)
     down_s = torch.cuda.Stream(device=dev)
     dbuf = [tuple(torch.empty_like(x) for x in pool[0]) for _ in range(2)]
@@ -495,11 +786,11 @@ def main():
     cbuf = [torch.empty(B, device=dev) for _ in range(2)]
     host_out = [torch.empty((L, B, Hq, D), pin_memory=True) for _ in range(2)]
     host_c = [torch.empty(B, pin_memory=True) for _ in range(2)]
-    ev_in = [torch.cuda.Event() for _ in range(2)]
     ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_in = [torch.cuda.Event() for _ in range(2)]
     ev_out = [torch.cuda.Event() for _ in range(2)]
     h2d = sum(x.numel() * x.element_size() for x in hpool[0])
-    d2h = host_out[0].numel() * 4 + host_c[0].numel() * 4
+    d2h = host_out[0].numel() * 4 + (0 if fixed else host_c[0].numel() * 4)
     E = args.e2e_steps
     torch.cuda.synchronize()
     if world > 1:
@@ -525,15 +816,17 @@ def main():
         stream.wait_event(ev_in[j])
         if i >= 2:
             stream.wait_event(ev_out[j])               # step i-2's results have left buffer set j
-        dq, dk, dv, dl = dbuf[j]
-        attn_call(dq, dk, dv, obuf[j])
-        h.confidence(dl, cbuf[j])
+        dq, dk, dv, dx = dbuf[j]
+        attn_call(h, dq, dk, dv, obuf[j], dx if fixed else None)
+        if not fixed:
+            h.confidence(dx, cbuf[j])
         h.evict_compact(ALL_LAYERS)
         ev_comp[j].record(stream)
         with torch.cuda.stream(down_s):
             down_s.wait_event(ev_comp[j])
             host_out[j].copy_(obuf[j], non_blocking=True)
-            host_c[j].copy_(cbuf[j], non_blocking=True)
+            if not fixed:
+                host_c[j].copy_(cbuf[j], non_blocking=True)
             ev_out[j].record(down_s)
     stream.wait_stream(up_s)
     stream.wait_stream(down_s)
@@ -542,94 +835,190 @@ def main():
     e2e_ms = e0.elapsed_time(e1)
     _report_device_error(h, "end-to-end region")
     e2e_ms = max_over_ranks(e2e_ms, dev)
-    e2e_value = whole_job_rate(world, B, E, e2e_ms)
+    return {"value": whole_job_rate(world, B, E, e2e_ms), "unit": "tok/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": E,
+            "pipelining": "two buffer sets; step i+1's upload and step i-1's download on two copy streams"}
 
-    # ---- optional: the same step replayed from a CUDA graph ----
-    graph_line = None
-    if args.graph:
-        sq, skn, svn, slg = (x.clone() for x in pool[0])
-        gout = torch.empty_like(out)
-        gc = torch.empty_like(c_out)
-        torch.cuda.synchronize()
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
-            attn_call(sq, skn, svn, gout)
-            h.confidence(slg, gc)
-            h.evict_compact(ALL_LAYERS)
 
-        def replay(i):
-            q, kn, vn, lg = pool[i % POOL]
-            sq.copy_(q)
-            skn.copy_(kn)
-            svn.copy_(vn)
-            slg.copy_(lg)
-            graph.replay()
+def graph_leg(h, w, pool, K, dev, world, attn_call):
+    """The same step replayed from one captured CUDA graph."""
+    import torch
+    from confidence_gated_kv_logit_b200 import ALL_LAYERS
+    fixed = w["mode"] == "fixed"
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sq, skn, svn, sx = (x.clone() for x in pool[0])
+    gout = torch.empty((w["L"], w["B"], w["Hq"], w["D"]), device=dev)
+    gc = torch.empty(w["B"], device=dev)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        attn_call(h, sq, skn, svn, gout, sx if fixed else None)
+        if not fixed:
+            h.confidence(sx, gc)
+        h.evict_compact(ALL_LAYERS)
 
-        for i in range(3):
-            replay(i)
-        torch.cuda.synchronize()
-        Kg = min(K, 1000)
-        e0.record(stream)
-        for i in range(Kg):
-            replay(i)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        _report_device_error(h, "graph replays")
-        g_ms = max_over_ranks(e0.elapsed_time(e1), dev)
-        graph_line = {"ms_per_step": g_ms / Kg, "value": whole_job_rate(world, B, Kg, g_ms), "steps": Kg,
-                      "note": "one captured step (inputs copied into its static buffers each step, inside the timing)"}
-        del graph
+    def replay(i):
+        for dst, src in zip((sq, skn, svn, sx), pool[i % POOL]):
+            dst.copy_(src)
+        graph.replay()
 
-    stats = h.query()
-    study = paged_study(h, w) if args.paged_study else None
-    full_cache = L * B * Hkv * (T + 1 + args.warmup + K + E) * 4 * D
-    sw512 = L * B * Hkv * 512 * 4 * D
-    _report_device_error(h, "the run")
+    for i in range(3):
+        replay(i)
+    torch.cuda.synchronize()
+    Kg = min(K, 1000)
+    e0.record(stream)
+    for i in range(Kg):
+        replay(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    _report_device_error(h, "graph replays")
+    g_ms = max_over_ranks(e0.elapsed_time(e1), dev)
+    del graph
+    return {"ms_per_step": g_ms / Kg, "value": whole_job_rate(world, w["B"], Kg, g_ms), "steps": Kg,
+            "note": "one captured step (inputs copied into its static buffers each step, inside the timing)"}
 
+
+def line_for(w, res, args, world, cpu):
+    traffic = attn_traffic(w, res["attn_tokens_per_launch"]) if not w["reduced"] else None
+    achieved = res["attn_bytes"] / (res["attn_ms"] * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": res["value"], "unit": "tok/s", "n_gpus": world, "steps": res["K"],
+        "warmup": args.warmup, "ms_per_step": res["ms_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": workload_name(w), "config": w["config"], "global_batch": w["B"] * world,
+                   "seq_len": w["T"], "gate": w["gate"] if w["mode"] != "fixed" else None,
+                   "parallelism": f"replicas x{world} (independent sequences, no collective)",
+                   "l2": "no flush: the per-step working set exceeds the 126 MB L2" if w["config"] >= 3 else
+                         "no flush: the whole cache fits in L2 (a launch-bound, latency-measured configuration)",
+                   "input_pool": f"{POOL} pre-generated step inputs reused cyclically"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": res["peak"], "unit": "GB/s",
+                     "frac": achieved / res["peak"], "traffic": traffic, "peak_kind": res["peak_kind"],
+                     "kernel": "attn_kernel", "algorithmic_bytes_per_launch": res["attn_bytes"],
+                     "ms_per_launch": res["attn_ms"], "attn_tokens_per_launch": res["attn_tokens_per_launch"]},
+        "cpu_baseline": cpu,
+        "e2e": res.get("e2e"),
+        "gpu_launches": res["gpu_launches"],
+        "clocks": res["clocks"],
+        "kernels": res["kernels"],
+        "evict_block_segments_per_step": res["counters"]["evict_block_segments"] / res["K"],
+        "step_hbm_gbs": res["step_hbm_gbs"],
+        "kernel_ms_per_step": res["kernel_ms"],
+        "kv_resident_bytes": {"conf_kv": res["stats"]["bytes_payload"], "full_fp16": res["full_cache"],
+                              "sliding_window_512": res["sw512"], "tokens_int8": res["stats"]["tokens_int8"],
+                              "tokens_fp16": res["stats"]["tokens_fp16"]},
+        "us_per_step": res["ms_step"] * 1e3,
+    }
+    for k in ("step1_ms", "step1_kernels", "step1_counts", "amortised", "prefill", "graph", "paged_study"):
+        if k in res:
+            line[k] = res[k]
+    return line
+
+
+def main():
+    args = args_parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import torch
+    import torch.distributed as dist
+
+    from __graft_entry__ import build
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
     if rank == 0:
-        cpu = None
-        if not args.no_cpu_baseline and world == 1:
-            r = oracle_sample(w, seconds=args.cpu_seconds)
-            cpu = {k: r[k] for k in ("value", "unit", "cores", "kind", "sample")}
-        line = {
-            "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
-            "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "f32", "data": "synthetic",
-            "config": {"workload": workload_name(w), "global_batch": B * world, "seq_len": T,
-                       "parallelism": f"replicas x{world} (independent sequences, no collective)",
-                       "l2": "no flush: the per-step working set (~1.4 GB of KV + inputs) exceeds the 126 MB L2",
-                       "input_pool": f"{POOL} pre-generated step inputs reused cyclically"},
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,
-                         "kernel": "attn_kernel", "algorithmic_bytes_per_launch": attn_bytes,
-                         "ms_per_launch": attn_ms},
-            "cpu_baseline": cpu,
-            "e2e": {"value": e2e_value, "unit": "tok/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "pipelining": "two buffer sets; step i+1's upload and step i-1's download on two copy streams",
-                    "steps": E},
-            "gpu_launches": sb["kernel_launches"] - sa["kernel_launches"],
-            "clocks": clocks,
-            "kernels": kernels,
-            "evict_block_segments_per_step": (sb["evict_block_segments"] - sa["evict_block_segments"]) / K,
-            "step1_ms": step1_ms,
-            "step1_kernels": step1_kernels,
-            "step1_counts": d1,
-            "step1_attn_tokens": {"int8": s1["attn_tokens_int8"] - s0["attn_tokens_int8"],
-                                  "fp16": s1["attn_tokens_fp16"] - s0["attn_tokens_fp16"]},
-            "step_hbm_gbs": step_bytes / (ms_step * 1e-3) / 1e9,
-            "kernel_ms_per_step": kernel_ms,
-            "kv_resident_bytes": {"conf_kv": stats["bytes_payload"], "full_fp16": full_cache, "sliding_window_512": sw512,
-                                  "tokens_int8": stats["tokens_int8"], "tokens_fp16": stats["tokens_fp16"]},
-        }
-        if study is not None:
-            line["paged_study"] = study
-        if graph_line is not None:
-            line["graph"] = graph_line
+        build()
+    if world > 1:
+        dist.barrier()
+    from confidence_gated_kv_logit_b200 import binding
+    binding.load_library()
+
+    if args.config == 5 and (args.batch is None or args.ctx is None):
+        points = [(b, c) for (b, c) in SWEEP5 if (args.batch in (None, b)) and (args.ctx in (None, c))]
+    else:
+        points = [(args.batch, args.ctx)]
+    w0 = workload(args, *points[-1])
+    warm_library(w0, dev)
+
+    lines = []
+    for (b, c) in points:
+        w = workload(args, b, c)
+        res = measure(w, args, dev, world, rank, local, with_graph=args.graph, study=args.paged_study)
+        lines.append((w, res))
+    w, res = lines[-1]
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
+        r = oracle_sample(w, seconds=args.cpu_seconds)
+        cpu = {k: r[k] for k in ("value", "unit", "cores", "kind", "sample")}
+    sw = None
+    if w["config"] == 2:
+        # the fixed 512-token sliding window in the same harness
+        ws = dict(w, shape="gpt2-small-shape sliding window 512", P=512, W=0, alpha=0.0, n_low=512, n_high=512)
+        sw = measure_sliding_window(ws, args, dev, world, rank, local)
+    if rank == 0:
+        line = line_for(w, res, args, world, cpu)
+        if len(lines) > 1:
+            line["sweep"] = [{"batch": wx["B"], "ctx": wx["T"], "decode_tok_s": rx["value"],
+                              "decode_ms_per_step": rx["ms_step"], "prefill": rx.get("prefill"),
+                              "attn_frac": rx["attn_bytes"] / (rx["attn_ms"] * 1e-3) / 1e9 / rx["peak"],
+                              "kernels": rx["kernels"], "e2e_tok_s": rx["e2e"]["value"],
+                              "kv_resident_bytes": rx["stats"]["bytes_payload"], "full_fp16": rx["full_cache"]}
+                             for (wx, rx) in lines]
+            line["config"]["workload"] += f" (headline point of a {len(lines)}-point batch x context sweep)"
+        if sw is not None:
+            line["sliding_window_512"] = sw
         print(json.dumps(line), flush=True)
-    h.close()
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def measure_sliding_window(ws, args, dev, world, rank, local):
+    """Config 2's comparison: a plain 512-token sliding window (recency-only
+    ranking, every token protected up to 512, FP16 throughout) on the same
+    shape and harness."""
+    import torch
+    from confidence_gated_kv_logit_b200 import ALL_LAYERS, synth
+    L, Hq, Hkv, D, B, T, V = (ws[k] for k in ("L", "Hq", "Hkv", "D", "B", "T", "V"))
+    h = make_handle(ws, sliding_window=True)
+    gen = synth.generator(2000 + rank, dev)
+    for l in range(L):
+        k, v = synth.prefill_kv(B, Hkv, T, D, gen, dev)
+        h.prefill(k, v, [T] * B, layer=l)
+    pool = [synth.step_qkv((L, B), Hq, Hkv, D, gen, dev) + (synth.bursty_logits(B, V, gen, dev),)
+            for _ in range(POOL)]
+    out = torch.empty((L, B, Hq, D), device=dev)
+    c = torch.empty(B, device=dev)
+    K = default_steps(ws, args)
+
+    def step(i):
+        q, kn, vn, lg = pool[i % POOL]
+        h.decode_attn(q, kn, vn, out, ALL_LAYERS)
+        h.confidence(lg, c)
+        h.evict_compact(ALL_LAYERS)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(K):
+        step(args.warmup + i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    _report_device_error(h, "sliding window")
+    ms = max_over_ranks(e0.elapsed_time(e1), dev)
+    st = h.query()
+    h.close()
+    return {"value": whole_job_rate(world, B, K, ms), "unit": "tok/s", "ms_per_step": ms / K, "steps": K,
+            "kv_resident_bytes": st["bytes_payload"], "max_len": st["max_len"]}
 
 
 if __name__ == "__main__":

@@ -53,3 +53,58 @@ def test_workload_names_mark_the_variants():
         prefill = None
     base = bench.workload_name(bench.workload(D))
     assert "per layer" not in base and "stable" not in base and "ranking" not in base
+
+
+def test_block_compaction_replay_counts_moved_rows():
+    # blocks of 4 slots: positions 0..7 fill blocks 0 and 1; then 0, 1, 2 are
+    # evicted and 8 arrives. Block 0 keeps 1 live token (< 0.5 x 4), so it is
+    # compacted: its one row moves to the tail (block 2, which 8 opened).
+    hist = [[np.arange(8), np.array([3, 4, 5, 6, 7, 8])]]
+    r = bench.block_compaction_study(hist, (4,), (0.5,), row_bytes=100)["block_4_theta_0.5"]
+    assert r["rows_moved_per_segment_step"] == 1.0
+    assert r["bytes_moved_per_segment_step"] == 200.0
+    # after the move: block 1 (4 live) and block 2 (8, 3) hold 2 x 4 slots for 6 live tokens
+    assert r["slots_per_live_token"] == (8 / 8 + 8 / 6) / 2
+    # a threshold of 0 never compacts; an empty block is freed without moves
+    r0 = bench.block_compaction_study([[np.arange(8), np.arange(4, 9)]], (4,), (0.0,), 100)["block_4_theta_0.0"]
+    assert r0["rows_moved_per_segment_step"] == 0.0
+    assert r0["slots_per_live_token"] == (8 / 8 + 8 / 5) / 2
+
+
+def test_amortised_rate_of_a_run():
+    r = bench.amortised_rate(16, 256, step1_ms=7.5, steady_ms=0.35)
+    ms = (7.5 + 255 * 0.35) / 256
+    assert abs(r["ms_per_step"] - ms) < 1e-12
+    assert abs(r["value"] - 16 / (ms * 1e-3)) < 1e-6
+
+
+def test_config_workloads_and_default_steps():
+    class A:
+        config = 4
+        steps = None
+        warmup = 10
+    w = bench.workload(A)
+    assert (w["L"], w["Hq"], w["Hkv"], w["B"], w["T"], w["V"]) == (64, 40, 8, 32, 512, 152064)
+    assert w["pyramidal"] and bench.default_steps(w, A) == 4096 - 10
+    A.config = 3
+    assert bench.default_steps(bench.workload(A), A) == 3000
+    class F:
+        config = 5
+        batch = 64
+        ctx = 131072
+        gate = "literal"
+    w = bench.workload(F)
+    assert (w["B"], w["T"], w["mode"], w["fixed"]) == (64, 131072, "fixed", 2048)
+    assert "B=2048 = 4 sinks + 512 window + 1532 top-k" in bench.workload_name(w)
+    class G:
+        gate = "literal"
+    assert "pseudo-code line" in bench.workload_name(bench.workload(G))
+
+
+def test_oracle_baseline_runs_one_segment_per_process():
+    class A:
+        config = 1
+    w = bench.workload(A)
+    r = bench.oracle_sample(w, seconds=0.5, workers=2)
+    assert r["cores"] == 2 and r["value"] > 0 and r["unit"] == "tok/s"
+    assert "2 single-threaded oracle processes" in r["sample"]

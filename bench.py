@@ -188,9 +188,7 @@ def paged_study(h, w, block_sizes=(16, 32, 64, 128), history=None, thresholds=(0
     segments over consecutive steps): a paged cache that rewrites a block
     once its live count falls below `theta * bs` -- moving its live tokens to
     the tail block -- holds fewer slots but moves rows. Replayed over the
-    history per block size and threshold: rows moved per segment-step, the
-    bytes that costs at the layout's row size, and the slots held per live
-    token at the end."""
+    history per block size and threshold (block_compaction_study)."""
     import numpy as np
     L, Hkv = w["L"], w["Hkv"]
     layers = sorted({0, L // 2, L - 1})
@@ -223,41 +221,42 @@ def block_compaction_study(history, block_sizes, thresholds, row_bytes):
     """Replay of a block-granular compaction policy over kept-position
     histories (one list of per-step position arrays per segment).
 
-    Model: a paged cache holds tokens in blocks of `bs` slots, filled in
-    arrival order; the newest block receives appended tokens. After each
-    step's eviction, every non-tail block whose live count is below
-    theta * bs is compacted: its live tokens are appended to the tail (moving
-    one row each, read and write), and the block is freed. Blocks left empty
-    are freed at no cost. Reported per (bs, theta): rows moved per
-    segment-step, bytes moved per segment-step (2 x row bytes per row), and
-    the slots held per live token averaged over the replay."""
+    Model: a paged cache holds tokens in blocks of `bs` slots. At the start
+    every kept token sits in the block of its position (pos // bs), as in a
+    cache that appended tokens in order and only freed empty blocks; the
+    block of the newest position is the tail, which receives appended
+    tokens (a new block when it is full). After each step's eviction, every
+    non-tail block whose live count is below theta * bs is compacted: its
+    live tokens are appended to the tail (one row moved each, read and
+    written) and the block is freed; blocks left empty are freed at no cost.
+    Reported per (bs, theta): the rows moved once to compact the starting
+    layout, then per segment-step the rows and bytes (2 x row bytes per row)
+    moved, and the slots held per live token averaged over the steps."""
     import numpy as np
     res = {}
     for bs in block_sizes:
         for theta in thresholds:
-            moved = steps = 0
+            moved = steps = initial = 0
             slot_ratio = []
             for seq in history:
-                block_of = {}                       # position -> block id
-                fill = {}                           # block id -> slots used (ever)
-                tail = -1
-                next_id = 0
-                prev = set()
-                for pos in seq:
-                    cur = set(int(x) for x in pos)
-                    for p in sorted(cur - prev):    # arrivals (the prompt, then one per step)
-                        if tail < 0 or fill[tail] >= bs:
-                            tail, next_id = next_id, next_id + 1
-                            fill[tail] = 0
-                        block_of[p] = tail
-                        fill[tail] += 1
-                    for p in prev - cur:            # evictions
-                        del block_of[p]
+                if not len(seq):
+                    continue
+                first = np.asarray(seq[0], np.int64)
+                block_of = {int(p): int(p) // bs for p in first}
+                tail = int(first.max()) // bs if first.size else 0
+                fill = {b: bs for b in set(block_of.values())}
+                fill[tail] = int(first.max()) % bs + 1 if first.size else 0
+                next_id = tail + 1
+                prev = set(block_of)
+
+                def compact(count_into):
+                    nonlocal tail, next_id
                     live = {}
-                    for p, bl in block_of.items():
+                    for bl in block_of.values():
                         live[bl] = live.get(bl, 0) + 1
                     for bl in [b for b in list(fill) if b != tail and live.get(b, 0) == 0]:
                         del fill[bl]                # empty blocks are freed
+                    n = 0
                     for bl in sorted(b for b in fill if b != tail and 0 < live.get(b, 0) < theta * bs):
                         for p in [p for p, b in block_of.items() if b == bl]:
                             if fill[tail] >= bs:
@@ -265,13 +264,27 @@ def block_compaction_study(history, block_sizes, thresholds, row_bytes):
                                 fill[tail] = 0
                             block_of[p] = tail
                             fill[tail] += 1
-                            moved += 1
+                            n += 1
                         del fill[bl]
-                    if prev:
-                        steps += 1
+                    return n
+
+                initial += compact(None)
+                for pos in seq[1:]:
+                    cur = set(int(x) for x in pos)
+                    for p in sorted(cur - prev):    # arrivals (one per step)
+                        if fill[tail] >= bs:
+                            tail, next_id = next_id, next_id + 1
+                            fill[tail] = 0
+                        block_of[p] = tail
+                        fill[tail] += 1
+                    for p in prev - cur:            # evictions
+                        del block_of[p]
+                    moved += compact(None)
+                    steps += 1
                     slot_ratio.append(len(fill) * bs / max(1, len(block_of)))
                     prev = cur
             res[f"block_{bs}_theta_{theta}"] = {
+                "initial_rows_moved_per_segment": initial / max(1, len(history)),
                 "rows_moved_per_segment_step": moved / max(1, steps),
                 "bytes_moved_per_segment_step": 2 * row_bytes * moved / max(1, steps),
                 "slots_per_live_token": float(np.mean(slot_ratio)) if slot_ratio else None}
@@ -741,7 +754,7 @@ def measure(w, args, dev, world, rank, local, with_e2e=True, with_graph=False, s
         layers = sorted({0, L // 2, L - 1})
         keys = [(l, hh) for l in layers for hh in range(Hkv)]
         hist = {key: [] for key in keys}
-        for i in range(24):
+        for i in range(64):
             step_on(h, base + K + i)
             for (l, hh) in keys:
                 ex = h.export_segment(l, 0, hh)
@@ -749,7 +762,7 @@ def measure(w, args, dev, world, rank, local, with_e2e=True, with_graph=False, s
                 hist[(l, hh)].append(np.concatenate([ex["pos_c"], ex["pos_r"][live]]).astype(np.int64))
         history = list(hist.values())
         res["paged_study"] = paged_study(h, w, history=history)
-        base += 24
+        base += 64
 
     # ---- end to end through the public API with pinned host buffers ----
     if with_e2e:

@@ -32,7 +32,7 @@ EXPORTED = ["confkv_default_params", "confkv_create", "confkv_destroy", "confkv_
             "confkv_export_segment", "confkv_last_error", "confkv_last_error_detail",
             "confkv_profile_enable", "confkv_profile_read", "confkv_confidence_noalloc",
             "confkv_status_string", "confkv_version"]
-KERNEL_KINDS = ["confidence", "append", "attention", "combine", "ema", "evict", "prefill", "unused"]
+KERNEL_KINDS = ["confidence", "append", "attention", "combine", "ema", "evict", "prefill", "ema_evict"]
 
 
 class ConfKVError(RuntimeError):
@@ -247,7 +247,7 @@ class ConfKV:
         pr = Profile()
         _check(load_library().confkv_profile_read(self._h, ctypes.byref(pr), 1 if reset else 0), "confkv_profile_read")
         return {name: {"launches": int(pr.launches[i]), "ms": float(pr.ms[i])}
-                for i, name in enumerate(KERNEL_KINDS) if name != "unused"}
+                for i, name in enumerate(KERNEL_KINDS)}
 
     def last_error(self, clear: bool = False) -> int:
         return int(load_library().confkv_last_error(self._h, 1 if clear else 0))

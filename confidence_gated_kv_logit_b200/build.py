@@ -1,6 +1,6 @@
 """Build libconfkv.so (the CUDA library behind include/confkv.h) in-tree.
 
-One nvcc invocation compiles every translation unit under csrc/ for sm_100a
+nvcc compiles every translation unit under csrc/ for sm_100a (in parallel)
 and links a shared library next to this file. The runtime is linked
 statically, so the library needs only the driver at run time.
 """
@@ -63,20 +63,36 @@ def build_checked(verbose: bool = False) -> str:
 
 
 def build(verbose: bool = False, ptxas_info: bool = False, force: bool = False) -> str:
+    """Compile every translation unit to an object (in parallel), then link
+    the shared library."""
     if not force and not needs_build():
         return LIB
+    import tempfile
+    from concurrent.futures import ThreadPoolExecutor
     nvcc = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
-    cmd = [nvcc, *NVCC_FLAGS, "-shared", "-I", os.path.join(ROOT, "include"), "-o", LIB + ".tmp", *sources()]
-    if ptxas_info:
-        cmd[1:1] = ["-Xptxas", "-v"]
-    if verbose:
-        print(" ".join(cmd), flush=True)
-    res = subprocess.run(cmd, capture_output=True, text=True)
-    if res.returncode != 0:
-        sys.stderr.write(res.stdout + res.stderr)
-        raise RuntimeError("nvcc failed to build libconfkv.so")
-    if ptxas_info or verbose:
-        sys.stdout.write(res.stdout + res.stderr)
+    extra = ["-Xptxas", "-v"] if ptxas_info else []
+    with tempfile.TemporaryDirectory(prefix="confkv_build_") as tmp:
+        def compile_one(src):
+            obj = os.path.join(tmp, os.path.basename(src) + ".o")
+            cmd = [nvcc, *extra, *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), "-c", src, "-o", obj]
+            if verbose:
+                print(" ".join(cmd), flush=True)
+            return obj, subprocess.run(cmd, capture_output=True, text=True)
+        with ThreadPoolExecutor(max_workers=max(1, min(len(sources()), os.cpu_count() or 1))) as ex:
+            results = list(ex.map(compile_one, sources()))
+        for _, res in results:
+            if res.returncode != 0:
+                sys.stderr.write(res.stdout + res.stderr)
+                raise RuntimeError("nvcc failed to build libconfkv.so")
+            if ptxas_info or verbose:
+                sys.stdout.write(res.stdout + res.stderr)
+        link = [nvcc, *NVCC_FLAGS, "-shared", "-o", LIB + ".tmp", *[o for o, _ in results]]
+        if verbose:
+            print(" ".join(link), flush=True)
+        res = subprocess.run(link, capture_output=True, text=True)
+        if res.returncode != 0:
+            sys.stderr.write(res.stdout + res.stderr)
+            raise RuntimeError("nvcc failed to link libconfkv.so")
     os.replace(LIB + ".tmp", LIB)
     with open(STAMP, "w") as f:
         f.write(source_digest())

@@ -13,7 +13,8 @@
 //                    tensor cores (mma.sync) and keep one online softmax per
 //                    CTA.
 //   combine_kernel : merges split partials into out and lse
-// and then (ema.cu) the second pass with the saved log-sum-exp.
+// The second pass with the saved log-sum-exp (the attention-mass EMA) runs in
+// the eviction kernel's fused variant, or on its own (ema.cu).
 //
 // Arithmetic. The G query heads of one KV head (padded to GP = 4 or 8) make
 // both products small GEMMs:
@@ -268,7 +269,14 @@ struct Cfg {
   static constexpr int FLAG_OFF = BAR_OFF + 2 * NSTAGE * 8;
   static constexpr int UQ = 8;                  // unit-id queue entries (> NSTAGE)
   static constexpr int UQ_OFF = FLAG_OFF + 16;
-  static constexpr int SMEM = UQ_OFF + UQ * 4;
+  static constexpr int UN_OFF = UQ_OFF + UQ * 4;  // each queued unit's cold-token count
+  // The query operands of the next unit are staged in shared memory when a
+  // slot fits beside two CTAs per SM (GP = 4); otherwise the consumers read
+  // them from global memory.
+  static constexpr bool QSM = GP == 4;
+  static constexpr int QBAR_OFF = UN_OFF + UQ * 4;                 // qfull, qempty mbarriers
+  static constexpr int QS_OFF = (QBAR_OFF + 16 + 127) / 128 * 128;
+  static constexpr int SMEM = QSM ? QS_OFF + QF<D, GP>::BYTES : QBAR_OFF + 16;
 };
 
 struct Unit {
@@ -277,14 +285,16 @@ struct Unit {
   int tiles_c, t0, t1;
 };
 
+// n_cold < -1: read the segment's count from global memory (the producer);
+// otherwise the count the producer read (the consumers, from the unit queue).
 template <int D, int GP, bool CI8>
-__device__ __forceinline__ Unit make_unit(const Cache& c, const Range& r, int splits, int unit) {
+__device__ __forceinline__ Unit make_unit(const Cache& c, const Range& r, int splits, int unit, int n_cold = -2) {
   using C = Cfg<D, GP, CI8>;
   Unit u;
   const int item = unit / splits;
   const int split = unit - item * splits;
   u.s = seg_of(c, r, item, &u.l, &u.b, &u.h);
-  u.n_cold = c.n_cold[u.s];
+  u.n_cold = n_cold < -1 ? c.n_cold[u.s] : n_cold;
   if (u.n_cold < 0 || u.n_cold > c.cap) {   // corrupt segment: record once (by its split 0) and skip
     if (split == 0 && threadIdx.x == 0) record_violation(c.err, kSiteAttnSeg, u.s, u.n_cold);
     u.n_cold = 0;
@@ -699,6 +709,10 @@ __global__ void __launch_bounds__(160, 2) attn_kernel(Cache c, AttnLaunch a, int
   uint64_t* empty = full + C::NSTAGE;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::FLAG_OFF);
   volatile int* uq = reinterpret_cast<volatile int*>(smem + C::UQ_OFF);
+  volatile int* uqn = reinterpret_cast<volatile int*>(smem + C::UN_OFF);
+  uint64_t* qfull = reinterpret_cast<uint64_t*>(smem + C::QBAR_OFF);
+  uint64_t* qempty = qfull + 1;
+  unsigned char* qsm = smem + C::QS_OFF;   // valid when C::QSM
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -712,6 +726,8 @@ __global__ void __launch_bounds__(160, 2) attn_kernel(Cache c, AttnLaunch a, int
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], C::NCW);
     }
+    mbar_init(qfull, 1);
+    mbar_init(qempty, C::NCW);
     abort_flag[0] = 0;
     fence_mbar_init();
   }
@@ -728,6 +744,7 @@ __global__ void __launch_bounds__(160, 2) attn_kernel(Cache c, AttnLaunch a, int
       // is published; a unit without tiles, and the end, are published as a
       // stage without data.
       int ctr = 0;
+      int nq = 0;   // query-operand copies issued
       bool stop = false;
       auto next_stage = [&]() -> int {
         const int st = ctr % C::NSTAGE;
@@ -751,6 +768,21 @@ __global__ void __launch_bounds__(160, 2) attn_kernel(Cache c, AttnLaunch a, int
         }
         const Unit u = make_unit<D, GP, CI8>(c, a.r, splits, unit);
         uq[k % C::UQ] = unit;
+        uqn[k % C::UQ] = u.n_cold;
+        // the consumers load the unit's query operands when they reach it (up
+        // to NSTAGE tiles from now)
+        if constexpr (C::QSM) {
+          // into the one shared slot, once the consumers have read the previous unit's
+          if (k > 0 && !mbar_wait_bounded(qempty, (k - 1) & 1)) {
+            set_error(c.err, kErrDevice);
+            *abort_flag = 1;
+            stop = true;
+            break;
+          }
+          mbar_arrive_expect_tx(qfull, (uint32_t)Q::BYTES);
+          bulk_g2s(qsm, a.qfrag + (size_t)u.s * a.qf_stride, (uint32_t)Q::BYTES, qfull);
+          ++nq;
+        }
         if (u.t0 == u.t1) {
           const int st = next_stage();
           if (stop) break;
@@ -807,6 +839,7 @@ __global__ void __launch_bounds__(160, 2) attn_kernel(Cache c, AttnLaunch a, int
       if (stop) {
         for (int k = max(0, ctr - C::NSTAGE); k < ctr; ++k)
           (void)mbar_wait_bounded(&full[k % C::NSTAGE], (k / C::NSTAGE) & 1, 1000000000ll);
+        if (C::QSM && nq > 0) (void)mbar_wait_bounded(qfull, (nq - 1) & 1, 1000000000ll);
       }
     }
     __syncthreads();
@@ -828,8 +861,15 @@ __global__ void __launch_bounds__(160, 2) attn_kernel(Cache c, AttnLaunch a, int
     }
     const int unit = uq[k % C::UQ];
     if (named_barrier_or(2, 128, unit < 0 || *abort_flag != 0)) break;   // the end, or an abort
-    const Unit u = make_unit<D, GP, CI8>(c, a.r, splits, unit);
+    const Unit u = make_unit<D, GP, CI8>(c, a.r, splits, unit, uqn[k % C::UQ]);
     const unsigned char* qf = a.qfrag + (size_t)u.s * a.qf_stride;
+    if constexpr (C::QSM) {
+      if (!mbar_wait_bounded(qfull, k & 1)) {
+        set_error(c.err, kErrDevice);
+        *abort_flag = 1;
+      }
+      qf = qsm;
+    }
     uint2 qi[C::KB][C::NB];
     float cq8[C::HPL];
     if constexpr (CI8) {
@@ -844,6 +884,10 @@ __global__ void __launch_bounds__(160, 2) attn_kernel(Cache c, AttnLaunch a, int
     uint2 qh[C::KS];
 #pragma unroll
     for (int ks = 0; ks < C::KS; ++ks) qh[ks] = reinterpret_cast<const uint2*>(qf + Q::H_OFF)[ks * 32 + lane];
+    if constexpr (C::QSM) {
+      __syncwarp();   // every lane of the warp has read the slot
+      if (lane == 0) mbar_arrive(qempty);
+    }
 
     SoftmaxState<D, GP> st;
 #pragma unroll
@@ -1055,27 +1099,11 @@ cudaError_t run_attn(const Cache& c, const Policy& pol, const AttnLaunch& a, cud
     combine_kernel<D><<<(warps * 32 + 255) / 256, 256, 0, st>>>(c, a, splits);
     ++*launches;
   }
-  if (pol.mode == 0) {
-    // The EMA pass only feeds eviction, so it can run beside whatever the
-    // caller issues next (the confidence reduction); eviction, the next
-    // append and prefill wait for ema_done.
-    cudaStream_t es = st;
-    if (a.ema_stream != nullptr) {
-      e = cudaEventRecord(a.attn_done, st);
-      if (e == cudaSuccess) e = cudaStreamWaitEvent(a.ema_stream, a.attn_done, 0);
-      if (e != cudaSuccess) return e;
-      es = a.ema_stream;
-    }
-    {
-      ProfScope ps(prof, kKEma, es);
-      e = run_ema(c, pol, a, es);
-      if (e != cudaSuccess) return e;
-    }
+  if (pol.mode == 0 && a.run_ema) {
+    ProfScope ps(prof, kKEma, st);
+    e = run_ema(c, pol, a, st);
+    if (e != cudaSuccess) return e;
     ++*launches;
-    if (a.ema_stream != nullptr) {
-      e = cudaEventRecord(a.ema_done, es);
-      if (e != cudaSuccess) return e;
-    }
   }
   return cudaGetLastError();
 }

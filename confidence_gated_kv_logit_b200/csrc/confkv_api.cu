@@ -81,17 +81,15 @@ struct confkv_handle {
   confkv::EvictCand* cand;       // [S] eviction candidates from the EMA pass
   uint32_t* kscratch;            // evict scratch, per CTA of the largest evict grid
   int* sched;                    // attention unit counters (zero between launches)
-  cudaStream_t ema_stream;       // side stream of the EMA pass
-  cudaEvent_t attn_done;
-  // Completion of the EMA passes, per layer: layer_ev[l] indexes the ring
-  // event recorded after the last EMA pass over layer l (-1: none yet). A
-  // call waits only for the passes of its own layers, so per-layer calls do
-  // not queue behind the previous layer's pass. Ring slots are reused oldest
-  // first; a reused slot completes after the pass it replaced (one side
-  // stream), so waiting on it is never too early.
-  std::vector<cudaEvent_t> ema_ev;
-  std::vector<int> layer_ev;
-  int ev_next = 0;
+  int* bulk_sched;               // bulk eviction segment counters (zero between launches)
+  // The EMA pass of a decode call is deferred (unless single_stream): the
+  // next eviction of the same layers runs it fused into the eviction kernel
+  // (one launch, no candidate records). Anything else that needs the EMA
+  // values first -- another decode call over those layers, export, query --
+  // runs the pass on its own; prefill drops it (the segment starts over).
+  std::vector<char> ema_pending;   // per layer
+  cudaEvent_t attn_done;           // recorded after each deferred decode call's attention
+  cudaStream_t attn_stream;        // the stream it was recorded on
   int scratch_stride;
   int32_t* keep_list;
   int32_t* keep_count;
@@ -315,6 +313,7 @@ confkv_status confkv_create(int32_t layers, int32_t kv_heads, int32_t q_heads, i
   chk(B.alloc(&h->qfrag, S * (size_t)h->qf_stride));
   chk(B.alloc(&h->cand, S));
   chk(B.alloc(&h->sched, 2));
+  chk(B.alloc(&h->bulk_sched, 2));
   h->scratch_stride = 3 * c.cap + c.Wst;
   chk(B.alloc(&h->kscratch, (size_t)confkv::evict_grid((int)S) * h->scratch_stride));
   if (p.mode == CONFKV_MODE_FIXED) {
@@ -346,6 +345,7 @@ confkv_status confkv_create(int32_t layers, int32_t kv_heads, int32_t q_heads, i
     chk(cudaMemset(h->qfrag, 0, S * (size_t)h->qf_stride));
     chk(cudaMemset(h->cand, 0xff, S * sizeof(confkv::EvictCand)));   // stamp -1: no record
     chk(cudaMemset(h->sched, 0, 2 * sizeof(int)));
+    chk(cudaMemset(h->bulk_sched, 0, 2 * sizeof(int)));
     chk(cudaDeviceSynchronize());
   }
   if (e != cudaSuccess) {
@@ -354,28 +354,10 @@ confkv_status confkv_create(int32_t layers, int32_t kv_heads, int32_t q_heads, i
     delete h;
     return cuda_status(e);
   }
-  h->ema_stream = nullptr;
   h->attn_done = nullptr;
-  // The EMA pass gets the device's highest stream priority: it and the
-  // caller's next kernel (the confidence reduction) become ready together
-  // when attention ends, and the EMA's long-segment warps should start first,
-  // with the other kernel filling the SM slots its short segments free.
-  int prio_least = 0, prio_greatest = 0;
-  if (cudaDeviceGetStreamPriorityRange(&prio_least, &prio_greatest) != cudaSuccess) prio_greatest = 0;
-  h->layer_ev.assign(layers, -1);
-  bool ev_ok = true;
-  if (!p.single_stream) {   // single stream: no side stream and no events (capturable calls)
-    h->ema_ev.assign(2 * (size_t)layers + 2, nullptr);
-    ev_ok = cudaStreamCreateWithPriority(&h->ema_stream, cudaStreamNonBlocking, prio_greatest) == cudaSuccess &&
-            cudaEventCreateWithFlags(&h->attn_done, cudaEventDisableTiming) == cudaSuccess;
-    for (cudaEvent_t& ev : h->ema_ev)
-      ev_ok = ev_ok && cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) == cudaSuccess;
-  }
-  if (!ev_ok) {
-    if (h->ema_stream) cudaStreamDestroy(h->ema_stream);
-    if (h->attn_done) cudaEventDestroy(h->attn_done);
-    for (cudaEvent_t ev : h->ema_ev)
-      if (ev) cudaEventDestroy(ev);
+  h->attn_stream = nullptr;
+  h->ema_pending.assign(layers, 0);
+  if (!p.single_stream && cudaEventCreateWithFlags(&h->attn_done, cudaEventDisableTiming) != cudaSuccess) {
     B.release();
     h->magic = kDead;
     delete h;
@@ -389,18 +371,64 @@ confkv_status confkv_create(int32_t layers, int32_t kv_heads, int32_t q_heads, i
   return CONFKV_OK;
 }
 
-// Make `st` wait for the last EMA pass over every layer of r.
-static cudaError_t wait_ema(confkv_handle* h, const confkv::Range& r, cudaStream_t st) {
-  if (h->ema_stream == nullptr) return cudaSuccess;   // single stream: stream order suffices
-  int last = -1;
-  for (int l = r.l0; l < r.l0 + r.nl; ++l) {
-    const int k = h->layer_ev[l];
-    if (k < 0 || k == last) continue;   // consecutive layers of one call share their event
-    const cudaError_t e = cudaStreamWaitEvent(st, h->ema_ev[k], 0);
-    if (e != cudaSuccess) return e;
-    last = k;
+static confkv::AttnLaunch ema_launch(const confkv_handle* h, int l0, int nl) {
+  confkv::AttnLaunch a;
+  std::memset(&a, 0, sizeof(a));
+  a.r.l0 = l0;
+  a.r.nl = nl;
+  a.r.B = h->batch;
+  a.lse_ws = h->lse_ws;
+  a.scores = h->scores;
+  a.score_stride = h->score_stride;
+  a.num_sms = h->num_sms;
+  a.cand = h->cand;
+  return a;
+}
+
+// Order st after the attention whose EMA pass was deferred (a no-op on the
+// stream that ran it).
+static cudaError_t join_attention(confkv_handle* h, cudaStream_t st) {
+  if (h->attn_done == nullptr || st == h->attn_stream) return cudaSuccess;
+  return cudaStreamWaitEvent(st, h->attn_done, 0);
+}
+
+// Run the deferred EMA passes of the layers in [l0, l0 + nl) on st, one
+// launch per run of consecutive pending layers. st first waits for the
+// attention that produced them (it may have run on another stream).
+static cudaError_t flush_ema(confkv_handle* h, int l0, int nl, cudaStream_t st) {
+  bool any = false;
+  for (int l = l0; l < l0 + nl; ++l) any = any || h->ema_pending[l];
+  if (!any) return cudaSuccess;
+  cudaError_t e = join_attention(h, st);
+  for (int l = l0; l < l0 + nl && e == cudaSuccess;) {
+    if (!h->ema_pending[l]) {
+      ++l;
+      continue;
+    }
+    int l1 = l;
+    while (l1 < l0 + nl && h->ema_pending[l1]) ++l1;
+    const confkv::AttnLaunch a = ema_launch(h, l, l1 - l);
+    {
+      confkv::ProfScope ps(h->prof_ptr(), confkv::kKEma, st);
+      e = confkv::run_ema(h->c, h->pol, a, st);
+    }
+    ++h->launches;
+    for (int k = l; k < l1; ++k) h->ema_pending[k] = 0;
+    l = l1;
   }
-  return cudaSuccess;
+  return e;
+}
+
+// Every deferred pass, for the synchronising queries: after the device is
+// idle, on the legacy stream, then idle again.
+static cudaError_t flush_all_ema(confkv_handle* h) {
+  bool any = false;
+  for (char f : h->ema_pending) any = any || f;
+  if (!any) return cudaSuccess;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = flush_ema(h, 0, h->L, nullptr);
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  return e;
 }
 
 confkv_status confkv_destroy(confkv_handle* h) {
@@ -410,10 +438,7 @@ confkv_status confkv_destroy(confkv_handle* h) {
     if (g_live.erase(h) == 0) return CONFKV_ERR_STATE;
   }
   cudaDeviceSynchronize();
-  if (h->ema_stream) cudaStreamDestroy(h->ema_stream);
   if (h->attn_done) cudaEventDestroy(h->attn_done);
-  for (cudaEvent_t ev : h->ema_ev)
-    if (ev) cudaEventDestroy(ev);
   h->buf.release();
   h->magic = kDead;
   delete h;
@@ -438,6 +463,7 @@ confkv_status confkv_prefill(confkv_handle* h, int32_t layer, int32_t batch, con
   if (batch != h->batch) {
     // a new batch: every layer must be ingested again, budgets start at the larger one
     std::fill(h->prefilled.begin(), h->prefilled.end(), 0);
+    std::fill(h->ema_pending.begin(), h->ema_pending.end(), 0);
     h->batch = batch;
     std::vector<int32_t> init((size_t)batch * h->L);
     for (int b = 0; b < batch; ++b)
@@ -453,7 +479,8 @@ confkv_status confkv_prefill(confkv_handle* h, int32_t layer, int32_t batch, con
   layer_range(h, layer, &r);
   cudaError_t e = cudaMemcpyAsync(h->lens_dev, lens_host, (size_t)batch * 4, cudaMemcpyHostToDevice, st);
   if (e != cudaSuccess) return CONFKV_ERR_CUDA;
-  if (wait_ema(h, r, st) != cudaSuccess) return CONFKV_ERR_CUDA;
+  // a deferred EMA pass of these layers is moot: their segments start over
+  for (int l = r.l0; l < r.l0 + r.nl; ++l) h->ema_pending[l] = 0;
   confkv::PrefillLaunch a;
   a.r = r;
   a.lens = h->lens_dev;
@@ -534,19 +561,20 @@ confkv_status confkv_decode_attn(confkv_handle* h, int32_t layer, const void* q,
   a.qf_stride = h->qf_stride;
   a.cand = h->cand;
   a.sched = h->sched;
-  a.ema_stream = h->ema_stream;
-  a.attn_done = h->attn_done;
-  const int ev = h->ev_next;
-  a.ema_done = h->ema_stream != nullptr ? h->ema_ev[ev] : nullptr;
-  // the previous EMA pass over these layers must be done before this step
-  // rewrites their scores and EMA values
-  if (wait_ema(h, r, static_cast<cudaStream_t>(stream)) != cudaSuccess) return CONFKV_ERR_CUDA;
-  cudaError_t e =
-      confkv::launch_decode_attn(h->c, h->pol, a, static_cast<cudaStream_t>(stream), &h->launches, h->prof_ptr());
+  const bool defer = h->pol.mode == 0 && !h->p.single_stream;
+  a.run_ema = (h->pol.mode == 0 && !defer) ? 1 : 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // a pass still deferred from the previous call over these layers reads the
+  // scores this call is about to overwrite: run it first
+  cudaError_t e = flush_ema(h, r.l0, r.nl, st);
   if (e != cudaSuccess) return cuda_status(e);
-  if (h->pol.mode == 0 && h->ema_stream != nullptr) {   // an EMA pass ran on the side stream and recorded ema_ev[ev]
-    for (int l = r.l0; l < r.l0 + r.nl; ++l) h->layer_ev[l] = ev;
-    h->ev_next = (ev + 1) % (int)h->ema_ev.size();
+  e = confkv::launch_decode_attn(h->c, h->pol, a, st, &h->launches, h->prof_ptr());
+  if (e != cudaSuccess) return cuda_status(e);
+  if (defer) {
+    e = cudaEventRecord(h->attn_done, st);
+    if (e != cudaSuccess) return cuda_status(e);
+    h->attn_stream = st;
+    for (int l = r.l0; l < r.l0 + r.nl; ++l) h->ema_pending[l] = 1;
   }
   for (int l = r.l0; l < r.l0 + r.nl; ++l) h->ub_len[l] += 1;
   return CONFKV_OK;
@@ -569,10 +597,31 @@ confkv_status confkv_evict_compact(confkv_handle* h, int32_t layer, void* stream
   a.kscratch = h->kscratch;
   a.scratch_stride = h->scratch_stride;
   a.scratch_keys = h->c.cap + h->c.Wst;
-  // the candidates and EMA values come from the EMA passes on the side stream
-  if (wait_ema(h, r, static_cast<cudaStream_t>(stream)) != cudaSuccess) return CONFKV_ERR_CUDA;
-  cudaError_t e =
-      confkv::launch_evict_compact(h->c, h->pol, a, static_cast<cudaStream_t>(stream), &h->launches, h->prof_ptr());
+  a.bulk_sched = h->bulk_sched;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // Every layer of the call has its EMA pass deferred (the steady decode
+  // step): the eviction kernel runs it fused. Otherwise the deferred passes
+  // run on their own first and eviction reads their candidate records.
+  bool all_pending = h->pol.mode == 0;
+  for (int l = r.l0; l < r.l0 + r.nl; ++l) all_pending = all_pending && h->ema_pending[l];
+  cudaError_t e = cudaSuccess;
+  confkv::EmaIn ein{h->lse_ws, h->scores, h->score_stride};
+  if (all_pending) {
+    // a segment may hold more than even the largest budget allows by more
+    // than the warp path takes (the first step after a long prompt, or after
+    // skipped evictions): the bulk-shaped variant
+    bool bulk = false;
+    for (int l = r.l0; l < r.l0 + r.nl; ++l) bulk = bulk || h->ub_len[l] > h->max_eff[l] + confkv::kWarpMaxVictims;
+    e = join_attention(h, st);
+    if (e == cudaSuccess)
+      e = confkv::launch_evict_compact(h->c, h->pol, a, &ein, bulk, h->num_sms, st, &h->launches, h->prof_ptr());
+    if (e == cudaSuccess)
+      for (int l = r.l0; l < r.l0 + r.nl; ++l) h->ema_pending[l] = 0;
+  } else {
+    e = flush_ema(h, r.l0, r.nl, st);
+    if (e == cudaSuccess)
+      e = confkv::launch_evict_compact(h->c, h->pol, a, nullptr, false, h->num_sms, st, &h->launches, h->prof_ptr());
+  }
   if (e != cudaSuccess) return cuda_status(e);
   for (int l = r.l0; l < r.l0 + r.nl; ++l) h->ub_len[l] = std::min<long long>(h->ub_len[l], h->max_eff[l]);
   return CONFKV_OK;
@@ -582,7 +631,8 @@ confkv_status confkv_query(confkv_handle* h, confkv_stats* out) {
   if (!alive(h)) return CONFKV_ERR_STATE;
   if (!out) return CONFKV_ERR_ARG;
   std::memset(out, 0, sizeof(*out));
-  cudaError_t e = cudaDeviceSynchronize();
+  cudaError_t e = flush_all_ema(h);
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return CONFKV_ERR_CUDA;
   const confkv::Cache& c = h->c;
   unsigned long long cnt[confkv::kNumCounters];
@@ -635,7 +685,8 @@ confkv_status confkv_export_segment(confkv_handle* h, int32_t layer, int32_t seq
     return CONFKV_ERR_ARG;
   const confkv::Cache& c = h->c;
   const size_t s = ((size_t)layer * c.Bmax + seq) * c.Hkv + kv_head;
-  cudaError_t e = cudaDeviceSynchronize();
+  cudaError_t e = flush_all_ema(h);
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return CONFKV_ERR_CUDA;
   int32_t hdr[8] = {0, c.W, 0, c.cold_int8, c.D, h->p.mode, 0, 0};
   e = cudaMemcpy(&hdr[0], c.n_cold + s, 4, cudaMemcpyDeviceToHost);

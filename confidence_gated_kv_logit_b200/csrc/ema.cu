@@ -4,11 +4,15 @@
 // eviction key is computed from the new value, and the segment's kCandMax
 // smallest keys go to its candidate record for the eviction kernel.
 //
+// In the steady decode step the pass runs inside the eviction kernel (its
+// fused variant, evict.cu), which evicts straight from the merged keys. The
+// kernels here run it on its own, when something needs the EMA values before
+// the next eviction (or a handle runs every pass inside its decode call):
+//
 //   ema_kernel     : one warp per segment, eight segments per CTA (calls over
-//                    many segments, e.g. all layers at once). Each lane takes
-//                    four consecutive tokens per 128 with 16-byte loads of the
-//                    G score rows, the EMA values and the positions, two such
-//                    groups in flight at a time.
+//                    many segments, e.g. all layers at once): the pass of
+//                    ema_warp.cuh, whose merged keys become the segment's
+//                    candidate record.
 //   ema_cta_kernel : one CTA of four warps per segment (calls over few
 //                    segments, e.g. one layer: four warps each still fit in
 //                    one wave and shorten the longest segment's chain of
@@ -17,6 +21,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "ema_warp.cuh"
 #include "warp_select.cuh"
 
 namespace confkv {
@@ -25,125 +30,29 @@ namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-template <int G>
-__device__ __forceinline__ float4 ema_update4(const float* __restrict__ sb, int stride, int col, float4 e,
-                                              const float (&lse)[G], const Policy& pol) {
-  float sum[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    const float4 v = *reinterpret_cast<const float4*>(sb + (size_t)g * stride + col);   // log2 units
-    sum[0] += ex2(v.x - lse[g]);
-    sum[1] += ex2(v.y - lse[g]);
-    sum[2] += ex2(v.z - lse[g]);
-    sum[3] += ex2(v.w - lse[g]);
-  }
-  const float invG = 1.0f / G;
-  e.x = fmaf(pol.beta, e.x, pol.one_minus_beta * (sum[0] * invG));
-  e.y = fmaf(pol.beta, e.y, pol.one_minus_beta * (sum[1] * invG));
-  e.z = fmaf(pol.beta, e.z, pol.one_minus_beta * (sum[2] * invG));
-  e.w = fmaf(pol.beta, e.w, pol.one_minus_beta * (sum[3] * invG));
-  return e;
-}
-
-// The pass also computes every token's eviction key from its new EMA value
-// and leaves the segment's kCandMax smallest keys, with the window slot count,
-// in a.cand for the eviction kernel (which then need not rescan the segment).
-template <int G>
+// One warp per segment; the pass itself is ema_segment_warp (ema_warp.cuh).
+// Its merged keys become the segment's candidate record for the eviction
+// kernel (which then need not rescan the segment).
+template <int GMAX>
 __global__ void __launch_bounds__(256) ema_kernel(Cache c, AttnLaunch a, Policy pol) {
   const int lane = threadIdx.x & 31;
   const int item = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (item >= a.r.items(c.Hkv)) return;
   int l, b, h;
   const int s = seg_of(c, a.r, item, &l, &b, &h);
-  float lse[G];
-#pragma unroll
-  for (int g = 0; g < G; ++g) lse[g] = a.lse_ws[(size_t)s * G + g] * kLog2e;   // log2 units, like the scores
-  const int n_cold = c.n_cold[s];
-  const int t = c.next_pos[s] - 1;
-  if (!(n_cold >= 0 && n_cold <= c.cap)) {
-    if (lane == 0) record_violation(c.err, kSiteEmaSeg, s, n_cold);
-    return;
-  }
-  const float* sb = a.scores + (size_t)s * G * a.score_stride;
-  float* scc = c.sc_c + (size_t)s * c.cap;
-  const int32_t* pc = c.pos_c + (size_t)s * c.cap;
-  LaneBest best;
-  best.init();
-  const bool use_bound = pol.one_minus_alpha >= 0x1p-60f;
-  const float t1_over_oma = use_bound ? (float)(t + 1) / pol.one_minus_alpha : 0.0f;
-  auto offer = [&](int pos, float ema, int idx) {
-    if (pos + 1 > best.pos_bound) return;
-    if (t - pos < pol.P || pos < pol.n_sink) return;   // protected: never a victim
-    best.offer(rank_key(pol, ema, pos, t), idx);
-    if (use_bound) best.update_bound(t1_over_oma);
-  };
-  // cold region [0, n_cold): the region and the score rows are multiples of 64
-  // long. A group of four whose smallest position is past the lane's bound
-  // offers nothing (one test for the group: the common case once the lane's
-  // list is full).
-  for (int base = 0; base < n_cold; base += 256) {
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int i0 = base + 128 * u + 4 * lane;
-      if (i0 + 3 < n_cold) {
-        const float4 e = ema_update4<G>(sb, a.score_stride, i0, *reinterpret_cast<const float4*>(scc + i0), lse, pol);
-        const int4 p4 = *reinterpret_cast<const int4*>(pc + i0);
-        *reinterpret_cast<float4*>(scc + i0) = e;
-        if (min(min(p4.x, p4.y), min(p4.z, p4.w)) + 1 <= best.pos_bound) {
-          offer(p4.x, e.x, i0);
-          offer(p4.y, e.y, i0 + 1);
-          offer(p4.z, e.z, i0 + 2);
-          offer(p4.w, e.w, i0 + 3);
-        }
-      } else if (i0 < n_cold) {   // the last, partial group
-        const float4 e = ema_update4<G>(sb, a.score_stride, i0, *reinterpret_cast<const float4*>(scc + i0), lse, pol);
-        const int4 p4 = *reinterpret_cast<const int4*>(pc + i0);
-        scc[i0] = e.x;
-        offer(p4.x, e.x, i0);
-        if (i0 + 1 < n_cold) {
-          scc[i0 + 1] = e.y;
-          offer(p4.y, e.y, i0 + 1);
-        }
-        if (i0 + 2 < n_cold) {
-          scc[i0 + 2] = e.z;
-          offer(p4.z, e.z, i0 + 2);
-        }
-      }
-    }
-  }
-  // window ring: occupied slots only (the ring stride is a multiple of 64)
-  const int32_t* pr = c.pos_r + (size_t)s * c.Wst;
-  float* scr = c.sc_r + (size_t)s * c.Wst;
-  int ring_here = 0;
-  for (int s0 = 4 * lane; s0 < c.W; s0 += 128) {
-    const int4 p4 = *reinterpret_cast<const int4*>(pr + s0);
-    const float4 e = ema_update4<G>(sb, a.score_stride, c.cap + s0, *reinterpret_cast<const float4*>(scr + s0), lse, pol);
-    const int pp[4] = {p4.x, p4.y, p4.z, p4.w};
-    const float ee[4] = {e.x, e.y, e.z, e.w};
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      if (s0 + q < c.W && pp[q] >= 0) {
-        scr[s0 + q] = ee[q];
-        ++ring_here;
-        offer(pp[q], ee[q], n_cold + s0 + q);
-      }
-    }
-  }
-  if (a.cand == nullptr) return;
-  const int n_ring = __reduce_add_sync(0xffffffffu, ring_here);
-  unsigned long long mk;
-  int mi, cnt, safe;
-  warp_merge_smallest(best, lane, kCandMax, &mk, &mi, &cnt, &safe);
+  EmaOut o;
+  ema_segment_warp<GMAX>(c, EmaIn{a.lse_ws, a.scores, a.score_stride}, pol, s, lane, &o);
+  if (!o.ok || a.cand == nullptr) return;
   EvictCand* cd = a.cand + s;
   if (lane < kCandMax) {
-    cd->key[lane] = mk;
-    cd->idx[lane] = mi;
+    cd->key[lane] = o.key;
+    cd->idx[lane] = o.idx;
   }
   if (lane == 0) {
-    cd->n_ring = n_ring;
-    cd->safe = safe;
-    cd->n_cold = n_cold;
-    cd->stamp = t + 1;
+    cd->n_ring = o.n_ring;
+    cd->safe = o.safe;
+    cd->n_cold = o.n_cold;
+    cd->stamp = o.t + 1;
   }
 }
 
@@ -157,7 +66,7 @@ constexpr int kCtaThreads = 32 * kCtaWarps;
 constexpr int kWarpWant = 8;
 static_assert(kCtaWarps * kWarpWant == 32, "the final merge holds one key per lane");
 
-template <int G>
+template <int GMAX>
 __global__ void __launch_bounds__(kCtaThreads, 8) ema_cta_kernel(Cache c, AttnLaunch a, Policy pol) {
   __shared__ unsigned long long w_key[kCtaWarps * kWarpWant];
   __shared__ int w_idx[kCtaWarps * kWarpWant];
@@ -166,9 +75,11 @@ __global__ void __launch_bounds__(kCtaThreads, 8) ema_cta_kernel(Cache c, AttnLa
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int l, b, h;
   const int s = seg_of(c, a.r, blockIdx.x, &l, &b, &h);
-  float lse[G];
+  const int G = c.G;
+  const float invG = 1.0f / (float)G;
+  float lse[GMAX];
 #pragma unroll
-  for (int g = 0; g < G; ++g) lse[g] = a.lse_ws[(size_t)s * G + g] * kLog2e;   // log2 units, like the scores
+  for (int g = 0; g < GMAX; ++g) lse[g] = g < G ? a.lse_ws[(size_t)s * G + g] * kLog2e : 0.0f;   // log2 units
   const int n_cold = c.n_cold[s];
   const int t = c.next_pos[s] - 1;
   if (!(n_cold >= 0 && n_cold <= c.cap)) {   // the same answer in every thread of the CTA
@@ -194,7 +105,7 @@ __global__ void __launch_bounds__(kCtaThreads, 8) ema_cta_kernel(Cache c, AttnLa
     for (int u = 0; u < 2; ++u) {
       const int i0 = base + 4 * kCtaThreads * u + 4 * tid;
       if (i0 + 3 < n_cold) {
-        const float4 e = ema_update4<G>(sb, a.score_stride, i0, *reinterpret_cast<const float4*>(scc + i0), lse, pol);
+        const float4 e = ema_update4<GMAX>(sb, a.score_stride, i0, *reinterpret_cast<const float4*>(scc + i0), lse, G, invG, pol);
         const int4 p4 = *reinterpret_cast<const int4*>(pc + i0);
         *reinterpret_cast<float4*>(scc + i0) = e;
         if (min(min(p4.x, p4.y), min(p4.z, p4.w)) + 1 <= best.pos_bound) {
@@ -204,7 +115,7 @@ __global__ void __launch_bounds__(kCtaThreads, 8) ema_cta_kernel(Cache c, AttnLa
           offer(p4.w, e.w, i0 + 3);
         }
       } else if (i0 < n_cold) {   // the last, partial group
-        const float4 e = ema_update4<G>(sb, a.score_stride, i0, *reinterpret_cast<const float4*>(scc + i0), lse, pol);
+        const float4 e = ema_update4<GMAX>(sb, a.score_stride, i0, *reinterpret_cast<const float4*>(scc + i0), lse, G, invG, pol);
         const int4 p4 = *reinterpret_cast<const int4*>(pc + i0);
         scc[i0] = e.x;
         offer(p4.x, e.x, i0);
@@ -225,7 +136,7 @@ __global__ void __launch_bounds__(kCtaThreads, 8) ema_cta_kernel(Cache c, AttnLa
   int ring_here = 0;
   for (int s0 = 4 * tid; s0 < c.W; s0 += 4 * kCtaThreads) {
     const int4 p4 = *reinterpret_cast<const int4*>(pr + s0);
-    const float4 e = ema_update4<G>(sb, a.score_stride, c.cap + s0, *reinterpret_cast<const float4*>(scr + s0), lse, pol);
+    const float4 e = ema_update4<GMAX>(sb, a.score_stride, c.cap + s0, *reinterpret_cast<const float4*>(scr + s0), lse, G, invG, pol);
     const int pp[4] = {p4.x, p4.y, p4.z, p4.w};
     const float ee[4] = {e.x, e.y, e.z, e.w};
 #pragma unroll
@@ -287,30 +198,22 @@ __global__ void __launch_bounds__(kCtaThreads, 8) ema_cta_kernel(Cache c, AttnLa
   }
 }
 
-template <int G>
+template <int GMAX>
 void launch_ema(const Cache& c, const Policy& pol, const AttnLaunch& a, cudaStream_t st) {
   const int items = a.r.items(c.Hkv);
   // four warps per segment while they fit in one wave (about 32 warps per SM)
   if ((long long)items * kCtaWarps <= (long long)a.num_sms * 32)
-    ema_cta_kernel<G><<<items, kCtaThreads, 0, st>>>(c, a, pol);
+    ema_cta_kernel<GMAX><<<items, kCtaThreads, 0, st>>>(c, a, pol);
   else
-    ema_kernel<G><<<(items + 7) / 8, 256, 0, st>>>(c, a, pol);
+    ema_kernel<GMAX><<<(items + 7) / 8, 256, 0, st>>>(c, a, pol);
 }
 
 }  // namespace
 
 cudaError_t run_ema(const Cache& c, const Policy& pol, const AttnLaunch& a, cudaStream_t st) {
-  switch (c.G) {
-    case 1: launch_ema<1>(c, pol, a, st); break;
-    case 2: launch_ema<2>(c, pol, a, st); break;
-    case 3: launch_ema<3>(c, pol, a, st); break;
-    case 4: launch_ema<4>(c, pol, a, st); break;
-    case 5: launch_ema<5>(c, pol, a, st); break;
-    case 6: launch_ema<6>(c, pol, a, st); break;
-    case 7: launch_ema<7>(c, pol, a, st); break;
-    case 8: launch_ema<8>(c, pol, a, st); break;
-    default: return cudaErrorInvalidValue;
-  }
+  if (c.G < 1 || c.G > 8) return cudaErrorInvalidValue;
+  if (c.G <= 4) launch_ema<4>(c, pol, a, st);
+  else launch_ema<8>(c, pol, a, st);
   return cudaGetLastError();
 }
 

@@ -22,8 +22,15 @@
 //      first hole down in order. Both leave the same logical content.
 //   4. the token that the next append would push out of the window
 //      (position t+1-W) is quantised into the end of the cold region.
+//
+// The fused variant (the steady decode step in confidence mode) first runs
+// the step's attention-mass EMA pass over the warp's segment (ema_warp.cuh)
+// and takes the victims of step 2 from the keys that pass merged, in
+// registers; segments with more victims go to the whole-CTA path as above,
+// which reads the EMA values the pass has just written.
 #include "common.cuh"
 #include "kernels.h"
+#include "ema_warp.cuh"
 #include "select.cuh"
 #include "warp_select.cuh"
 
@@ -117,7 +124,7 @@ struct WarpCounts {
 // ints of shared memory owned by this warp.
 template <int D, bool CI8>
 __device__ bool evict_segment_warp(const Cache& c, const Policy& pol, const EvictLaunch& a, int item, int lane,
-                                   WarpCounts* wc, int* ws_pairs) {
+                                   WarpCounts* wc, int* ws_pairs, const EmaOut* fused = nullptr) {
   using R = Rows<D, CI8>;
   int l, b, h;
   const int s = seg_of(c, a.r, item, &l, &b, &h);
@@ -164,7 +171,7 @@ __device__ bool evict_segment_warp(const Cache& c, const Policy& pol, const Evic
   int4 hdr = make_int4(0, 0, -1, -1);                 // n_ring, safe, stamp, n_cold
   unsigned long long rec_key = kNoKey;
   int rec_idx = -1;
-  if (cd != nullptr) {
+  if (cd != nullptr && fused == nullptr) {
     hdr = *reinterpret_cast<const int4*>(&cd->n_ring);
     if (lane < kCandMax) {
       rec_key = cd->key[lane];
@@ -175,7 +182,15 @@ __device__ bool evict_segment_warp(const Cache& c, const Policy& pol, const Evic
   int n_ring = 0, count = 0, safe = 0;
   unsigned long long my_key = kNoKey;
   int my_idx = -1;
-  if (cd != nullptr && pol.mode == 0 && !a.stable && hdr.z == t + 1 && hdr.w == n_cold) {
+  if (fused != nullptr) {
+    // this kernel's own EMA pass over the segment has just merged its keys
+    have = true;
+    n_ring = fused->n_ring;
+    safe = fused->safe;
+    my_key = lane < kCandMax ? fused->key : kNoKey;
+    my_idx = lane < kCandMax ? fused->idx : -1;
+    count = fused->count;
+  } else if (cd != nullptr && pol.mode == 0 && !a.stable && hdr.z == t + 1 && hdr.w == n_cold) {
     have = true;
     n_ring = hdr.x;
     safe = hdr.y;
@@ -420,9 +435,16 @@ struct EvictSmem {
 
 // One segment by the whole CTA (all NT threads call it with the same item):
 // any number of victims, both compaction orders.
+// Keys already in this CTA's scratch (the bulk variant's EMA pass wrote
+// them): the occupied window slots and this thread's range of counted keys.
+struct BlockKeys {
+  int n_ring;
+  uint32_t kmn, kmx;
+};
+
 template <int D, bool CI8>
 __device__ void evict_segment_block(const Cache& c, const Policy& pol, const EvictLaunch& a, int item,
-                                    EvictSmem& es) {
+                                    EvictSmem& es, const BlockKeys* pre = nullptr) {
   using R = Rows<D, CI8>;
   SelectSmem<NT>& sm = es.sm;
   int* list_h = es.list_h;
@@ -441,9 +463,14 @@ __device__ void evict_segment_block(const Cache& c, const Policy& pol, const Evi
   int32_t* pos_r = c.pos_r + (size_t)s * c.Wst;
   const float* sc_r = c.sc_r + (size_t)s * c.Wst;
 
-  int ring_here = 0;
-  for (int slot = threadIdx.x; slot < W; slot += NT) ring_here += pos_r[slot] >= 0;
-  const int n_ring = block_sum_int<NT>(ring_here, sm);
+  int n_ring;
+  if (pre != nullptr) {
+    n_ring = pre->n_ring;
+  } else {
+    int ring_here = 0;
+    for (int slot = threadIdx.x; slot < W; slot += NT) ring_here += pos_r[slot] >= 0;
+    n_ring = block_sum_int<NT>(ring_here, sm);
+  }
   const int n = n_cold + n_ring;
   const int budget_eff = pol.mode == 1 ? pol.fixed_budget
                                        : max(a.budget[(size_t)b * c.L + l], pol.P + pol.n_sink);
@@ -504,7 +531,11 @@ __device__ void evict_segment_block(const Cache& c, const Policy& pol, const Evi
         kmx = max(kmx, hv);
       }
     };
-    for (int i0 = 8 * threadIdx.x; i0 < n_cold; i0 += 8 * NT) {
+    if (pre != nullptr) {
+      kmn = pre->kmn;
+      kmx = pre->kmx;
+    }
+    for (int i0 = 8 * threadIdx.x; pre == nullptr && i0 < n_cold; i0 += 8 * NT) {
       const int4 p0 = reinterpret_cast<const int4*>(pos_c + i0)[0];
       const int4 p1 = reinterpret_cast<const int4*>(pos_c + i0)[1];
       const float4 f0 = reinterpret_cast<const float4*>(sc_c + i0)[0];
@@ -526,7 +557,7 @@ __device__ void evict_segment_block(const Cache& c, const Policy& pol, const Evi
           if (i0 + j < n_cold) khi[i0 + j] = hv[j];
       }
     }
-    for (int slot = threadIdx.x; slot < W; slot += NT) {
+    for (int slot = threadIdx.x; pre == nullptr && slot < W; slot += NT) {
       const uint32_t hv = hi_of(pos_r[slot], sc_r[slot]);
       khi[n_cold + slot] = hv;
       track(hv);
@@ -692,13 +723,20 @@ __device__ void evict_segment_block(const Cache& c, const Policy& pol, const Evi
     c.n_cold[s] = n_cold_new;
     atomicAdd(&c.counters[kCntEvictBlock], 1ull);
     if (a.cand != nullptr) a.cand[s].stamp = -1;
-    atomicAdd(&c.counters[kCntEvictScanned], (unsigned long long)n);
+    // tokens whose keys this path read from the cache (precomputed keys came
+    // with the EMA pass's own reads)
+    if (pre == nullptr || (e == 1 && !a.stable)) atomicAdd(&c.counters[kCntEvictScanned], (unsigned long long)n);
     if (moved > 0) atomicAdd(&c.counters[kCntMovedRows], (unsigned long long)moved);
   }
 }
 
-template <int D, bool CI8>
-__global__ void __launch_bounds__(NT, 4) evict_kernel(Cache c, Policy pol, EvictLaunch a, int items) {
+// GMAX > 0: the fused variant. Each warp first runs the step's EMA pass over
+// its segment (ema_warp.cuh, the same code as the EMA kernel, for G <= GMAX
+// query heads per KV head) and evicts from the merged keys it leaves in
+// registers: no candidate record, and no separate EMA launch.
+template <int D, bool CI8, int GMAX>
+__global__ void __launch_bounds__(NT, GMAX > 4 ? 3 : 4) evict_kernel(Cache c, Policy pol, EvictLaunch a, EmaIn ein,
+                                                                      int items) {
   __shared__ EvictSmem es;
   __shared__ int slow_items[kSegsPerCta];
   __shared__ int n_slow;
@@ -716,7 +754,18 @@ __global__ void __launch_bounds__(NT, 4) evict_kernel(Cache c, Policy pol, Evict
   const int item = slot < items ? (int)(((unsigned long long)slot * 2654435761ull) % (unsigned long long)items) : items;
   if (item < items) {
     WarpCounts wc;
-    if (!evict_segment_warp<D, CI8>(c, pol, a, item, lane, &wc, pairs[warp])) {
+    bool done;
+    if constexpr (GMAX > 0) {
+      int l, b, h;
+      const int s = seg_of(c, a.r, item, &l, &b, &h);
+      EmaOut eo;
+      ema_segment_warp<GMAX>(c, ein, pol, s, lane, &eo);
+      // a corrupt segment was recorded by the pass; eviction skips it likewise
+      done = !eo.ok || evict_segment_warp<D, CI8>(c, pol, a, item, lane, &wc, pairs[warp], &eo);
+    } else {
+      done = evict_segment_warp<D, CI8>(c, pol, a, item, lane, &wc, pairs[warp]);
+    }
+    if (!done) {
       if (lane == 0) slow_items[atomicAdd(&n_slow, 1)] = item;
     } else if (lane == 0) {
       if (wc.scanned) atomicAdd(&cnt[0], (unsigned long long)wc.scanned);
@@ -737,12 +786,164 @@ __global__ void __launch_bounds__(NT, 4) evict_kernel(Cache c, Policy pol, Evict
   }
 }
 
-template <int D, bool CI8>
-cudaError_t run(const Cache& c, const Policy& pol, const EvictLaunch& a, cudaStream_t st, long long* launches,
-                Prof* prof) {
+// The step's EMA pass over segment s by the whole CTA (the same arithmetic
+// per token as ema_segment_warp), also writing every token's key high half
+// into this CTA's scratch as the whole-CTA eviction path wants it, with each
+// thread's range of counted keys and the occupied window slots. Returns false
+// (recorded) for a corrupt segment.
+template <int GMAX>
+__device__ bool cta_ema_keys(const Cache& c, const EmaIn& in, const Policy& pol, int s, uint32_t* __restrict__ khi,
+                             BlockKeys* bk, SelectSmem<NT>& sm) {
+  constexpr float kLog2eF = 1.4426950408889634f;
+  const int G = c.G;
+  const float invG = 1.0f / (float)G;
+  float lse[GMAX];
+#pragma unroll
+  for (int g = 0; g < GMAX; ++g) lse[g] = g < G ? in.lse_ws[(size_t)s * G + g] * kLog2eF : 0.0f;   // log2 units
+  const int n_cold = c.n_cold[s];
+  const int t = c.next_pos[s] - 1;
+  if (!(n_cold >= 0 && n_cold <= c.cap && t >= -1)) {   // the same answer in every thread
+    if (threadIdx.x == 0) record_violation(c.err, kSiteEmaSeg, s, n_cold);
+    return false;
+  }
+  const float* sb = in.scores + (size_t)s * G * in.score_stride;
+  float* scc = c.sc_c + (size_t)s * c.cap;
+  const int32_t* pc = c.pos_c + (size_t)s * c.cap;
+  auto hi_of = [&](int pos, float sc) -> uint32_t {
+    const bool none = pos < 0 || t - pos < pol.P || pos < pol.n_sink;
+    return none ? 0xFFFFFFFFu : (uint32_t)(rank_key(pol, sc, pos, t) >> 32);
+  };
+  uint32_t kmn = 0xFFFFFFFFu, kmx = 0u;
+  auto track = [&](uint32_t hv) {
+    if (hv != 0xFFFFFFFFu) {
+      kmn = min(kmn, hv);
+      kmx = max(kmx, hv);
+    }
+  };
+  // cold region: four consecutive tokens per thread, two groups in flight
+  for (int base = 0; base < n_cold; base += 8 * NT) {
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int i0 = base + 4 * NT * u + 4 * (int)threadIdx.x;
+      if (i0 + 3 < n_cold) {
+        const float4 e =
+            ema_update4<GMAX>(sb, in.score_stride, i0, *reinterpret_cast<const float4*>(scc + i0), lse, G, invG, pol);
+        const int4 p4 = *reinterpret_cast<const int4*>(pc + i0);
+        *reinterpret_cast<float4*>(scc + i0) = e;
+        const uint4 hv = make_uint4(hi_of(p4.x, e.x), hi_of(p4.y, e.y), hi_of(p4.z, e.z), hi_of(p4.w, e.w));
+        *reinterpret_cast<uint4*>(khi + i0) = hv;
+        track(hv.x);
+        track(hv.y);
+        track(hv.z);
+        track(hv.w);
+      } else if (i0 < n_cold) {   // the last, partial group
+        const float4 e =
+            ema_update4<GMAX>(sb, in.score_stride, i0, *reinterpret_cast<const float4*>(scc + i0), lse, G, invG, pol);
+        const int4 p4 = *reinterpret_cast<const int4*>(pc + i0);
+        const int pp[3] = {p4.x, p4.y, p4.z};
+        const float ee[3] = {e.x, e.y, e.z};
+#pragma unroll
+        for (int q = 0; q < 3; ++q)
+          if (i0 + q < n_cold) {
+            scc[i0 + q] = ee[q];
+            const uint32_t h = hi_of(pp[q], ee[q]);
+            khi[i0 + q] = h;
+            track(h);
+          }
+      }
+    }
+  }
+  // window ring: occupied slots only (the ring stride is a multiple of 64)
+  const int32_t* pr = c.pos_r + (size_t)s * c.Wst;
+  float* scr = c.sc_r + (size_t)s * c.Wst;
+  int ring_here = 0;
+  for (int s0 = 4 * (int)threadIdx.x; s0 < c.W; s0 += 4 * NT) {
+    const int4 p4 = *reinterpret_cast<const int4*>(pr + s0);
+    const float4 e = ema_update4<GMAX>(sb, in.score_stride, c.cap + s0, *reinterpret_cast<const float4*>(scr + s0),
+                                       lse, G, invG, pol);
+    const int pp[4] = {p4.x, p4.y, p4.z, p4.w};
+    const float ee[4] = {e.x, e.y, e.z, e.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (s0 + q < c.W) {
+        uint32_t h = 0xFFFFFFFFu;
+        if (pp[q] >= 0) {
+          scr[s0 + q] = ee[q];
+          ++ring_here;
+          h = hi_of(pp[q], ee[q]);
+        }
+        khi[n_cold + s0 + q] = h;
+        track(h);
+      }
+    }
+  }
+  bk->n_ring = block_sum_int<NT>(ring_here, sm);   // includes a block barrier: the keys are visible
+  bk->kmn = kmn;
+  bk->kmx = kmx;
+  return true;
+}
+
+// The bulk variant of the fused kernel: a persistent grid whose CTAs claim
+// one segment at a time, run its EMA pass with every thread (writing the
+// keys), then evict it by the whole-CTA path. Claiming lets the CTAs of an
+// SM drift apart, so that one streams its segment while another selects.
+template <int D, bool CI8, int GMAX>
+__global__ void __launch_bounds__(NT, 3) evict_bulk_kernel(Cache c, Policy pol, EvictLaunch a, EmaIn ein,
+                                                           int items) {
+  __shared__ EvictSmem es;
+  __shared__ int claimed;
+  uint32_t* khi = a.kscratch + (size_t)blockIdx.x * a.scratch_stride;
+  while (true) {
+    if (threadIdx.x == 0) claimed = atomicAdd(a.bulk_sched, 1);
+    __syncthreads();
+    const int item = claimed;
+    __syncthreads();   // every thread has read it before the next claim
+    if (item >= items) break;
+    int l, b, h;
+    const int s = seg_of(c, a.r, item, &l, &b, &h);
+    BlockKeys bk;
+    if (!cta_ema_keys<GMAX>(c, ein, pol, s, khi, &bk, es.sm)) continue;
+    evict_segment_block<D, CI8>(c, pol, a, item, es, &bk);
+    __syncthreads();
+  }
+  // the last CTA to finish resets the counters for the next launch
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(a.bulk_sched + 1, 1) == (int)gridDim.x - 1) {
+      a.bulk_sched[0] = 0;
+      a.bulk_sched[1] = 0;
+    }
+  }
+}
+
+template <int D, bool CI8, int GMAX>
+cudaError_t run_bulk(const Cache& c, const Policy& pol, const EvictLaunch& a, const EmaIn& ema, int num_sms,
+                     cudaStream_t st) {
   const int items = a.r.items(c.Hkv);
-  ProfScope ps(prof, kKEvict, st);
-  evict_kernel<D, CI8><<<evict_grid(items), NT, 0, st>>>(c, pol, a, items);
+  int per_sm = 0;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, evict_bulk_kernel<D, CI8, GMAX>, NT, 0);
+  if (e != cudaSuccess) return e;
+  // the key scratch exists for evict_grid(items) CTAs
+  const int grid = max(1, min(evict_grid(items), max(1, per_sm) * num_sms));
+  evict_bulk_kernel<D, CI8, GMAX><<<grid, NT, 0, st>>>(c, pol, a, ema, items);
+  return cudaGetLastError();
+}
+
+template <int D, bool CI8>
+cudaError_t run(const Cache& c, const Policy& pol, const EvictLaunch& a, const EmaIn* ema, cudaStream_t st,
+                long long* launches, Prof* prof) {
+  const int items = a.r.items(c.Hkv);
+  const int grid = evict_grid(items);
+  if (ema == nullptr) {
+    ProfScope ps(prof, kKEvict, st);
+    evict_kernel<D, CI8, 0><<<grid, NT, 0, st>>>(c, pol, a, EmaIn{}, items);
+  } else {
+    ProfScope ps(prof, kKEmaEvict, st);
+    if (c.G <= 4)
+      evict_kernel<D, CI8, 4><<<grid, NT, 0, st>>>(c, pol, a, *ema, items);
+    else
+      evict_kernel<D, CI8, 8><<<grid, NT, 0, st>>>(c, pol, a, *ema, items);
+  }
   ++*launches;
   return cudaGetLastError();
 }
@@ -751,12 +952,31 @@ cudaError_t run(const Cache& c, const Policy& pol, const EvictLaunch& a, cudaStr
 
 int evict_grid(int items) { return (items + kSegsPerCta - 1) / kSegsPerCta; }
 
-cudaError_t launch_evict_compact(const Cache& c, const Policy& pol, const EvictLaunch& a, cudaStream_t st,
-                                 long long* launches, Prof* prof) {
+cudaError_t launch_evict_compact(const Cache& c, const Policy& pol, const EvictLaunch& a, const EmaIn* ema,
+                                 bool bulk, int num_sms, cudaStream_t st, long long* launches, Prof* prof) {
   if (a.r.items(c.Hkv) == 0) return cudaSuccess;
+  if (ema != nullptr && (pol.mode != 0 || c.G < 1 || c.G > 8)) return cudaErrorInvalidValue;
+  if (ema != nullptr && bulk) {
+    ProfScope ps(prof, kKEmaEvict, st);
+    cudaError_t e;
+    if (c.D == 128)
+      e = c.cold_int8 ? (c.G <= 4 ? run_bulk<128, true, 4>(c, pol, a, *ema, num_sms, st)
+                                  : run_bulk<128, true, 8>(c, pol, a, *ema, num_sms, st))
+                      : (c.G <= 4 ? run_bulk<128, false, 4>(c, pol, a, *ema, num_sms, st)
+                                  : run_bulk<128, false, 8>(c, pol, a, *ema, num_sms, st));
+    else
+      e = c.cold_int8 ? (c.G <= 4 ? run_bulk<64, true, 4>(c, pol, a, *ema, num_sms, st)
+                                  : run_bulk<64, true, 8>(c, pol, a, *ema, num_sms, st))
+                      : (c.G <= 4 ? run_bulk<64, false, 4>(c, pol, a, *ema, num_sms, st)
+                                  : run_bulk<64, false, 8>(c, pol, a, *ema, num_sms, st));
+    ++*launches;
+    return e;
+  }
   if (c.D == 128)
-    return c.cold_int8 ? run<128, true>(c, pol, a, st, launches, prof) : run<128, false>(c, pol, a, st, launches, prof);
-  return c.cold_int8 ? run<64, true>(c, pol, a, st, launches, prof) : run<64, false>(c, pol, a, st, launches, prof);
+    return c.cold_int8 ? run<128, true>(c, pol, a, ema, st, launches, prof)
+                       : run<128, false>(c, pol, a, ema, st, launches, prof);
+  return c.cold_int8 ? run<64, true>(c, pol, a, ema, st, launches, prof)
+                     : run<64, false>(c, pol, a, ema, st, launches, prof);
 }
 
 }  // namespace confkv

@@ -65,9 +65,7 @@ struct AttnLaunch {
   int qf_stride;
   EvictCand* cand;        // [S] eviction candidates written by the EMA pass (confidence mode)
   int* sched;             // [2] unit counter and finished-CTA counter of the attention kernel (zero between launches)
-  cudaStream_t ema_stream;  // when set, the EMA pass runs there (forked after attention, joined on ema_done)
-  cudaEvent_t attn_done;    // recorded on the caller's stream after attention
-  cudaEvent_t ema_done;     // recorded on ema_stream after the EMA pass
+  int run_ema;            // confidence mode: 1 runs the EMA pass after attention, 0 leaves it to the caller
 };
 cudaError_t launch_decode_attn(const Cache& c, const Policy& pol, const AttnLaunch& a, cudaStream_t st,
                                long long* launches, Prof* prof);
@@ -88,9 +86,22 @@ struct EvictLaunch {
   uint32_t* kscratch;     // per CTA of the evict grid: key high halves [cap + Wst], then hole and mover lists [cap] each
   int scratch_stride;     // uint32 words per CTA
   int scratch_keys;       // offset of the hole list (= cap + Wst)
+  int* bulk_sched;        // [2] segment counter and finished-CTA counter of the bulk variant (zero between launches)
 };
-cudaError_t launch_evict_compact(const Cache& c, const Policy& pol, const EvictLaunch& a, cudaStream_t st,
-                                 long long* launches, Prof* prof);
+// Where an EMA pass reads the step's attention results.
+struct EmaIn {
+  const float* lse_ws;   // [S][G] natural-log LSE of the step
+  const float* scores;   // [S][G][score_stride] scaled scores, log2 units
+  int score_stride;
+};
+// With `ema` set, the eviction kernel first runs the step's EMA pass over
+// each segment (the fused variant; confidence mode only). `bulk` selects the
+// variant for evictions of thousands of tokens per segment (the first step
+// after a long prompt): one segment at a time per CTA, claimed from a
+// counter, the EMA pass spread over the whole CTA and writing the keys the
+// select needs.
+cudaError_t launch_evict_compact(const Cache& c, const Policy& pol, const EvictLaunch& a, const EmaIn* ema,
+                                 bool bulk, int num_sms, cudaStream_t st, long long* launches, Prof* prof);
 // CTAs the evict kernel uses for `items` segments (the scratch is per CTA).
 int evict_grid(int items);
 

@@ -9,7 +9,7 @@
 namespace confkv {
 
 enum KernelKind { kKConfidence = 0, kKAppend = 1, kKAttention = 2, kKCombine = 3, kKEma = 4, kKEvict = 5,
-                  kKPrefill = 6, kNumKinds = 8 };
+                  kKPrefill = 6, kKEmaEvict = 7, kNumKinds = 8 };
 
 struct Prof {
   bool on = false;

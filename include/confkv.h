@@ -104,11 +104,12 @@ typedef struct {
   int32_t max_prefill;   /* longest prompt confkv_prefill accepts (tokens) */
   int32_t score_source;  /* CONFKV_SCORE_EMA, CONFKV_SCORE_ACCUM or CONFKV_SCORE_RANDOM (confidence mode) */
   uint32_t seed;         /* CONFKV_SCORE_RANDOM: seed of the per-token draws */
-  int32_t single_stream; /* nonzero: every kernel of a call runs on the caller's stream (the EMA pass
-                            too, instead of on the handle's side stream joined by events), so that a
-                            caller can capture a whole decode step in a CUDA graph. Launch
-                            configurations are then fixed at capture time, and the handle's host-side
-                            length bounds are not advanced by replays */
+  int32_t single_stream; /* nonzero: every kernel of a call runs inside that call, on the caller's
+                            stream (the EMA pass runs in confkv_decode_attn instead of being deferred
+                            to the next eviction, and no event joins calls), so that a caller can
+                            capture a whole decode step in a CUDA graph. Launch configurations are
+                            then fixed at capture time, and the handle's host-side length bounds are
+                            not advanced by replays */
 } confkv_params;
 
 typedef struct {
@@ -189,7 +190,12 @@ CONFKV_API confkv_status confkv_confidence(confkv_handle* h, const float* logits
  *   lse_out  fp32 [batch][q_heads] (likewise) natural-log log-sum-exp of the
  *          scaled scores; optional
  * Query head h reads KV head h / G. Errors: STATE before prefill, CAPACITY if
- * the cache could overflow (calls without eviction grow it). */
+ * the cache could overflow (calls without eviction grow it).
+ * Unless single_stream is set, the EMA update is deferred: the next
+ * confkv_evict_compact over the same layers runs it inside the eviction kernel
+ * (one launch for both). Whatever reads the cache first -- another decode call
+ * over those layers, confkv_query, confkv_export_segment -- sees it applied;
+ * a prefill of those layers discards it. */
 CONFKV_API confkv_status confkv_decode_attn(confkv_handle* h, int32_t layer, const void* q, const void* k_new,
                                  const void* v_new, const float* prio_new, float* out, float* lse_out,
                                  void* stream);
@@ -240,7 +246,9 @@ CONFKV_API confkv_status confkv_last_error_detail(confkv_handle* h, int32_t* det
  * milliseconds since the last reset. */
 enum {
   CONFKV_K_CONFIDENCE = 0, CONFKV_K_APPEND = 1, CONFKV_K_ATTENTION = 2, CONFKV_K_COMBINE = 3,
-  CONFKV_K_EMA = 4, CONFKV_K_EVICT = 5, CONFKV_K_PREFILL = 6, CONFKV_K_KINDS = 8
+  CONFKV_K_EMA = 4, CONFKV_K_EVICT = 5, CONFKV_K_PREFILL = 6,
+  CONFKV_K_EMA_EVICT = 7,   /* the eviction kernel with the step's EMA pass fused in */
+  CONFKV_K_KINDS = 8
 };
 typedef struct {
   int64_t launches[CONFKV_K_KINDS];

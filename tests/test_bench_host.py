@@ -56,19 +56,26 @@ def test_workload_names_mark_the_variants():
 
 
 def test_block_compaction_replay_counts_moved_rows():
-    # blocks of 4 slots: positions 0..7 fill blocks 0 and 1; then 0, 1, 2 are
-    # evicted and 8 arrives. Block 0 keeps 1 live token (< 0.5 x 4), so it is
-    # compacted: its one row moves to the tail (block 2, which 8 opened).
+    # blocks of 4 slots by position: 0..7 fill blocks 0 and 1 (block 1 is the
+    # tail); then 0, 1, 2 are evicted and 8 arrives (a new tail, block 2).
+    # Block 0 keeps 1 live token (< 0.5 x 4): its row moves to the tail.
     hist = [[np.arange(8), np.array([3, 4, 5, 6, 7, 8])]]
     r = bench.block_compaction_study(hist, (4,), (0.5,), row_bytes=100)["block_4_theta_0.5"]
+    assert r["initial_rows_moved_per_segment"] == 0
     assert r["rows_moved_per_segment_step"] == 1.0
     assert r["bytes_moved_per_segment_step"] == 200.0
     # after the move: block 1 (4 live) and block 2 (8, 3) hold 2 x 4 slots for 6 live tokens
-    assert r["slots_per_live_token"] == (8 / 8 + 8 / 6) / 2
+    assert r["slots_per_live_token"] == 8 / 6
     # a threshold of 0 never compacts; an empty block is freed without moves
     r0 = bench.block_compaction_study([[np.arange(8), np.arange(4, 9)]], (4,), (0.0,), 100)["block_4_theta_0.0"]
     assert r0["rows_moved_per_segment_step"] == 0.0
-    assert r0["slots_per_live_token"] == (8 / 8 + 8 / 5) / 2
+    assert r0["slots_per_live_token"] == 8 / 5
+    # a sparse starting layout is compacted once: blocks 0 and 1 hold one token
+    # each (positions 1 and 5), block 2 (the tail) holds 8..11
+    ri = bench.block_compaction_study([[np.array([1, 5, 8, 9, 10, 11]), np.array([1, 5, 8, 9, 10, 11, 12])]],
+                                      (4,), (0.5,), 100)["block_4_theta_0.5"]
+    assert ri["initial_rows_moved_per_segment"] == 2
+    assert ri["rows_moved_per_segment_step"] == 0.0
 
 
 def test_amortised_rate_of_a_run():

@@ -84,8 +84,9 @@ def args_parse(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--calls", default="all-layers", choices=["all-layers", "per-layer"],
                     help="per-layer: one attention call per layer, as a model's layers run (eviction stays one call)")
-    ap.add_argument("--compact", default="hole-fill", choices=["hole-fill", "stable"],
-                    help="stable: order-preserving compaction instead of hole-fill")
+    ap.add_argument("--compact", default="hole-fill", choices=["hole-fill", "stable", "linear"],
+                    help="stable: order-preserving compaction instead of hole-fill; linear: that, and the FP16 "
+                         "window without a ring (the whole cache in position order)")
     ap.add_argument("--graph", action="store_true",
                     help="also time the step replayed from a CUDA graph (the handle then runs single-stream)")
     ap.add_argument("--paged-study", action="store_true",
@@ -132,8 +133,10 @@ def workload_name(w):
                              else "confident -> N_low (prose)")
     if w.get("calls", "all-layers") != "all-layers":
         name += ", one attention call per layer"
-    if w.get("compact", "hole-fill") != "hole-fill":
+    if w.get("compact", "hole-fill") == "stable":
         name += ", stable compaction"
+    elif w.get("compact", "hole-fill") == "linear":
+        name += ", stable compaction and a linear FP16 window (no ring)"
     if w.get("graph"):
         name += ", single-stream handle (graph-capturable)"
     if w.get("score", "ema") != "ema":
@@ -562,7 +565,7 @@ def make_handle(w, L=None, args=None, sliding_window=False):
                   n_high=w["n_high"], tau=w["tau"], alpha=w["alpha"], ema_decay=w["beta"], protect_last=w["P"],
                   fp16_window=w["W"], pyramidal=1 if w["pyramidal"] else 0,
                   gate=1 if w["gate"] == "literal" else 0,
-                  compact=1 if w["compact"] == "stable" else 0,
+                  compact={"hole-fill": 0, "stable": 1, "linear": 2}[w["compact"]],
                   score_source={"ema": 0, "accum": 1, "random": 2}[w["score"]], seed=7,
                   single_stream=1 if w["graph"] else 0)
 
@@ -586,7 +589,8 @@ def step_bytes_model(w, d, K, launches_attn):
     cand = 0 if fixed else S * 208
     ema = 0 if fixed else (n8 + n16) * (4 * G + 12) / K + cand
     row = (2 * D + 16) if w.get("W", 0) and not fixed else (4 * D + 8)
-    evict = d["evict_tokens"] * 8 / K + cand + d["moved_rows"] * 2 * row / K + d["requant_rows"] * (6 * D + 8) / K
+    evict = (d["evict_tokens"] * 8 / K + cand + d["moved_rows"] * 2 * row / K + d["requant_rows"] * (6 * D + 8) / K
+             + d.get("moved_window_rows", 0) * 2 * (4 * D + 8) / K)
     conf = 0 if fixed else B * w["V"] * 4
     GP = 4 if G <= 4 else 8
     qf = 2 * D * G + (4 * GP + 16) * D + 4 * GP
@@ -600,7 +604,8 @@ def step_bytes_model(w, d, K, launches_attn):
 
 def counters_delta(a, b):
     return {k: b[k] - a[k] for k in ("attn_tokens_int8", "attn_tokens_fp16", "evict_tokens", "moved_rows",
-                                     "requant_rows", "kernel_launches", "evict_block_segments")}
+                                     "requant_rows", "kernel_launches", "evict_block_segments", "moved_window_rows")
+            if k in b}
 
 
 def measure(w, args, dev, world, rank, local, with_e2e=True, with_graph=False, study=False):
@@ -689,7 +694,7 @@ def measure(w, args, dev, world, rank, local, with_e2e=True, with_graph=False, s
         peak, _ = peaks()
         res["step1_kernels"] = roofline_table(b1, {k: v["ms"] for k, v in prof1.items() if v["launches"]}, peak)
         res["step1_counts"] = {k: d1[k] for k in ("attn_tokens_int8", "attn_tokens_fp16", "evict_tokens",
-                                                   "moved_rows", "requant_rows")}
+                                                   "moved_rows", "requant_rows", "moved_window_rows") if k in d1}
         first = 1
     else:
         # prefill's own traffic model (fixed mode: priorities read, kept rows gathered)
@@ -915,6 +920,7 @@ def line_for(w, res, args, world, cpu):
         "clocks": res["clocks"],
         "kernels": res["kernels"],
         "evict_block_segments_per_step": res["counters"]["evict_block_segments"] / res["K"],
+        "moved_window_rows_per_step": res["counters"].get("moved_window_rows", 0) / res["K"],
         "step_hbm_gbs": res["step_hbm_gbs"],
         "kernel_ms_per_step": res["kernel_ms"],
         "kv_resident_bytes": {"conf_kv": res["stats"]["bytes_payload"], "full_fp16": res["full_cache"],

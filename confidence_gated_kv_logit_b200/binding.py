@@ -21,7 +21,7 @@ LIB_PATH = os.environ.get("CONFKV_LIBRARY", os.path.join(HERE, "libconfkv.so"))
 ALL_LAYERS = -1
 MODE_CONF, MODE_FIXED = 0, 1
 GATE_PROSE, GATE_LITERAL = 0, 1
-COMPACT_HOLEFILL, COMPACT_STABLE = 0, 1
+COMPACT_HOLEFILL, COMPACT_STABLE, COMPACT_LINEAR = 0, 1, 2
 SCORE_EMA, SCORE_ACCUM, SCORE_RANDOM = 0, 1, 2
 
 STATUS = {0: "OK", 1: "ERR_ARG", 2: "ERR_CAPACITY", 3: "ERR_STATE", 4: "ERR_NONFINITE",
@@ -59,7 +59,8 @@ class Stats(ctypes.Structure):
                 ("max_len", ctypes.c_int32), ("attn_tokens_int8", ctypes.c_int64),
                 ("attn_tokens_fp16", ctypes.c_int64), ("evict_tokens", ctypes.c_int64),
                 ("moved_rows", ctypes.c_int64), ("requant_rows", ctypes.c_int64),
-                ("kernel_launches", ctypes.c_int64), ("evict_block_segments", ctypes.c_int64)]
+                ("kernel_launches", ctypes.c_int64), ("evict_block_segments", ctypes.c_int64),
+                ("moved_window_rows", ctypes.c_int64)]
 
 
 class Profile(ctypes.Structure):

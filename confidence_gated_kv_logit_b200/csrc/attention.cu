@@ -195,7 +195,46 @@ __global__ void __launch_bounds__(256) append_kernel(Cache c, AttnLaunch a, Poli
   row_load_plain<D>(vn, lane, vw);
   prepare_query<D, GP>(c, a, s, l, b, h, lane, qscale);   // independent of the cache state
   if (!guard(t >= 0 && n_cold0 >= 0 && n_cold0 <= c.cap, c.err, kSiteAppendSeg, s, t)) return;
-  if (c.W > 0) {
+  if (c.W > 0 && c.linear) {
+    // Linear window: slots [0, n16) hold the window in position order. If
+    // its oldest token has reached age W (a caller skipped eviction), it is
+    // converted to INT8 as eviction would have done and the window moves
+    // down by one slot; the new token goes after the last occupied slot.
+    const int32_t* pr = c.pos_r + (size_t)s * c.Wst;
+    int occ = 0;
+    for (int sl = lane; sl < c.W; sl += 32) occ += pr[sl] >= 0;
+    int n16 = __reduce_add_sync(0xffffffffu, occ);
+    const int oldest = n16 > 0 ? pr[0] : -1;
+    if (n16 > 0 && t - oldest >= c.W) {
+      const int idx = n_cold0;
+      if (idx >= c.cap) {
+        if (lane == 0) set_error(c.err, kErrDevice);
+        return;
+      }
+      warp_requant<D>(c, s, 0, idx, lane);
+      if (lane == 0) {
+        const size_t cs = (size_t)s * c.cap + idx;
+        c.pos_c[cs] = oldest;
+        c.sc_c[cs] = c.sc_r[(size_t)s * c.Wst];
+        c.n_cold[s] = idx + 1;
+        atomicAdd(&c.counters[kCntRequant], 1ull);
+        if (n16 > 1) atomicAdd(&c.counters[kCntMovedWin], (unsigned long long)(n16 - 1));
+      }
+      __syncwarp();
+      warp_window_shift<D>(c, s, 1, n16, lane);
+      --n16;
+    }
+    if (n16 >= c.W) {   // cannot happen: a full window's oldest token has age W
+      if (lane == 0) set_error(c.err, kErrDevice);
+      return;
+    }
+    row_store_h<D>(c.kr + (size_t)s * c.Wst * D, n16, lane, kw);
+    row_store_h<D>(c.vr + (size_t)s * c.Wst * D, n16, lane, vw);
+    if (lane == 0) {
+      c.pos_r[(size_t)s * c.Wst + n16] = t;
+      c.sc_r[(size_t)s * c.Wst + n16] = sc_new;
+    }
+  } else if (c.W > 0) {
     const int slot = t % c.W;
     const size_t rs = (size_t)s * c.Wst + slot;
     const int old = c.pos_r[rs];

@@ -7,7 +7,8 @@
 //       or fp16 rows  kc/vc [S][cap][D]                              (INT8 off)
 //       int32 pos_c [S][cap], fp32 sc_c [S][cap] (EMA, or priority in fixed mode)
 //   FP16 window ring (INT8 on only): W slots per segment, slot = pos mod W,
-//       allocated with a stride Wst = W rounded up to 4 slots
+//       allocated with a stride Wst = W rounded up to 4 slots (the linear
+//       layout keeps no ring: slots [0, n) hold the window in position order)
 //       fp16 kr/vr [S][Wst][D], int32 pos_r [S][Wst] (-1 = empty), fp32 sc_r [S][Wst]
 //   int32 n_cold [S], next_pos [S]
 // Rows are 64 or 128 B (INT8) and 128 or 256 B (fp16), so every row starts on a
@@ -34,6 +35,7 @@ enum Counter {
   kCntMovedRows = 3,
   kCntRequant = 4,
   kCntEvictBlock = 5,
+  kCntMovedWin = 6,
   kNumCounters = 8
 };
 
@@ -41,6 +43,7 @@ struct Cache {
   int L, Bmax, Hkv, Hq, G, D, W, cap;
   int Wst;            // ring allocation stride per segment: W rounded up to 4 slots
   int cold_int8;
+  int linear;         // window without a ring: slots [0, n) hold the FP16 tokens in position order
   int8_t* k8;
   int8_t* v8;
   __half* kc;
@@ -312,6 +315,52 @@ __device__ __forceinline__ void warp_requant(const Cache& c, int s, int ring_slo
   sc = row_quantize<D>(w, &pk);
   row_store_v8<D>(c.v8 + cb, cold_i, lane, pk);
   if (lane == 0) c.vs[cs] = sc;
+}
+
+// Linear window layout: move window slots [from, n) of segment s down to
+// [0, n - from), positions and score sources with them, and empty the slots
+// left behind; one warp. Rows are loaded four at a time before any is stored
+// (every destination is below its source, so no row is overwritten before it
+// has been read).
+template <int D>
+__device__ __forceinline__ void warp_window_shift(const Cache& c, int s, int from, int n, int lane) {
+  if (from <= 0 || n <= from) {
+    if (lane == 0)
+      for (int j = max(0, n - from); j < n; ++j) c.pos_r[(size_t)s * c.Wst + j] = -1;
+    return;
+  }
+  __half* kr = c.kr + (size_t)s * c.Wst * D;
+  __half* vr = c.vr + (size_t)s * c.Wst * D;
+  int32_t* pr = c.pos_r + (size_t)s * c.Wst;
+  float* sr = c.sc_r + (size_t)s * c.Wst;
+  for (int j = from; j < n; j += 4) {
+    uint32_t k[4][D / 64], v[4][D / 64];
+    int pp[4];
+    float ss[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (j + u < n) {
+        row_load_h<D>(kr, j + u, lane, k[u]);
+        row_load_h<D>(vr, j + u, lane, v[u]);
+        pp[u] = pr[j + u];
+        ss[u] = sr[j + u];
+      }
+    __syncwarp();
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (j + u < n) {
+        row_store_h<D>(kr, j + u - from, lane, k[u]);
+        row_store_h<D>(vr, j + u - from, lane, v[u]);
+        if (lane == 0) {
+          pr[j + u - from] = pp[u];
+          sr[j + u - from] = ss[u];
+        }
+      }
+    __syncwarp();
+  }
+  if (lane == 0)
+    for (int j = n - from; j < n; ++j) pr[j] = -1;
+  __syncwarp();
 }
 
 }  // namespace confkv

@@ -184,7 +184,10 @@ confkv_status confkv_create(int32_t layers, int32_t kv_heads, int32_t q_heads, i
   if (G < 1 || G > 8) return CONFKV_ERR_ARG;
   if (p.mode != CONFKV_MODE_CONF && p.mode != CONFKV_MODE_FIXED) return CONFKV_ERR_ARG;
   if (p.gate != CONFKV_GATE_PROSE && p.gate != CONFKV_GATE_LITERAL) return CONFKV_ERR_ARG;
-  if (p.compact != CONFKV_COMPACT_HOLEFILL && p.compact != CONFKV_COMPACT_STABLE) return CONFKV_ERR_ARG;
+  if (p.compact != CONFKV_COMPACT_HOLEFILL && p.compact != CONFKV_COMPACT_STABLE &&
+      p.compact != CONFKV_COMPACT_LINEAR)
+    return CONFKV_ERR_ARG;
+  if (p.compact == CONFKV_COMPACT_LINEAR && (p.mode != CONFKV_MODE_CONF || !p.int8_enable)) return CONFKV_ERR_ARG;
   if (p.score_source != CONFKV_SCORE_EMA && p.score_source != CONFKV_SCORE_ACCUM &&
       p.score_source != CONFKV_SCORE_RANDOM)
     return CONFKV_ERR_ARG;
@@ -249,6 +252,7 @@ confkv_status confkv_create(int32_t layers, int32_t kv_heads, int32_t q_heads, i
   c.Wst = round_up(W, 64);   // whole 64-slot tiles for the attention copies
   c.cap = (int)cap_ll;
   c.cold_int8 = p.int8_enable ? 1 : 0;
+  c.linear = p.compact == CONFKV_COMPACT_LINEAR ? 1 : 0;
 
   confkv::Policy& pol = h->pol;
   pol.mode = p.mode;
@@ -592,7 +596,7 @@ confkv_status confkv_evict_compact(confkv_handle* h, int32_t layer, void* stream
   a.budget = h->budget;
   a.vmask = h->vmask;
   a.mask_words = h->mask_words;
-  a.stable = h->p.compact == CONFKV_COMPACT_STABLE;
+  a.stable = h->p.compact != CONFKV_COMPACT_HOLEFILL;   // the linear layout compacts in order too
   a.cand = h->cand;
   a.kscratch = h->kscratch;
   a.scratch_stride = h->scratch_stride;
@@ -645,6 +649,7 @@ confkv_status confkv_query(confkv_handle* h, confkv_stats* out) {
   out->requant_rows = (int64_t)cnt[confkv::kCntRequant];
   out->kernel_launches = h->launches;
   out->evict_block_segments = (int64_t)cnt[confkv::kCntEvictBlock];
+  out->moved_window_rows = (int64_t)cnt[confkv::kCntMovedWin];
   out->bytes_capacity = (int64_t)h->buf.bytes;
   out->min_len = 0;
   out->max_len = 0;

@@ -110,7 +110,7 @@ __device__ __forceinline__ void move_cold_row(const Cache& c, int s, int src, in
 
 constexpr int kSegsPerCta = NT / 32;     // the fast path gives each warp one segment
 struct WarpCounts {
-  int scanned = 0, moved = 0, requant = 0;
+  int scanned = 0, moved = 0, requant = 0, moved_win = 0;
 };
 
 // One segment by one warp. Handles the common decode step (at most
@@ -151,7 +151,8 @@ __device__ bool evict_segment_warp(const Cache& c, const Policy& pol, const Evic
   // victims, except that the token may itself be one: checked below).
   const int leaving = t + 1 - W;
   const bool may_req = CI8 && W > 0 && leaving >= 0;
-  const int rq_slot = may_req ? (t + 1) % W : 0;
+  // ring: the slot the next append takes; linear window: the oldest slot
+  const int rq_slot = may_req && !c.linear ? (t + 1) % W : 0;
   int rq_pos = -1;
   float rq_sc = 0.0f;
   uint32_t rq_k[D / 64], rq_v[D / 64];
@@ -334,10 +335,19 @@ __device__ bool evict_segment_warp(const Cache& c, const Policy& pol, const Evic
       requant = 1;
     }
   }
+  int moved_win = 0;
+  if (c.linear && requant) {
+    // the window's oldest slot has been converted: the rest moves down one
+    // (no eviction ran here, so the window is slots [0, n_ring))
+    __syncwarp();
+    warp_window_shift<D>(c, s, 1, n_ring, lane);
+    moved_win = max(0, n_ring - 1);
+  }
   if (lane == 0) c.n_cold[s] = n_cold_new;
   wc->scanned = have ? 0 : n;   // tokens whose keys this call read
   wc->moved = moved;
   wc->requant = requant;
+  wc->moved_win = moved_win;
   return true;
 }
 
@@ -435,6 +445,62 @@ struct EvictSmem {
 
 // One segment by the whole CTA (all NT threads call it with the same item):
 // any number of victims, both compaction orders.
+// Linear window layout: move the occupied window slots of segment s, in
+// order, to slots [0, n) and empty the rest; the whole CTA, staging up to 64
+// slots at a time through shared memory (every destination is at or below
+// its source, and a chunk is read whole before any of it is written).
+// Returns the number of slots that moved (in every thread).
+template <int D>
+__device__ int block_window_compact(const Cache& c, int s, EvictSmem& es) {
+  constexpr int RB = 4 * D;                       // bytes of one slot: fp16 K and V rows
+  constexpr int CH = 16384 / RB < 64 ? 16384 / RB : 64;
+  constexpr int HP = RB / 32;                     // 16-byte parts of one row
+  unsigned char* kr = reinterpret_cast<unsigned char*>(c.kr + (size_t)s * c.Wst * D);
+  unsigned char* vr = reinterpret_cast<unsigned char*>(c.vr + (size_t)s * c.Wst * D);
+  int32_t* pr = c.pos_r + (size_t)s * c.Wst;
+  float* sr = c.sc_r + (size_t)s * c.Wst;
+  uint4* stage = reinterpret_cast<uint4*>(es.stage);
+  int dst_base = 0, moved = 0;
+  for (int base = 0; base < c.W; base += CH) {
+    const int slot = base + (int)threadIdx.x;
+    const bool live = threadIdx.x < CH && slot < c.W && pr[slot] >= 0;
+    int total;
+    const int r = block_scan_flag<NT>(live, es.sm, &total);
+    for (int w = threadIdx.x; w < CH * 2 * HP; w += NT) {
+      const int rr = w / (2 * HP), part = w - rr * 2 * HP;
+      const int sl = base + rr;
+      if (sl < c.W) {
+        const unsigned char* src = part < HP ? kr : vr;
+        stage[w] = *reinterpret_cast<const uint4*>(src + h_off(sl, 16 * (part % HP), D));
+      }
+    }
+    if (live) {
+      es.stage_meta[0][threadIdx.x] = pr[slot];
+      es.stage_meta[1][threadIdx.x] = __float_as_int(sr[slot]);
+      es.list_m[threadIdx.x] = dst_base + r;
+    }
+    if (threadIdx.x < CH) es.list_h[threadIdx.x] = live ? 1 : 0;
+    __syncthreads();
+    for (int w = threadIdx.x; w < CH * 2 * HP; w += NT) {
+      const int rr = w / (2 * HP), part = w - rr * 2 * HP;
+      if (base + rr < c.W && es.list_h[rr]) {
+        unsigned char* dst = part < HP ? kr : vr;
+        *reinterpret_cast<uint4*>(dst + h_off(es.list_m[rr], 16 * (part % HP), D)) = stage[w];
+      }
+    }
+    if (live) {
+      const int d = es.list_m[threadIdx.x];
+      pr[d] = es.stage_meta[0][threadIdx.x];
+      sr[d] = __int_as_float(es.stage_meta[1][threadIdx.x]);
+      moved += d != slot ? 1 : 0;
+    }
+    dst_base += total;
+    __syncthreads();
+  }
+  for (int j = dst_base + (int)threadIdx.x; j < c.W; j += NT) pr[j] = -1;
+  return block_sum_int<NT>(moved, es.sm);
+}
+
 // Keys already in this CTA's scratch (the bulk variant's EMA pass wrote
 // them): the occupied window slots and this thread's range of counted keys.
 struct BlockKeys {
@@ -698,8 +764,23 @@ __device__ void evict_segment_block(const Cache& c, const Policy& pol, const Evi
   // the token that the next append would push out of the window becomes INT8
   __syncthreads();
   const int leaving = t + 1 - W;
+  int conv_slot = W > 0 ? (t + 1) % W : 0;
+  if (c.linear) {
+    // linear window: the oldest occupied slot (the window is in position order)
+    int f = W;
+    for (int slot = threadIdx.x; slot < W; slot += NT)
+      if (pos_r[slot] >= 0) f = min(f, slot);
+    f = __reduce_min_sync(0xffffffffu, f);
+    if ((threadIdx.x & 31) == 0) sm.warp_tot[threadIdx.x >> 5] = f;
+    __syncthreads();
+    f = W;
+#pragma unroll
+    for (int i = 0; i < NT / 32; ++i) f = min(f, sm.warp_tot[i]);
+    __syncthreads();
+    conv_slot = f < W ? f : 0;
+  }
   if (W > 0 && leaving >= 0 && threadIdx.x < 32) {
-    const int slot = (t + 1) % W;
+    const int slot = conv_slot;
     const size_t rs = (size_t)s * c.Wst + slot;
     if (c.pos_r[rs] == leaving) {
       const int idx = n_cold_new;
@@ -719,8 +800,14 @@ __device__ void evict_segment_block(const Cache& c, const Policy& pol, const Evi
       }
     }
   }
+  int moved_win = 0;
+  if (c.linear) {
+    __syncthreads();   // the conversion above has emptied its slot
+    moved_win = block_window_compact<D>(c, s, es);
+  }
   if (threadIdx.x == 0) {
     c.n_cold[s] = n_cold_new;
+    if (moved_win > 0) atomicAdd(&c.counters[kCntMovedWin], (unsigned long long)moved_win);
     atomicAdd(&c.counters[kCntEvictBlock], 1ull);
     if (a.cand != nullptr) a.cand[s].stamp = -1;
     // tokens whose keys this path read from the cache (precomputed keys came
@@ -740,11 +827,11 @@ __global__ void __launch_bounds__(NT, GMAX > 4 ? 3 : 4) evict_kernel(Cache c, Po
   __shared__ EvictSmem es;
   __shared__ int slow_items[kSegsPerCta];
   __shared__ int n_slow;
-  __shared__ unsigned long long cnt[3];
+  __shared__ unsigned long long cnt[4];
   __shared__ int pairs[kSegsPerCta][2 * kWarpMaxVictims];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) n_slow = 0;
-  if (threadIdx.x < 3) cnt[threadIdx.x] = 0;
+  if (threadIdx.x < 4) cnt[threadIdx.x] = 0;
   __syncthreads();
   // Segments are dealt to warps through a multiplicative bijection of
   // [0, items) (the multiplier is a prime above any item count), so that the
@@ -771,6 +858,7 @@ __global__ void __launch_bounds__(NT, GMAX > 4 ? 3 : 4) evict_kernel(Cache c, Po
       if (wc.scanned) atomicAdd(&cnt[0], (unsigned long long)wc.scanned);
       if (wc.moved) atomicAdd(&cnt[1], (unsigned long long)wc.moved);
       if (wc.requant) atomicAdd(&cnt[2], (unsigned long long)wc.requant);
+      if (wc.moved_win) atomicAdd(&cnt[3], (unsigned long long)wc.moved_win);
     }
   }
   __syncthreads();
@@ -778,6 +866,7 @@ __global__ void __launch_bounds__(NT, GMAX > 4 ? 3 : 4) evict_kernel(Cache c, Po
     if (cnt[0]) atomicAdd(&c.counters[kCntEvictScanned], cnt[0]);
     if (cnt[1]) atomicAdd(&c.counters[kCntMovedRows], cnt[1]);
     if (cnt[2]) atomicAdd(&c.counters[kCntRequant], cnt[2]);
+    if (cnt[3]) atomicAdd(&c.counters[kCntMovedWin], cnt[3]);
   }
   const int ns = n_slow;
   for (int k = 0; k < ns; ++k) {

@@ -105,7 +105,13 @@ __global__ void __launch_bounds__(NT) prefill_ingest_kernel(Cache c, Policy pol,
   const float sc = fixed_mode ? a.prio[in_row] : initial_score(pol, l, b, h, p);
   uint32_t w[D / 64];
   if (c.W > 0 && p > len - c.W) {
-    const int slot = p % c.W;
+    // ring: slot pos mod W; linear window: the kept list's window part in
+    // order (it follows the n_cold cold tokens)
+    const int slot = c.linear ? i - c.n_cold[s] : p % c.W;
+    if (c.linear && (slot < 0 || slot >= c.W)) {
+      if (lane == 0) set_error(c.err, kErrDevice);
+      return;
+    }
     const size_t rs = (size_t)s * c.Wst + slot;
     row_load_plain<D>(ksrc, lane, w);
     row_store_h<D>(c.kr + (size_t)s * c.Wst * D, slot, lane, w);

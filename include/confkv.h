@@ -68,8 +68,19 @@ enum { CONFKV_MODE_CONF = 0, CONFKV_MODE_FIXED = 1 };
  * n_high, as the CONF-KV abstract and post describe. LITERAL: the
  * pseudo-code line's polarity, n_high when c >= tau. */
 enum { CONFKV_GATE_PROSE = 0, CONFKV_GATE_LITERAL = 1 };
-/* Compaction variant; both give the same logical cache content. */
-enum { CONFKV_COMPACT_HOLEFILL = 0, CONFKV_COMPACT_STABLE = 1 };
+/* Compaction variant and window layout; all give the same logical cache
+ * content (the tokens, their precision, payload, scales and EMA):
+ *   HOLEFILL  survivors above the new end of the INT8 region move into the
+ *             holes below it (bytes in proportion to the victims); the FP16
+ *             window is a ring, slot = position mod W;
+ *   STABLE    order-preserving compaction of the INT8 region (every survivor
+ *             after the first hole moves down); the window is a ring;
+ *   LINEAR    no ring: the INT8 region is compacted in order and the FP16
+ *             window occupies slots [0, n) in position order, so the whole
+ *             cache is position-ordered; every conversion or window eviction
+ *             moves the window's later slots down. Confidence mode with INT8
+ *             on only. */
+enum { CONFKV_COMPACT_HOLEFILL = 0, CONFKV_COMPACT_STABLE = 1, CONFKV_COMPACT_LINEAR = 2 };
 /* Score source of the confidence mode's ranking (score = alpha*source +
  * (1-alpha)*recency):
  *   EMA    ema <- beta*ema + (1-beta)*a (the CONF-KV post's EMA; the default);
@@ -126,6 +137,7 @@ typedef struct {
   int64_t requant_rows;       /* cumulative tokens converted FP16 -> INT8 */
   int64_t kernel_launches;    /* cumulative kernels launched by this handle */
   int64_t evict_block_segments; /* cumulative segments evicted by the whole-CTA path (many victims) */
+  int64_t moved_window_rows;  /* cumulative FP16 window rows moved (the linear layout's window shifts) */
 } confkv_stats;
 
 /* Fill *p with the defaults: CONF mode, N_low 256, N_high 512, tau 0.6,

@@ -48,6 +48,7 @@ int main(void) {
   FIELD(confkv_stats, requant_rows);
   FIELD(confkv_stats, kernel_launches);
   FIELD(confkv_stats, evict_block_segments);
+  FIELD(confkv_stats, moved_window_rows);
   printf("sizeof confkv_profile %zu\n", sizeof(confkv_profile));
   FIELD(confkv_profile, launches);
   FIELD(confkv_profile, ms);

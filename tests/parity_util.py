@@ -18,12 +18,16 @@ ATOL_EMA = 1e-9
 NEAR_TIE = 1e-5     # confidence within this of tau: both sides use the GPU's budget
 
 
-def c_params(p: Params, max_batch: int, max_prefill: int, stable: bool = False) -> dict:
+COMPACT = {"hole-fill": 0, "stable": 1, "linear": 2}
+
+
+def c_params(p: Params, max_batch: int, max_prefill: int, stable: bool = False, compact: str = None) -> dict:
     return dict(mode=1 if p.mode == "fixed" else 0, n_low=p.n_low, n_high=p.n_high, tau=p.tau,
                 alpha=p.alpha, ema_decay=p.ema_decay, protect_last=p.protect_last,
                 fp16_window=p.fp16_window, n_sink=p.n_sink, fixed_budget=p.fixed_budget,
                 pyramidal=int(p.pyramidal), gate=0 if p.gate == "prose" else 1,
-                int8_enable=int(p.int8), compact=1 if stable else 0, max_batch=max_batch,
+                int8_enable=int(p.int8), compact=COMPACT[compact or ("stable" if stable else "hole-fill")],
+                max_batch=max_batch,
                 max_prefill=max_prefill, score_source={"ema": 0, "accum": 1, "random": 2}[p.score_source],
                 seed=p.seed)
 
@@ -32,13 +36,14 @@ class Pair:
     """The library and the oracle, fed identical inputs."""
 
     def __init__(self, L, Hkv, Hq, D, B, params: Params, max_prefill: int, track=None, stable=False,
-                 seed=0, gen_chunk=None):
+                 seed=0, gen_chunk=None, compact=None):
         _build.build()
         self.L, self.Hkv, self.Hq, self.D, self.B, self.p = L, Hkv, Hq, D, B, params
         # prompt K/V are drawn this many sequences at a time (bounds the fp32
         # temporaries of the generator at the largest shapes)
         self.gen_chunk = gen_chunk or B
-        self.gpu = ConfKV(L, Hkv, Hq, D, **c_params(params, B, max_prefill, stable))
+        self.compact = compact or ("stable" if stable else "hole-fill")
+        self.gpu = ConfKV(L, Hkv, Hq, D, **c_params(params, B, max_prefill, compact=self.compact))
         self.orc = OracleCache(L, Hkv, Hq, D, params, track)
         self.track = track
         self.gen = synth.generator(seed, "cuda")
@@ -180,6 +185,20 @@ def assert_segment_equal(g: dict, o, key, exact_scores=True):
         np.testing.assert_allclose(g["score_src"], o.score_src, rtol=RTOL_EMA, atol=ATOL_EMA, err_msg=str(key))
 
 
+def assert_linear_layout(ex: dict, key):
+    """The linear layout's physical order: the INT8 region in increasing
+    position, the window in slots [0, n) in increasing position, every later
+    slot empty, and every window position above every INT8 one."""
+    pc = ex["pos_c"].astype(np.int64)
+    pr = ex["pos_r"].astype(np.int64)
+    assert np.all(np.diff(pc) > 0), key
+    n = int((pr >= 0).sum())
+    assert np.all(pr[:n] >= 0) and np.all(pr[n:] == -1), (key, pr[:8], n)
+    assert np.all(np.diff(pr[:n]) > 0), key
+    if n and pc.size:
+        assert pr[0] > pc[-1], key
+
+
 def run_synced(pair: Pair, lens, steps, V, T=None, check_every=1, schedule=None, all_rows_every=None):
     """Step-synchronised parity run: per step, attention (tolerance), EMA
     (tolerance), confidence and budgets, then -- with the oracle given the
@@ -225,5 +244,7 @@ def run_synced(pair: Pair, lens, steps, V, T=None, check_every=1, schedule=None,
             if check:
                 for key in pair.segments():
                     assert_segment_equal(pair.gpu_segment(*key), pair.orc.segment(*key), (step,) + key)
+                    if pair.compact == "linear":
+                        assert_linear_layout(pair.gpu.export_segment(*key), (step,) + key)
     assert pair.gpu.last_error() == 0
     return worst

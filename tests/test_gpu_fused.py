@@ -31,14 +31,15 @@ def _equal_caches(ha, hb, L, B, Hkv, where):
 
 
 @pytest.mark.parametrize("per_layer", [False, True], ids=["all_layers", "per_layer_calls"])
-@pytest.mark.parametrize("G,score", [(4, 0), (5, 0), (1, 1), (4, 2)], ids=["gqa4", "gqa5", "mha_accum", "gqa4_random"])
-def test_fused_pass_matches_separate_pass(per_layer, G, score):
+@pytest.mark.parametrize("G,score,compact", [(4, 0, 0), (5, 0, 0), (1, 1, 0), (4, 2, 0), (4, 0, 2)],
+                         ids=["gqa4", "gqa5", "mha_accum", "gqa4_random", "gqa4_linear_window"])
+def test_fused_pass_matches_separate_pass(per_layer, G, score, compact):
     build.build()
     dev = torch.device("cuda")
     L, Hkv, D, B, V = 3, 2, 128, 3, 2048
     Hq = Hkv * G
     kw = dict(max_batch=B, max_prefill=3000, n_low=64, n_high=160, protect_last=16, fp16_window=32, n_sink=2,
-              pyramidal=1, score_source=score, seed=9)
+              pyramidal=1, score_source=score, seed=9, compact=compact)
     ha, hb = ConfKV(L, Hkv, Hq, D, **kw), ConfKV(L, Hkv, Hq, D, **kw)
     g = synth.generator(31, dev)
     lens = [3000, 700, 90]     # the first step evicts thousands from the first sequence (whole-CTA path)

@@ -78,3 +78,37 @@ def test_graph_replay_matches_direct_calls(per_layer):
     assert handles[0].last_error() == 0 and handles[1].last_error() == 0
     for h in handles:
         h.close()
+
+
+def test_graph_replays_past_capacity_stop_at_the_device_guard():
+    # Replays of a captured decode call do not advance the handle's host-side
+    # length bounds, so a caller that replays decode steps without eviction
+    # can outgrow the cache. The append kernel's own capacity check then skips
+    # the work and sets the device error word; nothing is written out of bounds
+    # and the cache stays consistent.
+    build.build()
+    dev = torch.device("cuda")
+    L, Hkv, Hq, D, B = 1, 1, 4, 64, 1
+    h = ConfKV(L, Hkv, Hq, D, max_batch=B, max_prefill=100, n_low=32, n_high=48, protect_last=8, fp16_window=16,
+               single_stream=1)
+    cap_rows = 128                                           # max(100, 48) + 2 rounded up to 64
+    g = synth.generator(51, dev)
+    k, v = synth.prefill_kv(B, Hkv, 100, D, g, dev)
+    h.prefill(k, v, [100], layer=0)
+    q, kn, vn = synth.step_qkv((L, B), Hq, Hkv, D, g, dev)
+    out = torch.empty((L, B, Hq, D), device=dev)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        h.decode_attn(q, kn, vn, out)
+    for _ in range(cap_rows + 20):
+        graph.replay()
+    torch.cuda.synchronize()
+    assert h.last_error(clear=True) == 7                    # CONFKV_ERR_DEVICE: work skipped
+    ex = h.export_segment(0, 0, 0)
+    assert ex["n_cold"] == cap_rows
+    pos = np.concatenate([ex["pos_c"], ex["pos_r"][ex["pos_r"] >= 0]])
+    assert len(np.unique(pos)) == len(pos)                   # no token twice
+    assert torch.isfinite(out).all()
+    del graph
+    h.close()

@@ -98,6 +98,24 @@ def test_fixed_budget_mode_synced(int8):
     run_synced(pair, [700, 50], 10, 0)
 
 
+@pytest.mark.parametrize("case", [
+    dict(L=2, Hkv=2, Hq=8, D=128, B=2, lens=[900, 300], p=Params(n_low=100, n_high=200, protect_last=16, fp16_window=32,
+                                                                 n_sink=2)),
+    dict(L=3, Hkv=2, Hq=10, D=128, B=2, lens=[700, 129], p=Params(n_low=40, n_high=80, protect_last=8, fp16_window=24,
+                                                                  pyramidal=True)),
+    dict(L=1, Hkv=4, Hq=4, D=64, B=2, lens=[150, 31], p=Params(n_low=30, n_high=70, protect_last=10, fp16_window=48,
+                                                               gate="literal", alpha=1.0)),
+], ids=["gqa4_sinks", "gqa5_pyramid", "mha64_window_evictions"])
+def test_linear_window_layout_synced(case):
+    # no ring: the whole cache stays in position order (checked physically
+    # after every eviction), with the same logical content as the oracle
+    pair = Pair(case["L"], case["Hkv"], case["Hq"], case["D"], case["B"], case["p"],
+                max_prefill=max(case["lens"]), compact="linear", seed=27)
+    run_synced(pair, case["lens"], 14, 2048)
+    st = pair.gpu.query()
+    assert st["moved_window_rows"] > 0
+
+
 def test_stable_compaction_same_logical_content():
     p = Params(n_low=100, n_high=200, protect_last=16, fp16_window=32)
     pair = Pair(1, 2, 8, 128, 2, p, max_prefill=900, stable=True)
@@ -205,12 +223,12 @@ def test_budget_before_first_confidence_call_synced():
                 assert pair.gpu_segment(l, b, h)["pos"].tolist() == list(range(401 - eff, 401)), (l, b, h)
 
 
-@pytest.mark.parametrize("stable", [False, True], ids=["hole_fill", "stable"])
-def test_skipped_eviction_converts_on_append_synced(stable):
+@pytest.mark.parametrize("compact", ["hole-fill", "stable", "linear"])
+def test_skipped_eviction_converts_on_append_synced(compact):
     # a caller that skips eviction: the next append converts the token that
     # has left the FP16 window (the oracle converts t + 1 - W on append too)
     p = Params(n_low=100, n_high=200, protect_last=16, fp16_window=32, n_sink=2)
-    pair = Pair(2, 2, 8, 128, 2, p, max_prefill=400, seed=25, stable=stable)
+    pair = Pair(2, 2, 8, 128, 2, p, max_prefill=400, seed=25, compact=compact)
     schedule = ["a", "a", "ace", "ac", "a", "ace", "ace", "a", "ace"]
     run_synced(pair, [400, 130], 0, 2048, schedule=schedule)
     st = pair.gpu.query()

@@ -72,6 +72,9 @@ def test_param_struct_matches_the_header():
     ((1, 4, 4, 64), {"mode": 1, "fixed_budget": 10, "n_sink": 8, "protect_last": 8}),
     ((1, 4, 4, 64), {"gate": 7}),
     ((1, 4, 4, 64), {"score_source": 3}),
+    ((1, 4, 4, 64), {"compact": 3}),
+    ((1, 4, 4, 64), {"compact": 2, "int8_enable": 0}),       # the linear window needs INT8 on
+    ((1, 4, 4, 64), {"compact": 2, "mode": 1, "fixed_budget": 64, "protect_last": 16}),   # and confidence mode
 ])
 def test_create_rejects_bad_arguments_before_touching_the_device(lib, shape, kw):
     p = binding.default_params()

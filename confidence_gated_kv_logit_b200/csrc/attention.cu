@@ -450,6 +450,7 @@ struct TileCtx {
   float* sc_base;            // scores of this segment, [G][score_stride]
   int warp, lane;
   LaneOffsets lo;
+  uint64_t keep_policy;      // L2 policy of the score stores (read again by the EMA pass)
 };
 
 // One INT8 tile (128 tokens): warp w scores tokens 32w..32w+31 and builds the
@@ -504,8 +505,10 @@ __device__ __forceinline__ bool consume_i8(const Cache& c, const AttnLaunch& a, 
         const float ul = sg * kLog2e;
         if (valid) {
           const int col = x.j0 + r;
-          if (!kChecked || guard(col < a.score_stride, c.err, kSiteAttnScore, 0, col))
-            x.sc_base[(size_t)head * a.score_stride + col] = ul;   // scores are kept in log2 units
+          if (!kChecked || guard(col < a.score_stride, c.err, kSiteAttnScore, 0, col)) {
+            float* dst = x.sc_base + (size_t)head * a.score_stride + col;   // scores are kept in log2 units
+            st_f32_policy(dst, ul, x.keep_policy);
+          }
         }
         u[mb2][hr][j] = valid ? ul : -CUDART_INF_F;
       }
@@ -659,8 +662,10 @@ __device__ __forceinline__ bool consume_h(const Cache& c, const AttnLaunch& a, c
       const float ul = f[2 * hr + cc] * qscale * kLog2e;
       if (valid) {
         const int col = (RING ? c.cap : 0) + x.j0 + r;
-        if (!kChecked || guard(col < a.score_stride, c.err, kSiteAttnScore, 1, col))
-          x.sc_base[(size_t)head * a.score_stride + col] = ul;   // scores are kept in log2 units
+        if (!kChecked || guard(col < a.score_stride, c.err, kSiteAttnScore, 1, col)) {
+          float* dst = x.sc_base + (size_t)head * a.score_stride + col;   // scores are kept in log2 units
+          st_f32_policy(dst, ul, x.keep_policy);
+        }
       }
       u[hr][cc] = valid ? ul : -CUDART_INF_F;
     }
@@ -784,6 +789,11 @@ __global__ void __launch_bounds__(160, 2) attn_kernel(Cache c, AttnLaunch a, int
       // stage without data.
       int ctr = 0;
       int nq = 0;   // query-operand copies issued
+      // K/V tiles are read once per step: they go first when L2 needs room
+      const uint64_t stream_policy = l2_evict_first_policy();
+      auto copy = [&](void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+        bulk_g2s_hint(dst, src, bytes, bar, stream_policy);
+      };
       bool stop = false;
       auto next_stage = [&]() -> int {
         const int st = ctr % C::NSTAGE;
@@ -852,25 +862,25 @@ __global__ void __launch_bounds__(160, 2) attn_kernel(Cache c, AttnLaunch a, int
             const uint32_t vbytes = (uint32_t)((cnt + 31) >> 5) * 32 * D;                // whole 32-token blocks
             mbar_arrive_expect_tx(&full[st], kbytes + vbytes + 2u * cnt4 * 4u);
             const size_t row0 = (size_t)u.s * c.cap + j0;
-            bulk_g2s(sb, c.k8 + row0 * D, kbytes, &full[st]);
-            bulk_g2s(sb + C::KVB, c.v8 + row0 * D, vbytes, &full[st]);
-            bulk_g2s(sb + 2 * C::KVB, c.ks + row0, cnt4 * 4, &full[st]);
-            bulk_g2s(sb + 2 * C::KVB + 512, c.vs + row0, cnt4 * 4, &full[st]);
+            copy(sb, c.k8 + row0 * D, kbytes, &full[st]);
+            copy(sb + C::KVB, c.v8 + row0 * D, vbytes, &full[st]);
+            copy(sb + 2 * C::KVB, c.ks + row0, cnt4 * 4, &full[st]);
+            copy(sb + 2 * C::KVB + 512, c.vs + row0, cnt4 * 4, &full[st]);
           } else if (cold) {
             // fp16 cold rows: the whole 64-row tile (rows past n_cold hold finite older data or zeros)
             const uint32_t kvb = (uint32_t)C::TTR * 2 * D;
             mbar_arrive_expect_tx(&full[st], 2 * kvb);
             const size_t row0 = (size_t)u.s * c.cap + j0;
-            bulk_g2s(sb, c.kc + row0 * D, kvb, &full[st]);
-            bulk_g2s(sb + C::KVB, c.vc + row0 * D, kvb, &full[st]);
+            copy(sb, c.kc + row0 * D, kvb, &full[st]);
+            copy(sb + C::KVB, c.vc + row0 * D, kvb, &full[st]);
           } else {
             // window ring: the whole 64-slot tile (the ring stride is a multiple of 64)
             const uint32_t kvb = (uint32_t)C::TTR * 2 * D;
             mbar_arrive_expect_tx(&full[st], 2 * kvb + C::TTR * 4);
             const size_t row0 = (size_t)u.s * c.Wst + j0;
-            bulk_g2s(sb, c.kr + row0 * D, kvb, &full[st]);
-            bulk_g2s(sb + C::KVB, c.vr + row0 * D, kvb, &full[st]);
-            bulk_g2s(sb + 2 * C::KVB, c.pos_r + row0, C::TTR * 4, &full[st]);
+            copy(sb, c.kr + row0 * D, kvb, &full[st]);
+            copy(sb + C::KVB, c.vr + row0 * D, kvb, &full[st]);
+            copy(sb + 2 * C::KVB, c.pos_r + row0, C::TTR * 4, &full[st]);
           }
           ++ctr;
         }
@@ -888,6 +898,8 @@ __global__ void __launch_bounds__(160, 2) attn_kernel(Cache c, AttnLaunch a, int
   // -------------------------------- consumers --------------------------------
   const int g = lane >> 2, t = lane & 3;
   const LaneOffsets lane_offs = lane_offsets<D>(warp, lane);
+  // the scores are read again right after this kernel (the EMA pass): keep them in L2
+  const uint64_t keep_policy = l2_evict_last_policy();
   int ctr = 0;
   for (int k = 0;; ++k) {
     // the next unit: its id is published with its first stage
@@ -950,6 +962,7 @@ __global__ void __launch_bounds__(160, 2) attn_kernel(Cache c, AttnLaunch a, int
     x.warp = warp;
     x.lane = lane;
     x.lo = lane_offs;
+    x.keep_policy = keep_policy;
     bool aborted = false;
     if (u.t0 == u.t1) {   // a stage without data: release it and close the unit
       __syncwarp();

@@ -121,6 +121,11 @@ __device__ __forceinline__ int seg_of(const Cache& c, const Range& r, int item, 
 
 __device__ __forceinline__ void set_error(int32_t* err, int code) { atomicCAS(err, 0, code); }
 
+// A global store with an L2 eviction-priority policy (createpolicy).
+__device__ __forceinline__ void st_f32_policy(float* p, float v, uint64_t pol) {
+  asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(p), "f"(v), "l"(pol) : "memory");
+}
+
 // err[0] is the sticky status word; err[1..3] describe the first failed device
 // check: (site, segment, offending value).
 __device__ __forceinline__ void record_violation(int32_t* err, int site, int seg, int val) {

@@ -62,6 +62,7 @@ CONFIGS = {
 FULL = CONFIGS[3]
 SWEEP5 = [(b, c) for b in (1, 8, 64) for c in (4096, 32768, 131072)]
 POOL = 48   # distinct pre-generated step inputs, reused cyclically
+KERNEL_STEPS = 512   # steps of the per-kernel event region after the timed steps
 
 
 def args_parse(argv=None):
@@ -711,10 +712,8 @@ def measure(w, args, dev, world, rank, local, with_e2e=True, with_graph=False, s
     torch.cuda.synchronize()
     _report_device_error(h, "warm-up")
 
-    # ---- timed region ----
+    # ---- timed region: the step's kernels chained on one stream, no per-kernel events ----
     history = [] if study else None
-    h.profile(True)
-    h.profile_read(reset=True)
     sa = h.query()
     sampler = ClockSampler(physical_gpu_index(local))
     sampler.start()
@@ -730,26 +729,43 @@ def measure(w, args, dev, world, rank, local, with_e2e=True, with_graph=False, s
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    clocks = sampler.stop()
     _report_device_error(h, "timed region")
     elapsed_ms = e0.elapsed_time(e1)
+    sb = h.query()
+    # ---- kernel region: the next steps again, each kernel bracketed by CUDA
+    # events on its stream (the events sit between the chained launches and
+    # serialise them, so this region gives the per-kernel times, not the rate) ----
+    Kp = min(K, KERNEL_STEPS)
+    h.profile(True)
+    h.profile_read(reset=True)
+    if world > 1:
+        dist.barrier()
+    for i in range(Kp):
+        step_on(h, base + K + i)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    _report_device_error(h, "kernel region")
     prof = h.profile_read(reset=True)
     h.profile(False)
-    sb = h.query()
+    sc = h.query()
     elapsed_ms = max_over_ranks(elapsed_ms, dev)
     d = counters_delta(sa, sb)
+    dp = counters_delta(sb, sc)
     launches = max(1, prof["attention"]["launches"])
-    per_kernel, attn_bytes = step_bytes_model(w, d, K, launches)
+    per_kernel, attn_bytes = step_bytes_model(w, dp, Kp, launches)
+    step_bytes, _ = step_bytes_model(w, d, K, max(1, K))
     peak, peak_kind = peaks()
     attn_ms = prof["attention"]["ms"] / launches
-    res.update(K=K, elapsed_ms=elapsed_ms, ms_step=elapsed_ms / K, clocks=clocks, counters=d,
+    res.update(K=K, Kp=Kp, elapsed_ms=elapsed_ms, ms_step=elapsed_ms / K, clocks=clocks, counters=d,
                value=whole_job_rate(world, B, K, elapsed_ms), peak=peak, peak_kind=peak_kind,
                attn_bytes=attn_bytes, attn_ms=attn_ms,
-               attn_tokens_per_launch=(d["attn_tokens_int8"] + d["attn_tokens_fp16"]) / launches,
-               kernel_ms={k: round(v["ms"] / K, 4) for k, v in prof.items() if v["launches"]},
+               attn_tokens_per_launch=(dp["attn_tokens_int8"] + dp["attn_tokens_fp16"]) / launches,
+               kernel_ms={k: round(v["ms"] / Kp, 4) for k, v in prof.items() if v["launches"]},
                gpu_launches=d["kernel_launches"])
     res["kernels"] = roofline_table(per_kernel, res["kernel_ms"], peak)
-    res["step_hbm_gbs"] = sum(per_kernel.values()) / (res["ms_step"] * 1e-3) / 1e9
+    res["step_hbm_gbs"] = sum(step_bytes.values()) / (res["ms_step"] * 1e-3) / 1e9
     if w["config"] == 3:
         res["amortised"] = amortised_rate(B, w["run_steps"], res["step1_ms"], res["ms_step"])
 
@@ -913,7 +929,9 @@ def line_for(w, res, args, world, cpu):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": res["peak"], "unit": "GB/s",
                      "frac": achieved / res["peak"], "traffic": traffic, "peak_kind": res["peak_kind"],
                      "kernel": "attn_kernel", "algorithmic_bytes_per_launch": res["attn_bytes"],
-                     "ms_per_launch": res["attn_ms"], "attn_tokens_per_launch": res["attn_tokens_per_launch"]},
+                     "ms_per_launch": res["attn_ms"], "attn_tokens_per_launch": res["attn_tokens_per_launch"],
+                     "timed_over": f"{res['Kp']} steps after the timed ones, each kernel between CUDA events on "
+                                   "its stream (the timed steps run without per-kernel events)"},
         "cpu_baseline": cpu,
         "e2e": res.get("e2e"),
         "gpu_launches": res["gpu_launches"],

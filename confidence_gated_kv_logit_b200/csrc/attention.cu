@@ -174,6 +174,7 @@ __device__ __forceinline__ void prepare_query(const Cache& c, const AttnLaunch& 
 // ---------------------------------------------------------------------------
 template <int D, int GP>
 __global__ void __launch_bounds__(256) append_kernel(Cache c, AttnLaunch a, Policy pol, float qscale) {
+  chain_enter();
   const bool fixed_mode = pol.mode == 1;
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
@@ -741,6 +742,7 @@ __device__ __forceinline__ bool consume_h(const Cache& c, const AttnLaunch& a, c
 
 template <int D, int GP, bool CI8>
 __global__ void __launch_bounds__(160, 2) attn_kernel(Cache c, AttnLaunch a, int splits, int units, float qscale) {
+  chain_enter();
   using C = Cfg<D, GP, CI8>;
   using Q = QF<D, GP>;
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -1072,6 +1074,7 @@ __global__ void __launch_bounds__(160, 2) attn_kernel(Cache c, AttnLaunch a, int
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256) combine_kernel(Cache c, AttnLaunch a, int splits) {
+  chain_enter();
   const int G = c.G;
   const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
@@ -1114,7 +1117,7 @@ cudaError_t run_attn(const Cache& c, const Policy& pol, const AttnLaunch& a, cud
   const float qscale = rsqrtf((float)D);
   {
     ProfScope ps(prof, kKAppend, st);
-    append_kernel<D, GP><<<(items * 32 + 255) / 256, 256, 0, st>>>(c, a, pol, qscale);
+    (void)launch_chained(append_kernel<D, GP>, (items * 32 + 255) / 256, 256, 0, st, c, a, pol, qscale);
   }
   ++*launches;
   cudaError_t e = cudaGetLastError();
@@ -1142,13 +1145,13 @@ cudaError_t run_attn(const Cache& c, const Policy& pol, const AttnLaunch& a, cud
   const int grid = min(units, resident);
   {
     ProfScope ps(prof, kKAttention, st);
-    attn_kernel<D, GP, CI8><<<grid, 160, C::SMEM, st>>>(c, a, splits, units, qscale);
+    (void)launch_chained(attn_kernel<D, GP, CI8>, grid, 160, C::SMEM, st, c, a, splits, units, qscale);
   }
   ++*launches;
   if (splits > 1) {
     const int warps = items * c.G;
     ProfScope ps(prof, kKCombine, st);
-    combine_kernel<D><<<(warps * 32 + 255) / 256, 256, 0, st>>>(c, a, splits);
+    (void)launch_chained(combine_kernel<D>, (warps * 32 + 255) / 256, 256, 0, st, c, a, splits);
     ++*launches;
   }
   if (pol.mode == 0 && a.run_ema) {

@@ -368,4 +368,37 @@ __device__ __forceinline__ void warp_window_shift(const Cache& c, int s, int fro
   __syncwarp();
 }
 
+// ---------------------------------------------------------------------------
+// Chained launches (programmatic dependent launch). The kernels of one decode
+// step follow one another on the caller's stream; each is launched with
+// programmatic stream serialisation, so its CTAs may be scheduled while the
+// previous kernel is still finishing. Every chained kernel starts with
+// chain_enter(): it waits until the previous kernel has completed and its
+// writes are visible (so nothing is read or written early), then lets the next
+// kernel of the stream begin launching. Because each kernel waits before it
+// releases its successor, at most two kernels of the chain are resident at a
+// time and completion stays transitive: a kernel that has passed
+// chain_enter() knows every earlier kernel of the stream has completed. A
+// kernel launched without the attribute passes straight through.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void chain_enter() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... P, typename... A>
+cudaError_t launch_chained(void (*kern)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, A&&... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<A&&>(args)...);
+}
+
 }  // namespace confkv

@@ -64,6 +64,7 @@ __device__ __forceinline__ ConfPartial shfl_partial(const ConfPartial& p, int o)
 }
 
 __global__ void __launch_bounds__(NT) confidence_kernel(ConfLaunch a, Policy pol) {
+  chain_enter();
   __shared__ ConfPartial wpart[NT / 32];
   __shared__ int is_last;
   const int row = blockIdx.y;
@@ -244,10 +245,13 @@ __global__ void __launch_bounds__(NT) confidence_kernel(ConfLaunch a, Policy pol
 }  // namespace
 
 cudaError_t launch_confidence(const ConfLaunch& a, const Policy& pol, cudaStream_t st, long long* launches,
-                              Prof* prof) {
+                              Prof* prof, bool chained) {
   dim3 grid(a.cpr, a.B);
   ProfScope ps(prof, kKConfidence, st);
-  confidence_kernel<<<grid, NT, 0, st>>>(a, pol);
+  if (chained)
+    (void)launch_chained(confidence_kernel, grid, NT, 0, st, a, pol);
+  else
+    confidence_kernel<<<grid, NT, 0, st>>>(a, pol);
   ++*launches;
   return cudaGetLastError();
 }

@@ -89,7 +89,7 @@ confkv_status confkv_confidence_noalloc(const confkv_params* params, int32_t lay
   a.budget_out = nullptr;
   a.err = err;
   long long launches = 0;
-  return confkv::launch_confidence(a, pol, st, &launches, nullptr) == cudaSuccess ? CONFKV_OK : CONFKV_ERR_CUDA;
+  return confkv::launch_confidence(a, pol, st, &launches, nullptr, false) == cudaSuccess ? CONFKV_OK : CONFKV_ERR_CUDA;
 }
 
 }  // extern "C"

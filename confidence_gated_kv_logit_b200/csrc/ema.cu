@@ -35,6 +35,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 // kernel (which then need not rescan the segment).
 template <int GMAX>
 __global__ void __launch_bounds__(256) ema_kernel(Cache c, AttnLaunch a, Policy pol) {
+  chain_enter();
   const int lane = threadIdx.x & 31;
   const int item = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (item >= a.r.items(c.Hkv)) return;
@@ -68,6 +69,7 @@ static_assert(kCtaWarps * kWarpWant == 32, "the final merge holds one key per la
 
 template <int GMAX>
 __global__ void __launch_bounds__(kCtaThreads, 8) ema_cta_kernel(Cache c, AttnLaunch a, Policy pol) {
+  chain_enter();
   __shared__ unsigned long long w_key[kCtaWarps * kWarpWant];
   __shared__ int w_idx[kCtaWarps * kWarpWant];
   __shared__ unsigned long long w_bound[kCtaWarps];
@@ -203,9 +205,9 @@ void launch_ema(const Cache& c, const Policy& pol, const AttnLaunch& a, cudaStre
   const int items = a.r.items(c.Hkv);
   // four warps per segment while they fit in one wave (about 32 warps per SM)
   if ((long long)items * kCtaWarps <= (long long)a.num_sms * 32)
-    ema_cta_kernel<GMAX><<<items, kCtaThreads, 0, st>>>(c, a, pol);
+    (void)launch_chained(ema_cta_kernel<GMAX>, items, kCtaThreads, 0, st, c, a, pol);
   else
-    ema_kernel<GMAX><<<(items + 7) / 8, 256, 0, st>>>(c, a, pol);
+    (void)launch_chained(ema_kernel<GMAX>, (items + 7) / 8, 256, 0, st, c, a, pol);
 }
 
 }  // namespace

@@ -824,6 +824,7 @@ __device__ void evict_segment_block(const Cache& c, const Policy& pol, const Evi
 template <int D, bool CI8, int GMAX>
 __global__ void __launch_bounds__(NT, GMAX > 4 ? 3 : 4) evict_kernel(Cache c, Policy pol, EvictLaunch a, EmaIn ein,
                                                                       int items) {
+  chain_enter();
   __shared__ EvictSmem es;
   __shared__ int slow_items[kSegsPerCta];
   __shared__ int n_slow;
@@ -979,6 +980,7 @@ __device__ bool cta_ema_keys(const Cache& c, const EmaIn& in, const Policy& pol,
 template <int D, bool CI8, int GMAX>
 __global__ void __launch_bounds__(NT, 3) evict_bulk_kernel(Cache c, Policy pol, EvictLaunch a, EmaIn ein,
                                                            int items) {
+  chain_enter();
   __shared__ EvictSmem es;
   __shared__ int claimed;
   uint32_t* khi = a.kscratch + (size_t)blockIdx.x * a.scratch_stride;
@@ -1014,7 +1016,7 @@ cudaError_t run_bulk(const Cache& c, const Policy& pol, const EvictLaunch& a, co
   if (e != cudaSuccess) return e;
   // the key scratch exists for evict_grid(items) CTAs
   const int grid = max(1, min(evict_grid(items), max(1, per_sm) * num_sms));
-  evict_bulk_kernel<D, CI8, GMAX><<<grid, NT, 0, st>>>(c, pol, a, ema, items);
+  (void)launch_chained(evict_bulk_kernel<D, CI8, GMAX>, grid, NT, 0, st, c, pol, a, ema, items);
   return cudaGetLastError();
 }
 
@@ -1025,13 +1027,13 @@ cudaError_t run(const Cache& c, const Policy& pol, const EvictLaunch& a, const E
   const int grid = evict_grid(items);
   if (ema == nullptr) {
     ProfScope ps(prof, kKEvict, st);
-    evict_kernel<D, CI8, 0><<<grid, NT, 0, st>>>(c, pol, a, EmaIn{}, items);
+    (void)launch_chained(evict_kernel<D, CI8, 0>, grid, NT, 0, st, c, pol, a, EmaIn{}, items);
   } else {
     ProfScope ps(prof, kKEmaEvict, st);
     if (c.G <= 4)
-      evict_kernel<D, CI8, 4><<<grid, NT, 0, st>>>(c, pol, a, *ema, items);
+      (void)launch_chained(evict_kernel<D, CI8, 4>, grid, NT, 0, st, c, pol, a, *ema, items);
     else
-      evict_kernel<D, CI8, 8><<<grid, NT, 0, st>>>(c, pol, a, *ema, items);
+      (void)launch_chained(evict_kernel<D, CI8, 8>, grid, NT, 0, st, c, pol, a, *ema, items);
   }
   ++*launches;
   return cudaGetLastError();

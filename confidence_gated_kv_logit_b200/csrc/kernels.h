@@ -27,8 +27,10 @@ struct ConfLaunch {
   int32_t* budget_out;    // optional
   int32_t* err;
 };
+// chained: launched as the next kernel of the step's chain (set false when
+// the previous operation on the stream is not one of the library's kernels)
 cudaError_t launch_confidence(const ConfLaunch& a, const Policy& pol, cudaStream_t st, long long* launches,
-                              Prof* prof);
+                              Prof* prof, bool chained = true);
 
 // K2: prefill ingest.
 struct PrefillLaunch {

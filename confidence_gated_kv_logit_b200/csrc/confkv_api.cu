@@ -90,6 +90,11 @@ struct confkv_handle {
   std::vector<char> ema_pending;   // per layer
   cudaEvent_t attn_done;           // recorded after each deferred decode call's attention
   cudaStream_t attn_stream;        // the stream it was recorded on
+  // The handle's last launch was its confidence reduction, on conf_stream: an
+  // eviction call right after it on the same stream lets the fused kernel run
+  // its EMA pass beside that reduction (EvictLaunch::ema_early).
+  bool conf_last = false;
+  cudaStream_t conf_stream = nullptr;
   int scratch_stride;
   int32_t* keep_list;
   int32_t* keep_count;
@@ -426,6 +431,7 @@ static cudaError_t flush_ema(confkv_handle* h, int l0, int nl, cudaStream_t st) 
 // Every deferred pass, for the synchronising queries: after the device is
 // idle, on the legacy stream, then idle again.
 static cudaError_t flush_all_ema(confkv_handle* h) {
+  h->conf_last = false;
   bool any = false;
   for (char f : h->ema_pending) any = any || f;
   if (!any) return cudaSuccess;
@@ -457,6 +463,7 @@ confkv_status confkv_prefill(confkv_handle* h, int32_t layer, int32_t batch, con
   if (!aligned16(k) || !aligned16(v) || (priority && !aligned16(priority))) return CONFKV_ERR_ARG;
   const bool fixed = h->p.mode == CONFKV_MODE_FIXED;
   if (fixed != (priority != nullptr)) return CONFKV_ERR_ARG;
+  h->conf_last = false;
   int maxlen = 0;
   for (int b = 0; b < batch; ++b) {
     if (lens_host[b] < 0 || lens_host[b] > h->p.max_prefill || lens_host[b] > t_stride) return CONFKV_ERR_ARG;
@@ -525,8 +532,11 @@ confkv_status confkv_confidence(confkv_handle* h, const float* logits, int32_t b
   a.c_out = c_out;
   a.budget_out = budget_out;
   a.err = h->c.err;
-  return cuda_status(
-      confkv::launch_confidence(a, h->pol, static_cast<cudaStream_t>(stream), &h->launches, h->prof_ptr()));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const cudaError_t e = confkv::launch_confidence(a, h->pol, st, &h->launches, h->prof_ptr());
+  h->conf_last = e == cudaSuccess;
+  h->conf_stream = st;
+  return cuda_status(e);
 }
 
 confkv_status confkv_decode_attn(confkv_handle* h, int32_t layer, const void* q, const void* k_new,
@@ -568,6 +578,7 @@ confkv_status confkv_decode_attn(confkv_handle* h, int32_t layer, const void* q,
   const bool defer = h->pol.mode == 0 && !h->p.single_stream;
   a.run_ema = (h->pol.mode == 0 && !defer) ? 1 : 0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  h->conf_last = false;
   // a pass still deferred from the previous call over these layers reads the
   // scores this call is about to overwrite: run it first
   cudaError_t e = flush_ema(h, r.l0, r.nl, st);
@@ -603,6 +614,8 @@ confkv_status confkv_evict_compact(confkv_handle* h, int32_t layer, void* stream
   a.scratch_keys = h->c.cap + h->c.Wst;
   a.bulk_sched = h->bulk_sched;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  a.ema_early = h->conf_last && h->conf_stream == st ? 1 : 0;
+  h->conf_last = false;
   // Every layer of the call has its EMA pass deferred (the steady decode
   // step): the eviction kernel runs it fused. Otherwise the deferred passes
   // run on their own first and eviction reads their candidate records.

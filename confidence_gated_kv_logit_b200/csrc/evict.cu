@@ -824,7 +824,14 @@ __device__ void evict_segment_block(const Cache& c, const Policy& pol, const Evi
 template <int D, bool CI8, int GMAX>
 __global__ void __launch_bounds__(NT, GMAX > 4 ? 3 : 4) evict_kernel(Cache c, Policy pol, EvictLaunch a, EmaIn ein,
                                                                       int items) {
-  chain_enter();
+  // The fused variant's EMA pass reads only what attention and the kernels
+  // before it wrote. When the previous kernel is the confidence reduction
+  // (a.ema_early), which releases its successor only once everything before
+  // it has completed and which touches none of the pass's data, the pass runs
+  // before the wait, beside that reduction; the budgets it writes are read
+  // after the wait.
+  const bool early = GMAX > 0 && a.ema_early != 0;
+  if (!early) chain_enter();
   __shared__ EvictSmem es;
   __shared__ int slow_items[kSegsPerCta];
   __shared__ int n_slow;
@@ -840,14 +847,19 @@ __global__ void __launch_bounds__(NT, GMAX > 4 ? 3 : 4) evict_kernel(Cache c, Po
   // path at the same steps, land in different CTAs.
   const int slot = blockIdx.x * kSegsPerCta + warp;
   const int item = slot < items ? (int)(((unsigned long long)slot * 2654435761ull) % (unsigned long long)items) : items;
+  EmaOut eo;
+  if constexpr (GMAX > 0) {
+    if (item < items) {
+      int l, b, h;
+      const int s = seg_of(c, a.r, item, &l, &b, &h);
+      ema_segment_warp<GMAX>(c, ein, pol, s, lane, &eo);
+    }
+  }
+  if (early) chain_enter();
   if (item < items) {
     WarpCounts wc;
     bool done;
     if constexpr (GMAX > 0) {
-      int l, b, h;
-      const int s = seg_of(c, a.r, item, &l, &b, &h);
-      EmaOut eo;
-      ema_segment_warp<GMAX>(c, ein, pol, s, lane, &eo);
       // a corrupt segment was recorded by the pass; eviction skips it likewise
       done = !eo.ok || evict_segment_warp<D, CI8>(c, pol, a, item, lane, &wc, pairs[warp], &eo);
     } else {

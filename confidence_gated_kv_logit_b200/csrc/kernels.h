@@ -89,6 +89,9 @@ struct EvictLaunch {
   int scratch_stride;     // uint32 words per CTA
   int scratch_keys;       // offset of the hole list (= cap + Wst)
   int* bulk_sched;        // [2] segment counter and finished-CTA counter of the bulk variant (zero between launches)
+  // 1: the previous kernel on the stream is the confidence reduction, so the
+  // fused variant may run its EMA pass before waiting for it (see evict_kernel)
+  int ema_early = 0;
 };
 // Where an EMA pass reads the step's attention results.
 struct EmaIn {

@@ -503,9 +503,24 @@ __device__ int block_window_compact(const Cache& c, int s, EvictSmem& es) {
 
 // Keys already in this CTA's scratch (the bulk variant's EMA pass wrote
 // them): the occupied window slots and this thread's range of counted keys.
+// A bin map of key high halves fixed before the keys exist (confidence
+// mode): high halves at or below `lo` fall in bin 0, the rest in steps of
+// 2^shift, the last bin taking everything above; monotone in the key. With
+// `lo` below every score's bits and the steps sized to reach a score of 2,
+// the bins cover the scores' range at 2^(23 - shift) bins per octave.
+struct KeyBins {
+  uint32_t lo;
+  int shift;
+  __device__ __forceinline__ int operator()(uint32_t hv) const {
+    return hv <= lo ? 0 : (int)min((uint32_t)(kSelBins - 1), (hv - lo) >> shift);
+  }
+};
+
 struct BlockKeys {
   int n_ring;
   uint32_t kmn, kmx;
+  bool binned;    // the keys' histogram over `bins` is in the select buffer
+  KeyBins bins;
 };
 
 template <int D, bool CI8>
@@ -630,8 +645,11 @@ __device__ void evict_segment_block(const Cache& c, const Policy& pol, const Evi
     }
     __syncthreads();
     // the e-th smallest key: the victims are the keys up to it
-    const unsigned long long thr = block_select_threshold<NT>(
-        khi, pos_of, span, e, sm, reinterpret_cast<unsigned long long*>(es.stage), true, kmn, kmx);
+    unsigned long long* selbuf = reinterpret_cast<unsigned long long*>(es.stage);
+    const unsigned long long thr =
+        pre != nullptr && pre->binned
+            ? select_in_hist<NT>(khi, pos_of, span, e, sm, selbuf, pre->bins)
+            : block_select_threshold<NT>(khi, pos_of, span, e, sm, selbuf, true, kmn, kmx);
     const uint32_t thr_hi = (uint32_t)(thr >> 32), thr_lo = (uint32_t)thr;
     auto below_thr = [&](uint32_t hv, int i) -> bool {   // the position only matters on a tie of the high half
       return hv != 0xFFFFFFFFu && (hv < thr_hi || (hv == thr_hi && (uint32_t)pos_of(i) <= thr_lo));
@@ -895,7 +913,7 @@ __global__ void __launch_bounds__(NT, GMAX > 4 ? 3 : 4) evict_kernel(Cache c, Po
 // (recorded) for a corrupt segment.
 template <int GMAX>
 __device__ bool cta_ema_keys(const Cache& c, const EmaIn& in, const Policy& pol, int s, uint32_t* __restrict__ khi,
-                             BlockKeys* bk, SelectSmem<NT>& sm) {
+                             BlockKeys* bk, SelectSmem<NT>& sm, uint32_t* __restrict__ hist) {
   constexpr float kLog2eF = 1.4426950408889634f;
   const int G = c.G;
   const float invG = 1.0f / (float)G;
@@ -911,6 +929,39 @@ __device__ bool cta_ema_keys(const Cache& c, const EmaIn& in, const Policy& pol,
   const float* sb = in.scores + (size_t)s * G * in.score_stride;
   float* scc = c.sc_c + (size_t)s * c.cap;
   const int32_t* pc = c.pos_c + (size_t)s * c.cap;
+  // Confidence mode: every score is at least (1 - alpha)/(t + 1) (a recency
+  // term of at least 1/(t + 1), an EMA of probabilities >= 0), so a fixed bin
+  // map from half that up to 2 is known now and the select's histogram is
+  // built here, as the keys are computed (kSelBins 32-bit counts in `hist`).
+  KeyBins bins{0u, 0};
+  const bool binned = pol.mode == 0 && pol.one_minus_alpha > 0.0f && t >= 0;
+  if (binned) {
+    bins.lo = ordered_bits(0.5f * pol.one_minus_alpha / (float)(t + 1));
+    const uint32_t span = ordered_bits(2.0f) - bins.lo;
+    while ((span >> bins.shift) >= (uint32_t)kSelBins) ++bins.shift;
+    for (int i = threadIdx.x; i < kSelBins; i += NT) hist[i] = 0u;
+    __syncthreads();
+  }
+  // four consecutive keys (nq of them valid) into the histogram, runs of one
+  // bin added at once
+  auto hist_add = [&](uint32_t h0, uint32_t h1, uint32_t h2, uint32_t h3, int nq) {
+    const uint32_t hh[4] = {h0, h1, h2, h3};
+    int cur = -1;
+    uint32_t cnt = 0u;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (q < nq && hh[q] != 0xFFFFFFFFu) {
+        const int bq = bins(hh[q]);
+        if (bq != cur) {
+          if (cnt) atomicAdd(&hist[cur], cnt);
+          cur = bq;
+          cnt = 0u;
+        }
+        ++cnt;
+      }
+    }
+    if (cnt) atomicAdd(&hist[cur], cnt);
+  };
   auto hi_of = [&](int pos, float sc) -> uint32_t {
     const bool none = pos < 0 || t - pos < pol.P || pos < pol.n_sink;
     return none ? 0xFFFFFFFFu : (uint32_t)(rank_key(pol, sc, pos, t) >> 32);
@@ -938,12 +989,14 @@ __device__ bool cta_ema_keys(const Cache& c, const EmaIn& in, const Policy& pol,
         track(hv.y);
         track(hv.z);
         track(hv.w);
+        if (binned) hist_add(hv.x, hv.y, hv.z, hv.w, 4);
       } else if (i0 < n_cold) {   // the last, partial group
         const float4 e =
             ema_update4<GMAX>(sb, in.score_stride, i0, *reinterpret_cast<const float4*>(scc + i0), lse, G, invG, pol);
         const int4 p4 = *reinterpret_cast<const int4*>(pc + i0);
         const int pp[3] = {p4.x, p4.y, p4.z};
         const float ee[3] = {e.x, e.y, e.z};
+        uint32_t hq[3] = {0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu};
 #pragma unroll
         for (int q = 0; q < 3; ++q)
           if (i0 + q < n_cold) {
@@ -951,7 +1004,9 @@ __device__ bool cta_ema_keys(const Cache& c, const EmaIn& in, const Policy& pol,
             const uint32_t h = hi_of(pp[q], ee[q]);
             khi[i0 + q] = h;
             track(h);
+            hq[q] = h;
           }
+        if (binned) hist_add(hq[0], hq[1], hq[2], 0xFFFFFFFFu, 3);
       }
     }
   }
@@ -965,6 +1020,7 @@ __device__ bool cta_ema_keys(const Cache& c, const EmaIn& in, const Policy& pol,
                                        lse, G, invG, pol);
     const int pp[4] = {p4.x, p4.y, p4.z, p4.w};
     const float ee[4] = {e.x, e.y, e.z, e.w};
+    uint32_t hq[4] = {0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu};
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       if (s0 + q < c.W) {
@@ -976,12 +1032,16 @@ __device__ bool cta_ema_keys(const Cache& c, const EmaIn& in, const Policy& pol,
         }
         khi[n_cold + s0 + q] = h;
         track(h);
+        hq[q] = h;
       }
     }
+    if (binned) hist_add(hq[0], hq[1], hq[2], hq[3], 4);
   }
   bk->n_ring = block_sum_int<NT>(ring_here, sm);   // includes a block barrier: the keys are visible
   bk->kmn = kmn;
   bk->kmx = kmx;
+  bk->binned = binned;
+  bk->bins = bins;
   return true;
 }
 
@@ -1005,7 +1065,7 @@ __global__ void __launch_bounds__(NT, 3) evict_bulk_kernel(Cache c, Policy pol, 
     int l, b, h;
     const int s = seg_of(c, a.r, item, &l, &b, &h);
     BlockKeys bk;
-    if (!cta_ema_keys<GMAX>(c, ein, pol, s, khi, &bk, es.sm)) continue;
+    if (!cta_ema_keys<GMAX>(c, ein, pol, s, khi, &bk, es.sm, reinterpret_cast<uint32_t*>(es.stage))) continue;
     evict_segment_block<D, CI8>(c, pol, a, item, es, &bk);
     __syncthreads();
   }

@@ -360,6 +360,101 @@ constexpr int kSelBuf = 2048;   // 64-bit entries of the shared buffer block_sel
 constexpr int kSelBins = 2048;  // histogram bins (the first half of the buffer, as 32-bit counts)
 constexpr int kSelCand = (kSelBuf * 8 - kSelBins * 4) / 8;   // keys of one bin the rest of the buffer holds
 
+// The k-th smallest of the keys of block_select_threshold, given the
+// histogram of the counted high halves (first kSelBins 32-bit words of buf,
+// complete and visible) over a bin map `bin_of` that is monotone in the high
+// half: the bin holding the k-th key is located, its keys collected and
+// sorted; when that bin is too full for the buffer, the radix select decides.
+template <int NT, typename LoFn, typename BinFn>
+__device__ unsigned long long select_in_hist(const uint32_t* __restrict__ hi, LoFn lo, int n, int k,
+                                             SelectSmem<NT>& sm, unsigned long long* buf, BinFn bin_of) {
+  const uint4* hi4 = reinterpret_cast<const uint4*>(hi);
+  const int n4 = (n + 3) >> 2;
+  auto key_at = [&](const uint4& q, int j) { return j == 0 ? q.x : j == 1 ? q.y : j == 2 ? q.z : q.w; };
+  uint32_t* hist = reinterpret_cast<uint32_t*>(buf);
+  // the bin holding the k-th key: each thread sums its kSelBins/NT bins, a
+  // block scan places them
+  constexpr int BPT = kSelBins / NT;
+  uint32_t cnt[BPT];
+  uint32_t tot = 0u;
+#pragma unroll
+  for (int j = 0; j < BPT; ++j) {
+    cnt[j] = hist[threadIdx.x * BPT + j];
+    tot += cnt[j];
+  }
+  int all;
+  const int excl = block_excl_scan_int<NT>((int)tot, sm, &all);
+  if (threadIdx.x == 0) sm.misc[2] = -1;
+  __syncthreads();
+  if (excl < k && k <= excl + (int)tot) {
+    int below = excl;
+#pragma unroll
+    for (int j = 0; j < BPT; ++j) {
+      if (below + (int)cnt[j] >= k) {
+        sm.misc[2] = threadIdx.x * BPT + j;   // the bin
+        sm.misc[3] = below;                   // counted keys in lower bins
+        sm.misc[0] = (int)cnt[j];
+        break;
+      }
+      below += (int)cnt[j];
+    }
+  }
+  __syncthreads();
+  const int bstar = sm.misc[2], nbelow = sm.misc[3], ncand = sm.misc[0];
+  if (bstar >= 0 && ncand <= kSelCand) {
+    // pass 3: the keys of that bin into the second half of the buffer
+    unsigned long long* cand = buf + kSelBins / 2;
+    __syncthreads();   // every thread has read the bin
+    if (threadIdx.x == 0) sm.misc[1] = 0;
+    __syncthreads();
+    for (int v0 = threadIdx.x; v0 < n4; v0 += 4 * NT) {
+      uint4 q[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) q[r] = v0 + r * NT < n4 ? hi4[v0 + r * NT] : make_uint4(~0u, ~0u, ~0u, ~0u);
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int i = 4 * (v0 + r * NT) + j;
+          const uint32_t hv = key_at(q[r], j);
+          if (i < n && hv != 0xFFFFFFFFu && bin_of(hv) == bstar) {
+            const int slot = atomicAdd(&sm.misc[1], 1);
+            cand[slot] = ((unsigned long long)hv << 32) | (uint32_t)i;   // index for now
+          }
+        }
+    }
+    __syncthreads();
+    // the low halves, all loads of a thread in flight together
+    for (int j0 = (int)threadIdx.x; j0 < ncand; j0 += 4 * NT) {
+      int idx[4];
+      uint32_t lov[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int j = j0 + r * NT;
+        idx[r] = j < ncand ? (int)(uint32_t)cand[j] : -1;
+      }
+#pragma unroll
+      for (int r = 0; r < 4; ++r) lov[r] = idx[r] >= 0 ? (uint32_t)lo(idx[r]) : 0u;
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int j = j0 + r * NT;
+        if (j < ncand) cand[j] = (cand[j] & 0xFFFFFFFF00000000ull) | lov[r];
+      }
+    }
+    int m = 1;
+    while (m < ncand) m <<= 1;
+    for (int i = ncand + threadIdx.x; i < m; i += NT) cand[i] = kNoKey;
+    __syncthreads();
+    block_bitonic_sort<NT>(cand, m);
+    const unsigned long long r = cand[k - nbelow - 1];
+    __syncthreads();
+    return r;
+  }
+  __syncthreads();
+  const SelectResult r = block_select_smallest_hi<NT>(hi, lo, n, k, sm);
+  return r.prefix | ~r.mask;
+}
+
 // The k-th smallest (1-based) of the n 64-bit keys (hi[i] << 32) | lo(i),
 // where hi[i] == 0xFFFFFFFF marks an entry that is never counted (k must not
 // exceed the counted entries): every counted key <= the result is one of the
@@ -455,87 +550,7 @@ __device__ unsigned long long block_select_threshold(const uint32_t* __restrict_
       }
   }
   __syncthreads();
-  // the bin holding the k-th key: each thread sums its kSelBins/NT bins, a
-  // block scan places them
-  constexpr int BPT = kSelBins / NT;
-  uint32_t cnt[BPT];
-  uint32_t tot = 0u;
-#pragma unroll
-  for (int j = 0; j < BPT; ++j) {
-    cnt[j] = hist[threadIdx.x * BPT + j];
-    tot += cnt[j];
-  }
-  int all;
-  const int excl = block_excl_scan_int<NT>((int)tot, sm, &all);
-  if (threadIdx.x == 0) sm.misc[2] = -1;
-  __syncthreads();
-  if (excl < k && k <= excl + (int)tot) {
-    int below = excl;
-#pragma unroll
-    for (int j = 0; j < BPT; ++j) {
-      if (below + (int)cnt[j] >= k) {
-        sm.misc[2] = threadIdx.x * BPT + j;   // the bin
-        sm.misc[3] = below;                   // counted keys in lower bins
-        sm.misc[0] = (int)cnt[j];
-        break;
-      }
-      below += (int)cnt[j];
-    }
-  }
-  __syncthreads();
-  const int bstar = sm.misc[2], nbelow = sm.misc[3], ncand = sm.misc[0];
-  if (bstar >= 0 && ncand <= kSelCand) {
-    // pass 3: the keys of that bin into the second half of the buffer
-    unsigned long long* cand = buf + kSelBins / 2;
-    __syncthreads();   // every thread has read the bin
-    if (threadIdx.x == 0) sm.misc[1] = 0;
-    __syncthreads();
-    for (int v0 = threadIdx.x; v0 < n4; v0 += 4 * NT) {
-      uint4 q[4];
-#pragma unroll
-      for (int r = 0; r < 4; ++r) q[r] = v0 + r * NT < n4 ? hi4[v0 + r * NT] : make_uint4(~0u, ~0u, ~0u, ~0u);
-#pragma unroll
-      for (int r = 0; r < 4; ++r)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int i = 4 * (v0 + r * NT) + j;
-          const uint32_t hv = key_at(q[r], j);
-          if (i < n && hv != 0xFFFFFFFFu && bin_of(hv) == bstar) {
-            const int slot = atomicAdd(&sm.misc[1], 1);
-            cand[slot] = ((unsigned long long)hv << 32) | (uint32_t)i;   // index for now
-          }
-        }
-    }
-    __syncthreads();
-    // the low halves, all loads of a thread in flight together
-    for (int j0 = (int)threadIdx.x; j0 < ncand; j0 += 4 * NT) {
-      int idx[4];
-      uint32_t lov[4];
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int j = j0 + r * NT;
-        idx[r] = j < ncand ? (int)(uint32_t)cand[j] : -1;
-      }
-#pragma unroll
-      for (int r = 0; r < 4; ++r) lov[r] = idx[r] >= 0 ? (uint32_t)lo(idx[r]) : 0u;
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int j = j0 + r * NT;
-        if (j < ncand) cand[j] = (cand[j] & 0xFFFFFFFF00000000ull) | lov[r];
-      }
-    }
-    int m = 1;
-    while (m < ncand) m <<= 1;
-    for (int i = ncand + threadIdx.x; i < m; i += NT) cand[i] = kNoKey;
-    __syncthreads();
-    block_bitonic_sort<NT>(cand, m);
-    const unsigned long long r = cand[k - nbelow - 1];
-    __syncthreads();
-    return r;
-  }
-  __syncthreads();
-  const SelectResult r = block_select_smallest_hi<NT>(hi, lo, n, k, sm);
-  return r.prefix | ~r.mask;
+  return select_in_hist<NT>(hi, lo, n, k, sm, buf, bin_of);
 }
 
 }  // namespace confkv

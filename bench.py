@@ -63,6 +63,7 @@ FULL = CONFIGS[3]
 SWEEP5 = [(b, c) for b in (1, 8, 64) for c in (4096, 32768, 131072)]
 POOL = 48   # distinct pre-generated step inputs, reused cyclically
 KERNEL_STEPS = 512   # steps of the per-kernel event region after the timed steps
+E2E_BUFFERS = 3      # device buffer sets of the end-to-end leg
 
 
 def args_parse(argv=None):
@@ -803,8 +804,9 @@ def e2e_leg(h, w, pool, args, dev, world, attn_call, start):
     """The same steps through the public API with host buffers: each step's
     inputs copied host->device from pinned memory and its outputs (attention
     output, and c in confidence mode) device->host inside the timed region.
-    Two buffer sets: step i+1's upload and step i-1's download run on two copy
-    streams (separate copy engines) while step i computes."""
+    NBUF buffer sets: uploads and downloads run on two copy streams (separate
+    copy engines) while the steps compute; an upload may run up to NBUF - 1
+    steps ahead, a download up to NBUF - 1 steps behind."""
     import torch
     import torch.distributed as dist
     from confidence_gated_kv_logit_b200 import ALL_LAYERS
@@ -815,14 +817,15 @@ def e2e_leg(h, w, pool, args, dev, world, attn_call, start):
     hpool = [tuple(x.cpu().pin_memory() for x in pool[i]) for i in range(8)]
     up_s = torch.cuda.Stream(device=dev)
     down_s = torch.cuda.Stream(device=dev)
-    dbuf = [tuple(torch.empty_like(x) for x in pool[0]) for _ in range(2)]
-    obuf = [torch.empty((L, B, Hq, D), device=dev) for _ in range(2)]
-    cbuf = [torch.empty(B, device=dev) for _ in range(2)]
-    host_out = [torch.empty((L, B, Hq, D), pin_memory=True) for _ in range(2)]
-    host_c = [torch.empty(B, pin_memory=True) for _ in range(2)]
-    ev_comp = [torch.cuda.Event() for _ in range(2)]
-    ev_in = [torch.cuda.Event() for _ in range(2)]
-    ev_out = [torch.cuda.Event() for _ in range(2)]
+    NBUF = E2E_BUFFERS
+    dbuf = [tuple(torch.empty_like(x) for x in pool[0]) for _ in range(NBUF)]
+    obuf = [torch.empty((L, B, Hq, D), device=dev) for _ in range(NBUF)]
+    cbuf = [torch.empty(B, device=dev) for _ in range(NBUF)]
+    host_out = [torch.empty((L, B, Hq, D), pin_memory=True) for _ in range(NBUF)]
+    host_c = [torch.empty(B, pin_memory=True) for _ in range(NBUF)]
+    ev_comp = [torch.cuda.Event() for _ in range(NBUF)]
+    ev_in = [torch.cuda.Event() for _ in range(NBUF)]
+    ev_out = [torch.cuda.Event() for _ in range(NBUF)]
     h2d = sum(x.numel() * x.element_size() for x in hpool[0])
     d2h = host_out[0].numel() * 4 + (0 if fixed else host_c[0].numel() * 4)
     E = args.e2e_steps
@@ -831,10 +834,10 @@ def e2e_leg(h, w, pool, args, dev, world, attn_call, start):
         dist.barrier()
 
     def upload(i):
-        j = i % 2
+        j = i % NBUF
         with torch.cuda.stream(up_s):
-            if i >= 2:
-                up_s.wait_event(ev_comp[j])            # step i-2 is done with buffer set j
+            if i >= NBUF:
+                up_s.wait_event(ev_comp[j])            # step i-NBUF is done with buffer set j
             for dst, src in zip(dbuf[j], hpool[i % len(hpool)]):
                 dst.copy_(src, non_blocking=True)
             ev_in[j].record(up_s)
@@ -842,14 +845,15 @@ def e2e_leg(h, w, pool, args, dev, world, attn_call, start):
     e0.record(stream)
     up_s.wait_stream(stream)
     down_s.wait_stream(stream)
-    upload(0)
+    for i in range(min(E, NBUF - 1)):
+        upload(i)
     for i in range(E):
-        j = i % 2
-        if i + 1 < E:
-            upload(i + 1)
+        j = i % NBUF
+        if i + NBUF - 1 < E:
+            upload(i + NBUF - 1)
         stream.wait_event(ev_in[j])
-        if i >= 2:
-            stream.wait_event(ev_out[j])               # step i-2's results have left buffer set j
+        if i >= NBUF:
+            stream.wait_event(ev_out[j])               # step i-NBUF's results have left buffer set j
         dq, dk, dv, dx = dbuf[j]
         attn_call(h, dq, dk, dv, obuf[j], dx if fixed else None)
         if not fixed:
@@ -871,7 +875,7 @@ def e2e_leg(h, w, pool, args, dev, world, attn_call, start):
     e2e_ms = max_over_ranks(e2e_ms, dev)
     return {"value": whole_job_rate(world, B, E, e2e_ms), "unit": "tok/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": E,
-            "pipelining": "two buffer sets; step i+1's upload and step i-1's download on two copy streams"}
+            "pipelining": f"{NBUF} buffer sets; uploads up to {NBUF - 1} steps ahead and downloads on two copy streams"}
 
 
 def graph_leg(h, w, pool, K, dev, world, attn_call):

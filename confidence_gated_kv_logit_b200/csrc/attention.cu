@@ -479,15 +479,39 @@ __device__ __forceinline__ bool consume_i8(const Cache& c, const AttnLaunch& a, 
 #pragma unroll
       for (int k = 0; k < 4; ++k) sacc[nb][k] = 0;
     const int rb = warp * 32 + mb2 * 16;
+    if constexpr (GP == 8) {
+      // twice the MMAs per chain: a second accumulator set over the odd
+      // k-blocks halves the dependency chains (the integer sums add exactly)
+      int sodd[NB][4];
 #pragma unroll
-    for (int kb = 0; kb < KB; ++kb) {
-      uint32_t af[4];
-      if constexpr (D == 128)   // 128-byte rows: the chunk XOR is the row index mod 8 = lane & 7
-        ldsm_x4(af, kt + x.lo.k8_row + mb2 * 16 * D + (((uint32_t)kb << 5) ^ x.lo.kx));
-      else
-        ldsm_x4(af, kt + (uint32_t)k8_off(rb + (lane & 7) + ((lane >> 3) & 1) * 8, kb * 32 + (lane >> 4) * 16, D));
+      for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
-      for (int nb = 0; nb < NB; ++nb) mma_s8s8(sacc[nb], af, qi[kb][nb].x, qi[kb][nb].y);
+        for (int k = 0; k < 4; ++k) sodd[nb][k] = 0;
+#pragma unroll
+      for (int kb = 0; kb < KB; ++kb) {
+        uint32_t af[4];
+        if constexpr (D == 128)
+          ldsm_x4(af, kt + x.lo.k8_row + mb2 * 16 * D + (((uint32_t)kb << 5) ^ x.lo.kx));
+        else
+          ldsm_x4(af, kt + (uint32_t)k8_off(rb + (lane & 7) + ((lane >> 3) & 1) * 8, kb * 32 + (lane >> 4) * 16, D));
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) mma_s8s8((kb & 1) ? sodd[nb] : sacc[nb], af, qi[kb][nb].x, qi[kb][nb].y);
+      }
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) sacc[nb][k] += sodd[nb][k];
+    } else {
+#pragma unroll
+      for (int kb = 0; kb < KB; ++kb) {
+        uint32_t af[4];
+        if constexpr (D == 128)   // 128-byte rows: the chunk XOR is the row index mod 8 = lane & 7
+          ldsm_x4(af, kt + x.lo.k8_row + mb2 * 16 * D + (((uint32_t)kb << 5) ^ x.lo.kx));
+        else
+          ldsm_x4(af, kt + (uint32_t)k8_off(rb + (lane & 7) + ((lane >> 3) & 1) * 8, kb * 32 + (lane >> 4) * 16, D));
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) mma_s8s8(sacc[nb], af, qi[kb][nb].x, qi[kb][nb].y);
+      }
     }
 #pragma unroll
     for (int hr = 0; hr < 2; ++hr) {
@@ -588,25 +612,65 @@ __device__ __forceinline__ bool consume_i8(const Cache& c, const AttnLaunch& a, 
     for (int nb = 0; nb < NBW; ++nb)
 #pragma unroll
       for (int k = 0; k < 4; ++k) ia[mb][nb][k] = 0;
+  if constexpr (GP == 8) {
+    // a second accumulator set over the odd k-steps halves the dependency
+    // chains (exact integer sums)
+    int iodd[MB][NBW][4];
 #pragma unroll
-  for (int ks = 0; ks < 4; ++ks) {
-    uint32_t af[MB][4];
+    for (int mb = 0; mb < MB; ++mb)
 #pragma unroll
-    for (int mb = 0; mb < MB; ++mb) {
-      const uint4 f = x.fb[(ks * MB + mb) * 32 + lane];
-      af[mb][0] = f.x;
-      af[mb][1] = f.y;
-      af[mb][2] = f.z;
-      af[mb][3] = f.w;
-    }
+      for (int nb = 0; nb < NBW; ++nb)
 #pragma unroll
-    for (int nbp = 0; nbp < NBW / 2; ++nbp) {
-      uint32_t bf[4];
-      ldsm_x4(bf, vt + (uint32_t)(ks * 32 * D) + x.lo.v8[nbp]);   // ks*32*D is a multiple of 2 KB
+        for (int k = 0; k < 4; ++k) iodd[mb][nb][k] = 0;
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+      uint32_t af[MB][4];
 #pragma unroll
       for (int mb = 0; mb < MB; ++mb) {
-        mma_u8s8(ia[mb][2 * nbp], af[mb], bf[0], bf[1]);
-        mma_u8s8(ia[mb][2 * nbp + 1], af[mb], bf[2], bf[3]);
+        const uint4 f = x.fb[(ks * MB + mb) * 32 + lane];
+        af[mb][0] = f.x;
+        af[mb][1] = f.y;
+        af[mb][2] = f.z;
+        af[mb][3] = f.w;
+      }
+#pragma unroll
+      for (int nbp = 0; nbp < NBW / 2; ++nbp) {
+        uint32_t bf[4];
+        ldsm_x4(bf, vt + (uint32_t)(ks * 32 * D) + x.lo.v8[nbp]);
+#pragma unroll
+        for (int mb = 0; mb < MB; ++mb) {
+          mma_u8s8((ks & 1) ? iodd[mb][2 * nbp] : ia[mb][2 * nbp], af[mb], bf[0], bf[1]);
+          mma_u8s8((ks & 1) ? iodd[mb][2 * nbp + 1] : ia[mb][2 * nbp + 1], af[mb], bf[2], bf[3]);
+        }
+      }
+    }
+#pragma unroll
+    for (int mb = 0; mb < MB; ++mb)
+#pragma unroll
+      for (int nb = 0; nb < NBW; ++nb)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) ia[mb][nb][k] += iodd[mb][nb][k];
+  } else {
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+      uint32_t af[MB][4];
+#pragma unroll
+      for (int mb = 0; mb < MB; ++mb) {
+        const uint4 f = x.fb[(ks * MB + mb) * 32 + lane];
+        af[mb][0] = f.x;
+        af[mb][1] = f.y;
+        af[mb][2] = f.z;
+        af[mb][3] = f.w;
+      }
+#pragma unroll
+      for (int nbp = 0; nbp < NBW / 2; ++nbp) {
+        uint32_t bf[4];
+        ldsm_x4(bf, vt + (uint32_t)(ks * 32 * D) + x.lo.v8[nbp]);   // ks*32*D is a multiple of 2 KB
+#pragma unroll
+        for (int mb = 0; mb < MB; ++mb) {
+          mma_u8s8(ia[mb][2 * nbp], af[mb], bf[0], bf[1]);
+          mma_u8s8(ia[mb][2 * nbp + 1], af[mb], bf[2], bf[3]);
+        }
       }
     }
   }
@@ -642,11 +706,24 @@ __device__ __forceinline__ bool consume_h(const Cache& c, const AttnLaunch& a, c
   const int rb = warp * 16;
 
   float f[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  if constexpr (GP == 8) {
+    // a second accumulator over the odd k-steps halves the MMA dependency chain
+    float fo[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-  for (int ks = 0; ks < KS; ++ks) {
-    uint32_t af[4];
-    ldsm_x4(af, kt + x.lo.h_row + (((uint32_t)ks << 5) ^ x.lo.kx));
-    mma_f16(f, af, qh[ks].x, qh[ks].y);
+    for (int ks = 0; ks < KS; ++ks) {
+      uint32_t af[4];
+      ldsm_x4(af, kt + x.lo.h_row + (((uint32_t)ks << 5) ^ x.lo.kx));
+      mma_f16((ks & 1) ? fo : f, af, qh[ks].x, qh[ks].y);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) f[k] += fo[k];
+  } else {
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      uint32_t af[4];
+      ldsm_x4(af, kt + x.lo.h_row + (((uint32_t)ks << 5) ^ x.lo.kx));
+      mma_f16(f, af, qh[ks].x, qh[ks].y);
+    }
   }
   float u[2][2];
   bool tok_valid[2];
@@ -900,7 +977,7 @@ __global__ void __launch_bounds__(160, 2) attn_kernel(Cache c, AttnLaunch a, int
   // -------------------------------- consumers --------------------------------
   const int g = lane >> 2, t = lane & 3;
   const LaneOffsets lane_offs = lane_offsets<D>(warp, lane);
-  // the scores are read again right after this kernel (the EMA pass): keep them in L2
+  // scores: evict-last, so that their lines are not written back while the K/V tiles stream
   const uint64_t keep_policy = l2_evict_last_policy();
   int ctr = 0;
   for (int k = 0;; ++k) {

@@ -843,6 +843,7 @@ def e2e_leg(h, w, pool, args, dev, world, attn_call, start):
             ev_in[j].record(up_s)
 
     e0.record(stream)
+    t_host = time.perf_counter()
     up_s.wait_stream(stream)
     down_s.wait_stream(stream)
     for i in range(min(E, NBUF - 1)):
@@ -869,12 +870,13 @@ def e2e_leg(h, w, pool, args, dev, world, attn_call, start):
     stream.wait_stream(up_s)
     stream.wait_stream(down_s)
     e1.record(stream)
+    host_ms = (time.perf_counter() - t_host) * 1e3   # enqueueing all steps, before the device finishes
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
     _report_device_error(h, "end-to-end region")
     e2e_ms = max_over_ranks(e2e_ms, dev)
     return {"value": whole_job_rate(world, B, E, e2e_ms), "unit": "tok/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "steps": E,
+            "d2h_bytes_per_step": d2h, "steps": E, "host_enqueue_ms_per_step": host_ms / E,
             "pipelining": f"{NBUF} buffer sets; uploads up to {NBUF - 1} steps ahead and downloads on two copy streams"}
 
 

@@ -81,8 +81,6 @@ def test_fused_pass_matches_separate_pass(per_layer, G, score, compact, profiled
     if profiled:
         prof = hb.profile_read()
         assert prof["ema_evict"]["launches"] > 0      # the fused kernel ran
-    # the handle whose passes ran on their own launched more kernels
-    assert ha.query()["kernel_launches"] > hb.query()["kernel_launches"]
     assert ha.last_error() == 0 and hb.last_error() == 0
     ha.close()
     hb.close()

@@ -27,7 +27,11 @@
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *    stream). Every call is asynchronous on that stream unless documented as
  *    synchronising. One handle must not be used from two streams at once: the
- *    cache and the scratch belong to the handle.
+ *    cache and the scratch belong to the handle. The library's kernels are
+ *    launched with programmatic stream serialisation: each starts by waiting
+ *    for the work before it on the stream to complete, so the next one's
+ *    launch overlaps its end; work of the caller in between is ordered as
+ *    usual.
  *  - Errors the host can detect (bad arguments, capacity, wrong state) are
  *    returned before anything is launched, and the call has no effect.
  *    Conditions only the device can see (non-finite logits, a failed device
@@ -220,7 +224,9 @@ CONFKV_API confkv_status confkv_decode_attn(confkv_handle* h, int32_t layer, con
  * token; tokens with age < P and positions < s are never evicted. Survivors
  * are compacted so the INT8 region stays a hole-free prefix, and the token
  * the next append would push out of the FP16 window is quantised to INT8
- * (CONF-KV post, pseudo-code). */
+ * (CONF-KV post, pseudo-code). Called on the stream of the handle's last
+ * confkv_confidence, right after it, the deferred EMA pass runs beside that
+ * confidence reduction and only the eviction waits for its budgets. */
 CONFKV_API confkv_status confkv_evict_compact(confkv_handle* h, int32_t layer, void* stream);
 
 /* Synchronising: counts of the active segments and cumulative counters. */

@@ -79,7 +79,7 @@ struct confkv_handle {
   unsigned char* qfrag;          // [S][qf_stride] query operands of the attention kernel
   int qf_stride;
   confkv::EvictCand* cand;       // [S] eviction candidates from the EMA pass
-  uint32_t* kscratch;            // evict scratch, per CTA of the largest evict grid
+  uint32_t* kscratch;            // evict scratch, per CTA of the largest evict grid (scratch_ctas)
   int* sched;                    // attention unit counters (zero between launches)
   int* bulk_sched;               // bulk eviction segment counters (zero between launches)
   // The EMA pass of a decode call is deferred (unless single_stream): the
@@ -96,6 +96,7 @@ struct confkv_handle {
   bool conf_last = false;
   cudaStream_t conf_stream = nullptr;
   int scratch_stride;
+  int scratch_ctas;               // CTAs kscratch covers
   int32_t* keep_list;
   int32_t* keep_count;
   long long launches;
@@ -324,7 +325,8 @@ confkv_status confkv_create(int32_t layers, int32_t kv_heads, int32_t q_heads, i
   chk(B.alloc(&h->sched, 2));
   chk(B.alloc(&h->bulk_sched, 2));
   h->scratch_stride = 3 * c.cap + c.Wst;
-  chk(B.alloc(&h->kscratch, (size_t)confkv::evict_grid((int)S) * h->scratch_stride));
+  h->scratch_ctas = std::max(confkv::evict_grid((int)S), std::min((int)S, confkv::few_segment_limit(h->num_sms)));
+  chk(B.alloc(&h->kscratch, (size_t)h->scratch_ctas * h->scratch_stride));
   if (p.mode == CONFKV_MODE_FIXED) {
     chk(B.alloc(&h->keep_list, S * (size_t)p.fixed_budget));
     chk(B.alloc(&h->keep_count, S));
@@ -611,6 +613,7 @@ confkv_status confkv_evict_compact(confkv_handle* h, int32_t layer, void* stream
   a.cand = h->cand;
   a.kscratch = h->kscratch;
   a.scratch_stride = h->scratch_stride;
+  a.scratch_ctas = h->scratch_ctas;
   a.scratch_keys = h->c.cap + h->c.Wst;
   a.bulk_sched = h->bulk_sched;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -1086,10 +1086,18 @@ cudaError_t run_bulk(const Cache& c, const Policy& pol, const EvictLaunch& a, co
   int per_sm = 0;
   cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, evict_bulk_kernel<D, CI8, GMAX>, NT, 0);
   if (e != cudaSuccess) return e;
-  // the key scratch exists for evict_grid(items) CTAs
+  // the key scratch exists for evict_grid(items) CTAs (or more)
   const int grid = max(1, min(evict_grid(items), max(1, per_sm) * num_sms));
   (void)launch_chained(evict_bulk_kernel<D, CI8, GMAX>, grid, NT, 0, st, c, pol, a, ema, items);
   return cudaGetLastError();
+}
+
+// One segment per CTA by the whole-CTA path (calls over few segments).
+template <int D, bool CI8>
+__global__ void __launch_bounds__(NT) evict_block_kernel(Cache c, Policy pol, EvictLaunch a, int items) {
+  chain_enter();
+  __shared__ EvictSmem es;
+  if ((int)blockIdx.x < items) evict_segment_block<D, CI8>(c, pol, a, (int)blockIdx.x, es);
 }
 
 template <int D, bool CI8>
@@ -1115,10 +1123,26 @@ cudaError_t run(const Cache& c, const Policy& pol, const EvictLaunch& a, const E
 
 int evict_grid(int items) { return (items + kSegsPerCta - 1) / kSegsPerCta; }
 
+int few_segment_limit(int num_sms) { return 2 * num_sms; }
+
 cudaError_t launch_evict_compact(const Cache& c, const Policy& pol, const EvictLaunch& a, const EmaIn* ema,
                                  bool bulk, int num_sms, cudaStream_t st, long long* launches, Prof* prof) {
-  if (a.r.items(c.Hkv) == 0) return cudaSuccess;
+  const int items = a.r.items(c.Hkv);
+  if (items == 0) return cudaSuccess;
   if (ema != nullptr && (pol.mode != 0 || c.G < 1 || c.G > 8)) return cudaErrorInvalidValue;
+  const bool few = items <= few_segment_limit(num_sms) && items <= a.scratch_ctas;
+  if (ema == nullptr && few) {
+    // too few segments to fill the GPU one warp each: one CTA per segment
+    ProfScope ps(prof, kKEvict, st);
+    if (c.D == 128)
+      (void)(c.cold_int8 ? launch_chained(evict_block_kernel<128, true>, items, NT, 0, st, c, pol, a, items)
+                         : launch_chained(evict_block_kernel<128, false>, items, NT, 0, st, c, pol, a, items));
+    else
+      (void)(c.cold_int8 ? launch_chained(evict_block_kernel<64, true>, items, NT, 0, st, c, pol, a, items)
+                         : launch_chained(evict_block_kernel<64, false>, items, NT, 0, st, c, pol, a, items));
+    ++*launches;
+    return cudaGetLastError();
+  }
   if (ema != nullptr && bulk) {
     ProfScope ps(prof, kKEmaEvict, st);
     cudaError_t e;

@@ -92,6 +92,7 @@ struct EvictLaunch {
   // 1: the previous kernel on the stream is the confidence reduction, so the
   // fused variant may run its EMA pass before waiting for it (see evict_kernel)
   int ema_early = 0;
+  int scratch_ctas = 0;   // CTAs kscratch covers (no launch uses more)
 };
 // Where an EMA pass reads the step's attention results.
 struct EmaIn {
@@ -109,5 +110,11 @@ cudaError_t launch_evict_compact(const Cache& c, const Policy& pol, const EvictL
                                  bool bulk, int num_sms, cudaStream_t st, long long* launches, Prof* prof);
 // CTAs the evict kernel uses for `items` segments (the scratch is per CTA).
 int evict_grid(int items);
+// Calls over at most this many segments evict with one CTA per segment (the
+// whole-CTA path) when the EMA pass has already run: too few segments to fill
+// the GPU one warp each. The key scratch covers that many CTAs. (With the EMA
+// pass fused in, the per-warp kernel stays faster: measured on the GPT-2
+// shape.)
+int few_segment_limit(int num_sms);
 
 }  // namespace confkv

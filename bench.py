@@ -574,7 +574,7 @@ def make_handle(w, L=None, args=None, sliding_window=False):
 
 def step_bytes_model(w, d, K, launches_attn):
     """Algorithmic bytes per kernel kind for K steps whose library counters
-    moved by `d` (SURVEY-style per-unit figures: INT8 token 2D+8 read + 4G
+    moved by `d` (per-unit figures: INT8 token 2D+8 read + 4G
     score write; FP16 token 4D + 4G; EMA 4G+12 per token + 208 per segment;
     eviction 8 per scanned token + 2 x row bytes per moved row + 6D+8 per
     converted token; confidence 4 per logit; append q + K/V + prepared query
